@@ -1,0 +1,68 @@
+"""Test-side helpers: lay logical token data out in a block pool, dtype views.
+
+The pool layout is [num_blocks, Hkv, block_size, D]; token t of a sequence
+whose block table is ``table`` lives at pool[table[t // bs], :, t % bs, :].
+This is the layout definition written as a scatter, independently of the
+oracle's gather.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def place_logical(logical_k, logical_v, tables, num_blocks, block_size, fill=0.0):
+    """logical_k[b]: array [L_b, Hkv, D] -> (k_pool, v_pool) float32 arrays.
+
+    tables[b] lists the physical blocks of sequence b in logical order.
+    Slots that hold no token are set to ``fill``.
+    """
+    Hkv, D = None, None
+    for lk in logical_k:
+        if len(lk):
+            Hkv, D = lk.shape[1], lk.shape[2]
+            break
+    assert Hkv is not None
+    k_pool = np.full((num_blocks, Hkv, block_size, D), fill, np.float32)
+    v_pool = np.full((num_blocks, Hkv, block_size, D), fill, np.float32)
+    for b, (lk, lv) in enumerate(zip(logical_k, logical_v)):
+        for t in range(len(lk)):
+            phys = tables[b][t // block_size]
+            off = t % block_size
+            for h in range(Hkv):
+                k_pool[phys, h, off, :] = lk[t, h, :]
+                v_pool[phys, h, off, :] = lv[t, h, :]
+    return k_pool, v_pool
+
+
+def pad_tables(tables, width, pad=-1):
+    """List of per-sequence block lists -> int32 [B, width], padded with ``pad``."""
+    out = np.full((len(tables), max(width, 1)), pad, np.int32)
+    for b, row in enumerate(tables):
+        out[b, : len(row)] = row
+    return out
+
+
+def random_tables(rng, lengths, block_size, num_blocks):
+    """Scatter every sequence's logical blocks over distinct random physical ids."""
+    need = [-(-L // block_size) for L in lengths]
+    assert sum(need) <= num_blocks
+    ids = rng.permutation(num_blocks)
+    tables, at = [], 0
+    for n in need:
+        tables.append([int(x) for x in ids[at: at + n]])
+        at += n
+    return tables
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 to bfloat16 bits via torch (round to nearest even)."""
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def to_logical_lists(arr_list):
+    """[array [L, Hkv, D]] -> nested python lists for the brute force."""
+    return [[[list(map(float, arr[t, h])) for h in range(arr.shape[1])] for t in range(arr.shape[0])]
+            for arr in arr_list]
