@@ -1,0 +1,464 @@
+"""Benchmark of the paged decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one decode step of one attention layer over one batch: the new
+token's slot (pa_decode_slot_mapping), its K/V write (pa_reshape_and_cache),
+copy-on-write copies when the workload has them (pa_copy_blocks), and paged
+decode attention over every sequence (pa_paged_attention_decode, pass 1 plus
+the split-KV merge when a sequence is split).  Inputs are seeded synthetic
+tensors shaped like the named workload, resident in HBM before timing.
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
+on the launching stream, with a 256 MiB write between steps (outside the
+events) to flush the 126 MB L2; the region is bracketed by a barrier and
+torch.cuda.synchronize(); the reported time is the max over ranks.
+
+value  = K/V bytes attention reads (tokens < length, K and V) / step time,
+         summed over ranks (each rank runs its own batch: weak scaling, no
+         data-path collective).
+e2e    = the same metric through the public API with the step's inputs in
+         pinned host memory: H2D of q, new K/V, block tables and lengths, the
+         step, and D2H of the output, all inside the timed events.
+roofline = the decode call alone (pass 1 + merge) against the measured HBM
+         copy bandwidth.
+
+--impl reference times the CPU oracle (fp64, OpenMP) on the host cores on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Paged decode attn: achieved HBM GB/s vs peak; decode tokens/s per batch"
+FALLBACK_HBM_GBS = 6650.0
+FLUSH_BYTES = 256 << 20
+
+DESCRIPTIONS = {
+    "tiny": "tiny: batch 4, lengths 1,7,16,33 (+1 appended), 4/4 heads, head_dim 64, block_size 16, fp32",
+    "llama7b": "Llama-7B-shaped decode: batch 64, 32 q = 32 kv heads, head_dim 128, block_size 16, bf16, "
+               "lengths U[128, 2048], blocks drawn without replacement from a 1.25x pool",
+    "gqa": "GQA decode: batch 256, 32 q / 8 kv heads, head_dim 128, block_size 16, bf16, lengths lognormal "
+           "(median 1000, sigma 0.8) clipped to [16, 4096], blocks scattered",
+    "cow": "shared-prefix parallel sampling: 32 prompts x 8 samples, 32/8 heads, head_dim 128, bf16, block_size 16, "
+           "1000-token prompt shared (refcount 8), partial block copied by copy_blocks, 0-512 generated tokens",
+    "long16": "long-context split-KV decode: batch 16, 64 q / 8 kv heads, head_dim 128, bf16, block_size 16, "
+              "lengths U[32768, 131072], pool 1.1x",
+    "long32": "long-context split-KV decode: batch 16, 64 q / 8 kv heads, head_dim 128, bf16, block_size 32, "
+              "lengths U[32768, 131072], pool 1.1x",
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="llama7b", choices=sorted(DESCRIPTIONS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--partition", type=int, default=0, help="tokens per KV split (0 = automatic)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def dram_traffic(workload: str):
+    """Per-launch DRAM bytes of the decode kernel from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    src = os.path.join(ROOT, "paged_kv_cache_355_b200", "csrc", "pa_decode.cu")
+    try:
+        rec = json.load(open(path))
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        entry = rec.get(workload)
+        if entry and entry.get("kernel_source_sha256") == sha:
+            return int(entry["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples (SM clock, throttle reasons) while the region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[3:]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for _, _, flags in rows:
+            for n, f in zip(names, flags[1:]):
+                if f.lower() == "active":
+                    reasons.add(n)
+        loaded = [r[0] for r in rows if r[0] > 0.5 * r[1]] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and --impl reference)
+# ---------------------------------------------------------------------------
+def oracle_sample(case, max_seqs: int):
+    """Host arrays of the first `max_seqs` sequences of a case (a bounded
+    sample of the same workload) for the oracle."""
+    import numpy as np
+
+    def bits(t):
+        t = t.detach().cpu().contiguous()
+        return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+
+    n = min(max_seqs, case.workload.batch)
+    sel = (case.new_seq_ids < n).numpy()
+    return dict(q=bits(case.q[:n]), k_new=bits(case.k_new)[sel], v_new=bits(case.v_new)[sel],
+                sid=case.new_seq_ids.numpy()[sel], pos=case.new_positions.numpy()[sel],
+                bt=case.block_tables[:n].numpy(), lens=case.lengths[:n].numpy(),
+                k_pool=bits(case.k_pool).copy(), v_pool=bits(case.v_pool).copy(),
+                pairs=case.cow_pairs.numpy(), bytes=int(case.lengths[:n].sum()) * case.workload.num_kv_heads
+                * case.workload.head_dim * case.k_pool.element_size() * 2, seqs=n)
+
+
+def oracle_step(s, scale, bs):
+    import oracle
+
+    if len(s["pairs"]):
+        oracle.copy_blocks(s["k_pool"], s["v_pool"], s["pairs"])
+    slots = oracle.slot_mapping(s["bt"], s["sid"], s["pos"], bs)
+    oracle.reshape_and_cache(s["k_new"], s["v_new"], s["k_pool"], s["v_pool"], slots)
+    return oracle.paged_decode(s["q"], s["k_pool"], s["v_pool"], s["bt"], s["lens"], scale, bs)
+
+
+def time_oracle(case, min_seconds=10.0, max_reps=3, max_seqs=None):
+    import oracle
+
+    n = max_seqs or case.workload.batch
+    s = oracle_sample(case, n)
+    reps, t_total = 0, 0.0
+    while reps < max_reps and (reps == 0 or t_total < min_seconds):
+        t0 = time.perf_counter()
+        oracle_step(s, case.scale, case.workload.block_size)
+        t_total += time.perf_counter() - t0
+        reps += 1
+    sec = t_total / reps
+    return {"value": s["bytes"] / sec / 1e9, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{s['seqs']} of {case.workload.batch} sequences of the same workload, one full decode step "
+                      f"(slot mapping, cache write, attention) per repetition, {reps} repetition(s), "
+                      f"{sec:.2f} s each", "seconds_per_step": sec}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from paged_kv_cache_355_b200.workloads import make_case
+
+    import oracle
+
+    case = make_case(args.workload, device="cpu")
+    w = case.workload
+    # each step: the oracle over a bounded sample of the workload's sequences
+    seqs = {"tiny": 4, "llama7b": 8, "gqa": 16, "cow": 16, "long16": 1, "long32": 1}[args.workload]
+    s = oracle_sample(case, seqs)
+    for _ in range(args.warmup):
+        oracle_step(s, case.scale, w.block_size)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_step(s, case.scale, w.block_size)
+        times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    value = s["bytes"] / sec / 1e9
+    sample = (f"{s['seqs']} of {w.batch} sequences of the workload per step (slot mapping, cache write, attention), "
+              f"fp64 oracle")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": DESCRIPTIONS[args.workload], "sample_sequences": s["seqs"]},
+            "tokens_per_s": s["seqs"] / sec,
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    world, rank, local = dist_setup(args.gpus)
+    import paged_kv_cache_355_b200 as pa
+    from paged_kv_cache_355_b200.workloads import SEEDS, make_case
+
+    dev = torch.device("cuda", local)
+    case = make_case(args.workload, device=dev, seed=SEEDS[args.workload] + 101 * rank)
+    w = case.workload
+    B, Hq, Hkv, D, bs = w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size
+    stream = torch.cuda.current_stream()
+    bt = case.block_tables.to(dev)
+    lens = case.lengths.to(dev)
+    max_len = case.max_len
+    kv_bytes = case.kv_bytes()
+    out = torch.empty(B, Hq, D, dtype=torch.float32, device=dev)
+    slots = torch.empty(case.new_seq_ids.numel(), dtype=torch.int64, device=dev)
+    sid, pos = case.new_seq_ids.to(dev), case.new_positions.to(dev)
+    pairs = case.cow_pairs.to(dev)
+    part = args.partition or pa.pa_paged_attention_partition_size(B, Hq, Hkv, D, max_len, bs)
+    ws_bytes = pa.pa_paged_attention_workspace_size(B, Hq, Hkv, D, max_len, bs, part)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    plain_decode = pairs.numel() == 0 and case.new_seq_ids.numel() == B
+
+    def cache_part():
+        if pairs.numel():
+            pa.pa_copy_blocks(case.k_pool, case.v_pool, pairs)
+        if plain_decode:
+            pa.pa_decode_slot_mapping(bt, lens, bs, slots)
+        else:
+            pa.pa_slot_mapping(bt, sid, pos, bs, slots)
+        pa.pa_reshape_and_cache(case.k_new, case.v_new, case.k_pool, case.v_pool, slots)
+
+    def decode_part():
+        pa.pa_paged_attention_decode(case.q, case.k_pool, case.v_pool, bt, lens, max_len, case.scale, out,
+                                     partition_size=part, workspace=ws)
+
+    max_splits = -(-max(max_len, 1) // part)
+    launches_per_step = (1 if pairs.numel() else 0) + 2 + 1 + (1 if max_splits > 1 else 0)
+
+    # ---- device-resident timed region
+    for _ in range(args.warmup):
+        flush.zero_()
+        cache_part()
+        decode_part()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    barrier(world)
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        torch.cuda.synchronize()
+        barrier(world)
+        t_wall = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            cache_part()
+            ev[i][1].record(stream)
+            decode_part()
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        t_wall = time.perf_counter() - t_wall
+    step_ms = [a.elapsed_time(c) for a, _, c in ev]
+    dec_ms = [b_.elapsed_time(c) for _, b_, c in ev]
+    ms_step = max_over_ranks(sum(step_ms) / len(step_ms), world)
+    ms_dec = max_over_ranks(sum(dec_ms) / len(dec_ms), world)
+    assert pa.pa_read_error_flag() == 0, "device error during the timed steps"
+
+    # ---- contiguous-cache variant of the same kernel on the same lengths (paging overhead)
+    L_pad = -(-max_len // 32) * 32
+    k_c = torch.empty(B, Hkv, L_pad, D, dtype=w.dtype, device=dev).normal_()
+    v_c = torch.empty_like(k_c).normal_()
+    out_c = torch.empty_like(out)
+    contig_ms = []
+    for i in range(args.warmup + min(args.steps, 200)):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        pa.pa_paged_attention_decode_contiguous(case.q, k_c, v_c, lens, max_len, case.scale, out_c, block_size=bs,
+                                                partition_size=part, workspace=ws)
+        e1.record(stream)
+        if i >= args.warmup:
+            contig_ms.append((e0, e1))
+    torch.cuda.synchronize()
+    ms_contig = max_over_ranks(sum(a.elapsed_time(b_) for a, b_ in contig_ms) / len(contig_ms), world)
+    paged_med = statistics.median(dec_ms)
+    contig_med = statistics.median(a.elapsed_time(b_) for a, b_ in contig_ms)
+    del k_c, v_c
+
+    # ---- end to end through the public API with host buffers
+    pin = lambda t: t.detach().to("cpu").pin_memory()
+    h_q, h_kn, h_vn = pin(case.q), pin(case.k_new), pin(case.v_new)
+    h_bt, h_lens = pin(case.block_tables), pin(case.lengths)
+    h_out = torch.empty(B, Hq, D, dtype=torch.float32).pin_memory()
+    d_q, d_kn, d_vn = torch.empty_like(case.q), torch.empty_like(case.k_new), torch.empty_like(case.v_new)
+    d_bt, d_lens = torch.empty_like(bt), torch.empty_like(lens)
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_kn, h_vn, h_bt, h_lens))
+    d2h = h_out.numel() * h_out.element_size()
+    e2e_ev = []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for dst, src in ((d_q, h_q), (d_kn, h_kn), (d_vn, h_vn), (d_bt, h_bt), (d_lens, h_lens)):
+            dst.copy_(src, non_blocking=True)
+        if plain_decode:
+            pa.decode_step(d_q, d_kn, d_vn, case.k_pool, case.v_pool, d_bt, d_lens, max_len, case.scale, out, slots,
+                           workspace=ws, partition_size=part)
+        else:
+            if pairs.numel():
+                pa.pa_copy_blocks(case.k_pool, case.v_pool, pairs)
+            pa.pa_slot_mapping(d_bt, sid, pos, bs, slots)
+            pa.pa_reshape_and_cache(d_kn, d_vn, case.k_pool, case.v_pool, slots)
+            pa.pa_paged_attention_decode(d_q, case.k_pool, case.v_pool, d_bt, d_lens, max_len, case.scale, out,
+                                         partition_size=part, workspace=ws)
+        h_out.copy_(out, non_blocking=True)
+        e1.record(stream)
+        if i >= args.warmup:
+            e2e_ev.append((e0, e1))
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(sum(a.elapsed_time(b_) for a, b_ in e2e_ev) / len(e2e_ev), world)
+
+    # ---- CPU oracle on this machine's host cores (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = time_oracle(case)
+
+    if rank != 0:
+        return
+    peak, peak_kind = measured_hbm_peak()
+    achieved = kv_bytes / (ms_dec * 1e-3) / 1e9
+    value = world * kv_bytes / (ms_step * 1e-3) / 1e9
+    traffic = dram_traffic(args.workload)
+    clk = clocks.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+        "config": {"workload": DESCRIPTIONS[args.workload], "batch_per_gpu": B, "partition_tokens": part,
+                   "max_splits": max_splits, "kv_bytes_per_step": kv_bytes,
+                   "l2": "flushed between steps by a 256 MiB write outside the timed events; "
+                         "K/V read per step also exceeds the 126 MB L2",
+                   "parallelism": f"{world} independent replicas (sequences sharded, no collective)"},
+        "tokens_per_s": world * B / (ms_step * 1e-3),
+        "decode_attention_ms": ms_dec,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "kernel": "pa_paged_attention_decode (pass 1 + split merge)",
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)"},
+        "paging_overhead": {"paged_ms_median": paged_med, "contiguous_ms_median": contig_med,
+                            "overhead": paged_med / contig_med - 1.0, "contiguous_ms_mean_max_ranks": ms_contig},
+        "e2e": {"value": world * kv_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+        "wall_s_timed_region": t_wall,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    run_ours(args)
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

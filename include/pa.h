@@ -1,0 +1,210 @@
+/*
+ * pa.h -- C ABI of libpa.so, the paged KV-cache decode path for NVIDIA B200
+ * (sm_100a).
+ *
+ * The pages this follows:
+ *   [P1] "PagedAttention and KV memory management" (guide.dupenodi.dev)
+ *   [P2] "Paged Attention: OS-Inspired Memory Management for KV Caches"
+ *        (Modern AI Engineering, lesson 13.6)
+ *   [P3] "How does vLLM PagedAttention manage Virtual Memory Pages to
+ *        eliminate KV cache fragmentation?" (iloveeagents.com)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  * Every array argument is a device pointer owned by the caller (for
+ *    example the storage of a contiguous torch tensor), 16-byte aligned, and
+ *    stays owned by the caller.  The library allocates no device memory and
+ *    keeps no state between calls other than one device-side error word per
+ *    device (see pa_read_error_flag).
+ *  * `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Every call only enqueues work on it and returns; a returned
+ *    PA_OK means the arguments passed host-side validation and the launches
+ *    were accepted, not that the kernels have finished.
+ *  * Element types: PA_F32 (IEEE fp32) or PA_BF16 (bfloat16).  Query, key
+ *    and value share one element type; all arithmetic accumulates in fp32.
+ *  * KV pool layout (the pages fix none; [P1] "The kernel side" only says
+ *    "a pool of blocks"): k_pool and v_pool are separate arrays, each
+ *    [num_blocks][num_kv_heads][block_size][head_dim] row-major, so one
+ *    (block, kv head) tile is block_size * head_dim contiguous elements.
+ *  * A slot is block_id * block_size + offset: token position pos of a
+ *    sequence whose block table is `table` has slot
+ *    table[pos / block_size] * block_size + pos % block_size ([P3] "Detail",
+ *    virtual block i -> physical block table[i], one block of block_size
+ *    tokens allocated at a time).
+ *  * Grouped query heads: query head h reads kv head h / (Hq / Hkv).
+ *  * Supported shapes: head_dim in {64, 128}; block_size in {8, 16, 32};
+ *    Hq % Hkv == 0 with Hq / Hkv in {1, 2, 4, 8}.  Anything else returns
+ *    PA_ERR_UNSUPPORTED without launching.
+ *  * Device-side checks: a block id outside [0, num_blocks), a negative or
+ *    too-long context length, or a slot outside the pool is never
+ *    dereferenced.  The kernel skips it and records the first such error in
+ *    the device error word (PA_ERR_BAD_BLOCK_ID), which pa_read_error_flag
+ *    returns; outputs that depended on it are unspecified.  No kernel traps.
+ *  * Every wait inside a kernel is bounded in time; a wait that runs out
+ *    records PA_ERR_TIMEOUT in the error word and the kernel returns.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,  /* null pointer, negative size, misaligned pointer, bad enum */
+    PA_ERR_UNSUPPORTED = 2,  /* valid but unsupported head_dim / block_size / group size */
+    PA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required */
+    PA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+    PA_ERR_BAD_BLOCK_ID = 5, /* device side: block id / slot / length outside its range */
+    PA_ERR_TIMEOUT = 6       /* device side: a bounded wait ran out */
+} pa_status;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* pa_status_string(int status);
+
+/* Library version as "major.minor.patch" (static storage). */
+const char* pa_version(void);
+
+/*
+ * pa_read_error_flag -- synchronise `stream`, then return the first
+ * device-side error recorded by any kernel of this library on the current
+ * device since the previous call (PA_OK if none), and clear it.  Returns
+ * PA_ERR_CUDA if the synchronisation itself fails.
+ */
+int pa_read_error_flag(void* stream);
+
+/*
+ * pa_slot_mapping -- slot of each new token ([P3] "Detail": logical block
+ * pos / block_size of the sequence maps to the physical block its table
+ * names; the token sits at offset pos % block_size inside it).
+ *   block_tables      int32 [batch][max_blocks_per_seq]
+ *   seq_ids           int32 [num_tokens]  sequence of token i
+ *   positions         int32 [num_tokens]  0-based position of token i
+ *   slot_mapping      int64 [num_tokens]  output
+ * A token whose sequence id or position is out of range, or whose table
+ * entry is negative, gets slot -1 (reshape_and_cache then skips it) and
+ * records PA_ERR_BAD_BLOCK_ID.
+ */
+int pa_slot_mapping(const int32_t* block_tables, int max_blocks_per_seq, int batch,
+                    const int32_t* seq_ids, const int32_t* positions, int64_t num_tokens,
+                    int block_size, int64_t* slot_mapping, void* stream);
+
+/*
+ * pa_decode_slot_mapping -- the decode-step special case of pa_slot_mapping:
+ * token b is the last token (position context_lens[b] - 1) of sequence b.
+ * A sequence of length 0 gets slot -1 (nothing to write).
+ *   context_lens int32 [batch] (lengths INCLUDING the token being written)
+ *   slot_mapping int64 [batch] output
+ */
+int pa_decode_slot_mapping(const int32_t* block_tables, int max_blocks_per_seq,
+                           const int32_t* context_lens, int batch, int block_size,
+                           int64_t* slot_mapping, void* stream);
+
+/*
+ * pa_reshape_and_cache -- write each new token's K and V into its slot:
+ *   k_pool[s / bs][h][s % bs][:] = key[i][h][:]  and the same for value,
+ * for every token i with s = slot_mapping[i] >= 0 ([P3] "Key Technical
+ * Innovations" item 2: blocks fill one token at a time as generation
+ * proceeds).  Bit-exact copy.
+ *   key, value    [num_tokens][num_kv_heads][head_dim]   (dtype)
+ *   k_pool,v_pool [num_blocks][num_kv_heads][block_size][head_dim] (dtype), updated in place
+ *   slot_mapping  int64 [num_tokens]; negative = skip.  Slots must be
+ *                 distinct within one call (caller's precondition).
+ */
+int pa_reshape_and_cache(const void* key, const void* value, void* k_pool, void* v_pool,
+                         const int64_t* slot_mapping, int64_t num_tokens, int num_kv_heads,
+                         int head_dim, int block_size, int64_t num_blocks, int dtype,
+                         void* stream);
+
+/*
+ * pa_copy_blocks -- copy-on-write duplication of shared blocks ([P2] "Key
+ * terms in this lesson", Copy-on-write: a block is shared until someone
+ * writes to it, and the writer then gets a private copy; [P1] "Myths and
+ * failure modes", parallel samples share their prompt this way).
+ * For every pair p: block block_mapping[p][1] := block block_mapping[p][0],
+ * whole K block and whole V block, bit-exact.
+ *   block_mapping int64 [num_pairs][2] as (src, dst).  Destinations must be
+ *                 distinct and no destination may also be a source in the
+ *                 same call (caller's precondition).  An id outside
+ *                 [0, num_blocks) skips the pair and records PA_ERR_BAD_BLOCK_ID.
+ */
+int pa_copy_blocks(void* k_pool, void* v_pool, const int64_t* block_mapping, int64_t num_pairs,
+                   int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, int dtype,
+                   void* stream);
+
+/*
+ * pa_paged_attention_partition_size -- tokens per KV split that
+ * pa_paged_attention_decode uses for these sizes when called with
+ * partition_size == 0 (a multiple of 32, at most 8192).  Sequences longer
+ * than it are processed as several splits merged by a second pass.
+ */
+int pa_paged_attention_partition_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                                      int max_context_len, int block_size, int* partition_size);
+
+/*
+ * pa_paged_attention_workspace_size -- bytes of scratch the decode call
+ * needs for the split-KV partial results (0 when no sequence can need more
+ * than one split).  partition_size: 0 = automatic, else a multiple of 32 in
+ * [32, 8192].
+ */
+int pa_paged_attention_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                                      int max_context_len, int block_size, int partition_size,
+                                      size_t* workspace_bytes);
+
+/*
+ * pa_paged_attention_decode -- single-query (decode) attention that reads
+ * every sequence's K and V straight from the block pool through its block
+ * table, with no gather into a contiguous buffer ([P1] "The kernel side":
+ * read the block table, load each physical block's K and V tiles in turn,
+ * compute scores and weighted values in place).  For each sequence b and
+ * query head h, with L = context_lens[b] and kv head g = h / (Hq / Hkv):
+ *   s_t = scale * <q[b][h], K_t>,  out[b][h] = sum_t softmax(s)_t * V_t,
+ * over the tokens t < L; L == 0 gives a zero row.  Softmax is evaluated
+ * online in fp32; sequences longer than the partition size are split and
+ * merged by a log-sum-exp second pass (deterministic, no atomics).
+ *   q             [batch][num_q_heads][head_dim] (kv_dtype)
+ *   k_pool,v_pool [num_blocks][num_kv_heads][block_size][head_dim] (kv_dtype)
+ *   block_tables  int32 [batch][max_blocks_per_seq]; only the first
+ *                 ceil(L / block_size) entries of a row are read
+ *   context_lens  int32 [batch]
+ *   max_context_len  host-side upper bound of context_lens (sizes the grid;
+ *                 must be <= max_blocks_per_seq * block_size)
+ *   out           [batch][num_q_heads][head_dim], out_dtype PA_F32 or PA_BF16
+ *   partition_size  0 = automatic (pa_paged_attention_partition_size)
+ *   workspace     device scratch of at least the size
+ *                 pa_paged_attention_workspace_size returns (NULL if 0)
+ */
+int pa_paged_attention_decode(const void* q, const void* k_pool, const void* v_pool,
+                              const int32_t* block_tables, int max_blocks_per_seq,
+                              const int32_t* context_lens, int max_context_len, float scale,
+                              int block_size, void* out, int out_dtype, int batch,
+                              int num_q_heads, int num_kv_heads, int head_dim,
+                              int64_t num_blocks, int kv_dtype, int partition_size,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * pa_paged_attention_decode_contiguous -- the same attention over a
+ * contiguous cache, the "ideal contiguous attention" [P1] "The kernel side"
+ * measures the paged kernel against.  Same kernel, same tiling and staging
+ * (tiles of block_size tokens), only the address of a tile differs:
+ *   k_c, v_c  [batch][num_kv_heads][L_pad][head_dim] (kv_dtype), L_pad >= max_context_len
+ */
+int pa_paged_attention_decode_contiguous(const void* q, const void* k_c, const void* v_c,
+                                         int64_t L_pad, const int32_t* context_lens,
+                                         int max_context_len, float scale, int block_size,
+                                         void* out, int out_dtype, int batch, int num_q_heads,
+                                         int num_kv_heads, int head_dim, int kv_dtype,
+                                         int partition_size, void* workspace,
+                                         size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

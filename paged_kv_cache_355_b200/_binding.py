@@ -1,0 +1,209 @@
+"""Thin ctypes binding of libpa.so.
+
+Every function here has the name of the C entry point it calls and only
+marshals arguments: it reads shapes, dtypes and device pointers off torch
+tensors, checks that they are CUDA tensors laid out as the C ABI expects,
+calls the library on the current (or given) stream, and raises PAError on a
+non-zero status.  All computation happens in the library's CUDA kernels;
+there is no other code path.  If libpa.so has not been built the import of
+this module fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpa.so")
+
+PA_F32, PA_BF16 = 0, 1
+_STATUS = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_WORKSPACE",
+           4: "PA_ERR_CUDA", 5: "PA_ERR_BAD_BLOCK_ID", 6: "PA_ERR_TIMEOUT"}
+_DTYPES = {torch.float32: PA_F32, torch.bfloat16: PA_BF16}
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_355_b200.build` "
+                      "(or __graft_entry__.build()); there is no fallback implementation")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_P, _I, _I64, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+_SIGS = {
+    "pa_status_string": ([_I], ctypes.c_char_p),
+    "pa_version": ([], ctypes.c_char_p),
+    "pa_read_error_flag": ([_P], _I),
+    "pa_slot_mapping": ([_P, _I, _I, _P, _P, _I64, _I, _P, _P], _I),
+    "pa_decode_slot_mapping": ([_P, _I, _P, _I, _I, _P, _P], _I),
+    "pa_reshape_and_cache": ([_P, _P, _P, _P, _P, _I64, _I, _I, _I, _I64, _I, _P], _I),
+    "pa_copy_blocks": ([_P, _P, _P, _I64, _I, _I, _I, _I64, _I, _P], _I),
+    "pa_paged_attention_partition_size": ([_I, _I, _I, _I, _I, _I, ctypes.POINTER(_I)], _I),
+    "pa_paged_attention_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
+    "pa_paged_attention_decode": ([_P, _P, _P, _P, _I, _P, _I, _F, _I, _P, _I, _I, _I, _I, _I, _I64, _I, _I, _P,
+                                   _SZ, _P], _I),
+    "pa_paged_attention_decode_contiguous": ([_P, _P, _P, _I64, _P, _I, _F, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P,
+                                              _SZ, _P], _I),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = _res
+
+EXPORTED = tuple(_SIGS)
+
+
+class PAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {_STATUS.get(status, status)}")
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise PAError(fn, status)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _kv_dtype(t: torch.Tensor) -> int:
+    if t.dtype not in _DTYPES:
+        raise TypeError(f"unsupported element type {t.dtype}: use float32 or bfloat16")
+    return _DTYPES[t.dtype]
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def pa_status_string(status: int) -> str:
+    return _lib.pa_status_string(status).decode()
+
+
+def pa_version() -> str:
+    return _lib.pa_version().decode()
+
+
+def pa_read_error_flag(stream=None) -> int:
+    """Synchronise the stream and return (then clear) the device error word."""
+    return int(_lib.pa_read_error_flag(_stream(stream)))
+
+
+def pa_slot_mapping(block_tables, seq_ids, positions, block_size: int, slot_mapping, stream=None) -> None:
+    B, MBS = block_tables.shape
+    n = seq_ids.numel()
+    _check("pa_slot_mapping", _lib.pa_slot_mapping(
+        _dev(block_tables, "block_tables", torch.int32), MBS, B, _dev(seq_ids, "seq_ids", torch.int32),
+        _dev(positions, "positions", torch.int32), n, block_size, _dev(slot_mapping, "slot_mapping", torch.int64),
+        _stream(stream)))
+
+
+def pa_decode_slot_mapping(block_tables, context_lens, block_size: int, slot_mapping, stream=None) -> None:
+    B, MBS = block_tables.shape
+    _check("pa_decode_slot_mapping", _lib.pa_decode_slot_mapping(
+        _dev(block_tables, "block_tables", torch.int32), MBS, _dev(context_lens, "context_lens", torch.int32), B,
+        block_size, _dev(slot_mapping, "slot_mapping", torch.int64), _stream(stream)))
+
+
+def pa_reshape_and_cache(key, value, k_pool, v_pool, slot_mapping, stream=None) -> None:
+    T, Hkv, D = key.shape
+    NB, Hkv2, bs, D2 = k_pool.shape
+    if (Hkv2, D2) != (Hkv, D) or value.shape != key.shape or v_pool.shape != k_pool.shape:
+        raise ValueError("key/value and pool shapes disagree")
+    dt = _kv_dtype(key)
+    for t, n in ((value, "value"), (k_pool, "k_pool"), (v_pool, "v_pool")):
+        _dev(t, n, key.dtype)
+    _check("pa_reshape_and_cache", _lib.pa_reshape_and_cache(
+        _dev(key, "key"), value.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
+        _dev(slot_mapping, "slot_mapping", torch.int64), T, Hkv, D, bs, NB, dt, _stream(stream)))
+
+
+def pa_copy_blocks(k_pool, v_pool, block_mapping, stream=None) -> None:
+    NB, Hkv, bs, D = k_pool.shape
+    _dev(v_pool, "v_pool", k_pool.dtype)
+    P = block_mapping.numel() // 2
+    _check("pa_copy_blocks", _lib.pa_copy_blocks(
+        _dev(k_pool, "k_pool"), v_pool.data_ptr(), _dev(block_mapping, "block_mapping", torch.int64), P, Hkv, D, bs,
+        NB, _kv_dtype(k_pool), _stream(stream)))
+
+
+def pa_paged_attention_partition_size(batch, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                                      block_size) -> int:
+    out = _I(0)
+    _check("pa_paged_attention_partition_size", _lib.pa_paged_attention_partition_size(
+        batch, num_q_heads, num_kv_heads, head_dim, max_context_len, block_size, ctypes.byref(out)))
+    return out.value
+
+
+def pa_paged_attention_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, block_size,
+                                      partition_size: int = 0) -> int:
+    out = _SZ(0)
+    _check("pa_paged_attention_workspace_size", _lib.pa_paged_attention_workspace_size(
+        batch, num_q_heads, num_kv_heads, head_dim, max_context_len, block_size, partition_size, ctypes.byref(out)))
+    return out.value
+
+
+def _workspace(workspace, nbytes: int, device, stream) -> tuple[int, int]:
+    """Device pointer and size of the split-KV scratch.
+
+    If the caller gives none, one is taken from torch's caching allocator and
+    tied to the stream the kernels run on, so it is not reused before they
+    finish.  Callers that launch on a raw stream handle should pass their own.
+    """
+    if workspace is None:
+        if nbytes == 0:
+            return 0, 0
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        if isinstance(stream, torch.cuda.Stream):
+            workspace.record_stream(stream)
+    _dev(workspace, "workspace")
+    return workspace.data_ptr(), workspace.numel() * workspace.element_size()
+
+
+def pa_paged_attention_decode(q, k_pool, v_pool, block_tables, context_lens, max_context_len: int, scale: float,
+                              out, partition_size: int = 0, workspace=None, stream=None) -> None:
+    """out[b, h] = softmax(scale * q[b, h] . K_b^T) V_b over the paged cache."""
+    B, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_pool.shape
+    if D2 != D or v_pool.shape != k_pool.shape or tuple(out.shape) != (B, Hq, D):
+        raise ValueError("q / pool / out shapes disagree")
+    MBS = block_tables.shape[1]
+    dt = _kv_dtype(q)
+    _dev(k_pool, "k_pool", q.dtype)
+    _dev(v_pool, "v_pool", q.dtype)
+    need = pa_paged_attention_workspace_size(B, Hq, Hkv, D, max_context_len, bs, partition_size)
+    ws, ws_bytes = _workspace(workspace, need, q.device, stream)
+    _check("pa_paged_attention_decode", _lib.pa_paged_attention_decode(
+        _dev(q, "q"), k_pool.data_ptr(), v_pool.data_ptr(), _dev(block_tables, "block_tables", torch.int32), MBS,
+        _dev(context_lens, "context_lens", torch.int32), int(max_context_len), float(scale), bs, _dev(out, "out"),
+        _kv_dtype(out), B, Hq, Hkv, D, NB, dt, partition_size, ws, ws_bytes, _stream(stream)))
+
+
+def pa_paged_attention_decode_contiguous(q, k_c, v_c, context_lens, max_context_len: int, scale: float, out,
+                                         block_size: int = 16, partition_size: int = 0, workspace=None,
+                                         stream=None) -> None:
+    """The same attention over a contiguous cache k_c, v_c: [B, Hkv, L_pad, D]."""
+    B, Hq, D = q.shape
+    B2, Hkv, L_pad, D2 = k_c.shape
+    if B2 != B or D2 != D or v_c.shape != k_c.shape or tuple(out.shape) != (B, Hq, D):
+        raise ValueError("q / cache / out shapes disagree")
+    dt = _kv_dtype(q)
+    _dev(k_c, "k_c", q.dtype)
+    _dev(v_c, "v_c", q.dtype)
+    need = pa_paged_attention_workspace_size(B, Hq, Hkv, D, max_context_len, block_size, partition_size)
+    ws, ws_bytes = _workspace(workspace, need, q.device, stream)
+    _check("pa_paged_attention_decode_contiguous", _lib.pa_paged_attention_decode_contiguous(
+        _dev(q, "q"), k_c.data_ptr(), v_c.data_ptr(), L_pad, _dev(context_lens, "context_lens", torch.int32),
+        int(max_context_len), float(scale), block_size, _dev(out, "out"), _kv_dtype(out), B, Hq, Hkv, D, dt,
+        partition_size, ws, ws_bytes, _stream(stream)))

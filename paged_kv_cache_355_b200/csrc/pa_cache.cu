@@ -1,0 +1,193 @@
+// pa_cache.cu -- the kernels that feed the KV pool: slot mapping,
+// reshape_and_cache (write a new token's K/V into its slot) and copy_blocks
+// (copy-on-write duplication of a shared block).
+//
+// All three are bit copies or integer index work, bound by latency (tiny
+// per-step sizes) or by HBM bandwidth (copy_blocks).  Each moves 16-byte
+// vectors: one (token, kv head) row of head_dim elements is head_dim *
+// elt / 16 vectors (8 to 32), contiguous in both source and destination.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pa.h"
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+namespace {
+
+constexpr int kThreads = 256;
+
+// slot of (sequence seq_ids[i], position positions[i]); -1 if unmappable.
+// "How does vLLM PagedAttention manage Virtual Memory Pages ...", "Detail":
+// virtual block pos / bs -> physical block table[pos / bs], offset pos % bs.
+__global__ void slot_mapping_kernel(const int32_t* __restrict__ block_tables, int max_blocks_per_seq, int batch,
+                                    const int32_t* __restrict__ seq_ids, const int32_t* __restrict__ positions,
+                                    int64_t num_tokens, int block_size, int64_t* __restrict__ slots, int* err) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < num_tokens;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int b = seq_ids[i];
+        const int pos = positions[i];
+        int64_t slot = -1;
+        if (b >= 0 && b < batch && pos >= 0 && pos / block_size < max_blocks_per_seq) {
+            const int32_t phys = block_tables[(int64_t)b * max_blocks_per_seq + pos / block_size];
+            if (phys >= 0) slot = (int64_t)phys * block_size + pos % block_size;
+        }
+        if (slot < 0) record_error(err, PA_ERR_BAD_BLOCK_ID);
+        slots[i] = slot;
+    }
+}
+
+// decode step: token b is position context_lens[b] - 1 of sequence b.
+__global__ void decode_slot_mapping_kernel(const int32_t* __restrict__ block_tables, int max_blocks_per_seq,
+                                           const int32_t* __restrict__ context_lens, int batch, int block_size,
+                                           int64_t* __restrict__ slots, int* err) {
+    for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < batch; b += gridDim.x * blockDim.x) {
+        const int L = context_lens[b];
+        int64_t slot = -1;
+        if (L > 0) {
+            const int pos = L - 1;
+            if (pos / block_size < max_blocks_per_seq) {
+                const int32_t phys = block_tables[(int64_t)b * max_blocks_per_seq + pos / block_size];
+                if (phys >= 0) slot = (int64_t)phys * block_size + pos % block_size;
+            }
+            if (slot < 0) record_error(err, PA_ERR_BAD_BLOCK_ID);
+        } else if (L < 0) {
+            record_error(err, PA_ERR_BAD_BLOCK_ID);
+        }
+        slots[b] = slot;
+    }
+}
+
+// One thread per 16-byte vector of one (token, kv head) row, for K and V.
+__global__ void reshape_and_cache_kernel(const uint4* __restrict__ key, const uint4* __restrict__ value,
+                                         uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
+                                         const int64_t* __restrict__ slots, int64_t num_tokens, int num_kv_heads,
+                                         int row_vecs, int block_size, int64_t num_blocks, int* err) {
+    const int64_t per_token = (int64_t)num_kv_heads * row_vecs;
+    const int64_t total = num_tokens * per_token;
+    for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t tok = idx / per_token;
+        const int64_t rem = idx - tok * per_token;
+        const int64_t slot = slots[tok];
+        if (slot < 0) continue;
+        const int64_t blk = slot / block_size;
+        if (blk >= num_blocks) {
+            if (rem == 0) record_error(err, PA_ERR_BAD_BLOCK_ID);
+            continue;
+        }
+        const int h = (int)(rem / row_vecs);
+        const int c = (int)(rem - (int64_t)h * row_vecs);
+        const int64_t off = slot - blk * block_size;
+        const int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * row_vecs + c;
+        k_pool[dst] = key[idx];
+        v_pool[dst] = value[idx];
+    }
+}
+
+// blockIdx.x = pair; blockIdx.y strides over the block's 16-byte vectors.
+__global__ void copy_blocks_kernel(uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
+                                   const int64_t* __restrict__ block_mapping, int64_t num_blocks,
+                                   int64_t block_vecs, int* err) {
+    const int64_t p = blockIdx.x;
+    const int64_t src = block_mapping[2 * p];
+    const int64_t dst = block_mapping[2 * p + 1];
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+        if (threadIdx.x == 0 && blockIdx.y == 0) record_error(err, PA_ERR_BAD_BLOCK_ID);
+        return;
+    }
+    const uint4* ks = k_pool + src * block_vecs;
+    const uint4* vs = v_pool + src * block_vecs;
+    uint4* kd = k_pool + dst * block_vecs;
+    uint4* vd = v_pool + dst * block_vecs;
+    for (int64_t i = blockIdx.y * (int64_t)blockDim.x + threadIdx.x; i < block_vecs;
+         i += (int64_t)gridDim.y * blockDim.x) {
+        const uint4 a = ks[i];
+        const uint4 b = vs[i];
+        kd[i] = a;
+        vd[i] = b;
+    }
+}
+
+inline int grid_for(int64_t work) {
+    int64_t blocks = (work + kThreads - 1) / kThreads;
+    const int64_t cap = (int64_t)num_sms() * 16;
+    if (blocks > cap) blocks = cap;
+    return (int)(blocks < 1 ? 1 : blocks);
+}
+
+}  // namespace
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" int pa_slot_mapping(const int32_t* block_tables, int max_blocks_per_seq, int batch,
+                               const int32_t* seq_ids, const int32_t* positions, int64_t num_tokens,
+                               int block_size, int64_t* slot_mapping, void* stream) {
+    if (num_tokens < 0 || batch < 0 || max_blocks_per_seq < 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PA_OK;
+    if (!block_tables || !seq_ids || !positions || !slot_mapping) return PA_ERR_INVALID_ARG;
+    int* err = error_word_ptr();
+    if (!err) return PA_ERR_CUDA;
+    slot_mapping_kernel<<<grid_for(num_tokens), kThreads, 0, (cudaStream_t)stream>>>(
+        block_tables, max_blocks_per_seq, batch, seq_ids, positions, num_tokens, block_size, slot_mapping, err);
+    return launch_status();
+}
+
+extern "C" int pa_decode_slot_mapping(const int32_t* block_tables, int max_blocks_per_seq,
+                                      const int32_t* context_lens, int batch, int block_size,
+                                      int64_t* slot_mapping, void* stream) {
+    if (batch < 0 || max_blocks_per_seq < 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
+    if (batch == 0) return PA_OK;
+    if (!block_tables || !context_lens || !slot_mapping) return PA_ERR_INVALID_ARG;
+    int* err = error_word_ptr();
+    if (!err) return PA_ERR_CUDA;
+    decode_slot_mapping_kernel<<<grid_for(batch), kThreads, 0, (cudaStream_t)stream>>>(
+        block_tables, max_blocks_per_seq, context_lens, batch, block_size, slot_mapping, err);
+    return launch_status();
+}
+
+extern "C" int pa_reshape_and_cache(const void* key, const void* value, void* k_pool, void* v_pool,
+                                    const int64_t* slot_mapping, int64_t num_tokens, int num_kv_heads,
+                                    int head_dim, int block_size, int64_t num_blocks, int dtype,
+                                    void* stream) {
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks < 0 ||
+        !valid_dtype(dtype))
+        return PA_ERR_INVALID_ARG;
+    if (!supported_head_dim(head_dim) || !supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return PA_OK;
+    if (!key || !value || !k_pool || !v_pool || !slot_mapping) return PA_ERR_INVALID_ARG;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(k_pool) || !aligned16(v_pool))
+        return PA_ERR_INVALID_ARG;
+    int* err = error_word_ptr();
+    if (!err) return PA_ERR_CUDA;
+    const int row_vecs = (int)(head_dim * dtype_bytes(dtype) / 16);
+    reshape_and_cache_kernel<<<grid_for(num_tokens * num_kv_heads * row_vecs), kThreads, 0,
+                               (cudaStream_t)stream>>>(
+        static_cast<const uint4*>(key), static_cast<const uint4*>(value), static_cast<uint4*>(k_pool),
+        static_cast<uint4*>(v_pool), slot_mapping, num_tokens, num_kv_heads, row_vecs, block_size, num_blocks, err);
+    return launch_status();
+}
+
+extern "C" int pa_copy_blocks(void* k_pool, void* v_pool, const int64_t* block_mapping, int64_t num_pairs,
+                              int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, int dtype,
+                              void* stream) {
+    if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks < 0 ||
+        !valid_dtype(dtype))
+        return PA_ERR_INVALID_ARG;
+    if (!supported_head_dim(head_dim) || !supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
+    if (num_pairs == 0) return PA_OK;
+    if (num_pairs > 0x7fffffff) return PA_ERR_INVALID_ARG;
+    if (!k_pool || !v_pool || !block_mapping || !aligned16(k_pool) || !aligned16(v_pool)) return PA_ERR_INVALID_ARG;
+    int* err = error_word_ptr();
+    if (!err) return PA_ERR_CUDA;
+    const int64_t block_vecs = (int64_t)num_kv_heads * block_size * head_dim * (int64_t)dtype_bytes(dtype) / 16;
+    int64_t slices = (block_vecs + kThreads * 4 - 1) / (kThreads * 4);
+    if (slices > 64) slices = 64;
+    if (slices < 1) slices = 1;
+    dim3 grid((unsigned)num_pairs, (unsigned)slices);
+    copy_blocks_kernel<<<grid, kThreads, 0, (cudaStream_t)stream>>>(
+        static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), block_mapping, num_blocks, block_vecs, err);
+    return launch_status();
+}

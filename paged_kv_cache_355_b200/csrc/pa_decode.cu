@@ -1,0 +1,682 @@
+// pa_decode.cu -- paged decode attention for sm_100a.
+//
+// What it computes ("PagedAttention and KV memory management", section "The
+// kernel side"): for each sequence, read its block table, load each physical
+// block's K and V tiles in turn, and compute scores and weighted values in
+// place, without first gathering the sequence into one buffer.
+//
+// Design (one GPU, HBM-bound: every K/V byte is read exactly once):
+//  * Work item = (split, kv head, sequence), one CTA each.  A split is a run
+//    of `partition` tokens (a multiple of 32); sequences longer than that are
+//    cut into several splits whose partial results a second kernel merges
+//    with a log-sum-exp rescale.  Split boundaries depend only on logical
+//    token positions, so the result is independent of where the blocks sit
+//    in the pool and bit-identical from run to run (no atomics).
+//  * Warp 0 is the producer: its lane 0 reads the CTA's slice of the block
+//    table (staged once into shared memory) and streams K and V tiles with
+//    bulk copies (cp.async.bulk, the TMA engine) into a ring of `stages`
+//    shared-memory stages, each holding 32 tokens of K and 32 of V.  A stage
+//    gathers 32 / block_size physical blocks into one contiguous 32-token
+//    tile, so the math never depends on block_size.  Full/empty mbarriers
+//    hand stages to the consumers and back.
+//  * Warps 1..4 are consumers.  Stage j goes to consumer warp j % 4, which
+//    keeps its own fp32 online-softmax state (running max m, running sum l,
+//    output accumulator o) for all G = Hq / Hkv query heads of the kv head:
+//    every K and V element loaded from shared memory is used by all G heads.
+//    Inside a warp, a group of TPT lanes owns one token row (16 bytes per
+//    lane), so K/V shared-memory reads are conflict-free row segments; the
+//    q.k partial sums are reduced across the TPT lanes with shuffles, and the
+//    32 / TPT groups of a warp are independent softmax states.
+//  * At the end the groups and the warps are merged (shuffles, then shared
+//    memory), and the CTA writes either the final row (one split) or its
+//    normalised partial row plus (m, l) for the merge kernel.
+//  * Scores are kept in the log2 domain: q is pre-multiplied by
+//    scale * log2(e) and exp2f is used throughout.
+//  * Tokens past the sequence end are masked to -inf and their V rows are
+//    never multiplied (stale shared memory may hold anything, NaN included).
+//
+// The contiguous-cache variant is the same kernel: only the producer's source
+// address differs (one bulk copy per 32-token stage instead of one per block).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "pa.h"
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+namespace {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kDecodeThreads = 32 * (1 + kConsumerWarps);
+constexpr int kStageTokens = 32;
+constexpr int kMaxPartition = 8192;
+constexpr int kMinAutoPartition = 512;
+constexpr int kRingTargetBytes = 64 * 1024;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct DecodeParams {
+    const void* q;
+    const void* k;  // pool [NB, Hkv, bs, D] or contiguous cache [B, Hkv, L_pad, D]
+    const void* v;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    void* out;
+    float* part_o;   // [B, Hq, max_splits, D]
+    float* part_ml;  // [B, Hq, max_splits, 2] = (m in log2 units, l)
+    int* err;
+    int64_t num_blocks;
+    int64_t L_pad;
+    int64_t max_len;  // max_context_len: longer sequences are clamped and flagged
+    int max_blocks_per_seq;
+    int num_q_heads;
+    int num_kv_heads;
+    int block_size;
+    int partition;
+    int max_splits;
+    int stages;
+    int ring_offset;
+    int out_bf16;
+    int contiguous;
+    float scale_log2;
+};
+
+template <typename T>
+struct Elt;
+
+template <>
+struct Elt<float> {
+    static constexpr int VEC = 4;  // elements per 16-byte lane vector
+    __device__ __forceinline__ static void unpack(const uint4& r, float* f) {
+        f[0] = __uint_as_float(r.x);
+        f[1] = __uint_as_float(r.y);
+        f[2] = __uint_as_float(r.z);
+        f[3] = __uint_as_float(r.w);
+    }
+};
+
+template <>
+struct Elt<__nv_bfloat16> {
+    static constexpr int VEC = 8;
+    __device__ __forceinline__ static void unpack(const uint4& r, float* f) {
+        // bf16 -> fp32 is exact: the 16 bits become the high half of the word.
+        f[0] = __uint_as_float(r.x << 16);
+        f[1] = __uint_as_float(r.x & 0xffff0000u);
+        f[2] = __uint_as_float(r.y << 16);
+        f[3] = __uint_as_float(r.y & 0xffff0000u);
+        f[4] = __uint_as_float(r.z << 16);
+        f[5] = __uint_as_float(r.z & 0xffff0000u);
+        f[6] = __uint_as_float(r.w << 16);
+        f[7] = __uint_as_float(r.w & 0xffff0000u);
+    }
+};
+
+__device__ __forceinline__ int clamp_len(const DecodeParams& p, int b, bool report) {
+    int L = p.context_lens[b];
+    if (L < 0 || (int64_t)L > p.max_len) {
+        if (report) record_error(p.err, PA_ERR_BAD_BLOCK_ID);
+        L = L < 0 ? 0 : (int)p.max_len;
+    }
+    return L;
+}
+
+__device__ __forceinline__ void store_out(const DecodeParams& p, int64_t idx, float v) {
+    if (p.out_bf16)
+        static_cast<__nv_bfloat16*>(p.out)[idx] = __float2bfloat16_rn(v);
+    else
+        static_cast<float*>(p.out)[idx] = v;
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const DecodeParams p) {
+    using E = Elt<T>;
+    constexpr int VEC = E::VEC;
+    constexpr int TPT = D / VEC;             // lanes per token row
+    constexpr int NG = 32 / TPT;             // token groups per warp
+    constexpr int PASSES = kStageTokens / NG;  // rows per lane per stage
+    constexpr int PCH = PASSES < 32 / G ? PASSES : 32 / G;  // rows per softmax update
+    constexpr int NCH = PASSES / PCH;
+    constexpr int ROW_BYTES = D * (int)sizeof(T);
+    constexpr int STAGE_BYTES = kStageTokens * ROW_BYTES;  // K (or V) part of one stage
+    static_assert(TPT >= 1 && TPT <= 32 && NG * TPT == 32, "lane layout");
+    static_assert(PASSES % PCH == 0, "chunking");
+
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + p.stages;
+    int32_t* tbl = reinterpret_cast<int32_t*>(empty + p.stages);
+    uint8_t* ring = smem + p.ring_offset;
+    __shared__ int s_abort;
+
+    const int split = blockIdx.x;
+    const int kvh = blockIdx.y;
+    const int b = blockIdx.z;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    const int L = clamp_len(p, b, threadIdx.x == 0 && split == 0 && kvh == 0);
+    const int tok_begin = split * p.partition;
+    if (split > 0 && tok_begin >= L) return;  // uniform over the CTA, before any barrier
+    const int ntok = max(0, min(L, tok_begin + p.partition) - tok_begin);
+    const int nstage = (ntok + kStageTokens - 1) / kStageTokens;
+    const int num_splits_b = L > 0 ? (L + p.partition - 1) / p.partition : 1;
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        fence_barrier_init();
+    }
+    if (!p.contiguous) {
+        const int first_blk = tok_begin / p.block_size;
+        const int nblk = (ntok + p.block_size - 1) / p.block_size;
+        const int32_t* row = p.block_tables + (int64_t)b * p.max_blocks_per_seq + first_blk;
+        for (int i = threadIdx.x; i < nblk; i += blockDim.x) tbl[i] = row[i];
+    }
+    __syncthreads();
+
+    // per-consumer-lane softmax state (unused by the producer warp)
+    float o[G][VEC];
+    float m[G], l[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        m[h] = -INFINITY;
+        l[h] = 0.f;
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) o[h][v] = 0.f;
+    }
+    const int grp = lane / TPT;
+    const int sub = lane % TPT;
+
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        if (lane == 0) {
+            const uint64_t policy = l2_policy_evict_first();
+            const char* kbase = static_cast<const char*>(p.k);
+            const char* vbase = static_cast<const char*>(p.v);
+            const int bs = p.block_size;
+            for (int j = 0; j < nstage; ++j) {
+                const int slot = j % p.stages;
+                if (j >= p.stages && !mbar_wait(&empty[slot], ((j / p.stages) - 1) & 1, p.err)) {
+                    s_abort = 1;
+                    break;
+                }
+                uint8_t* kdst = ring + (size_t)slot * 2 * STAGE_BYTES;
+                uint8_t* vdst = kdst + STAGE_BYTES;
+                const int t0 = j * kStageTokens;
+                const int rows = min(kStageTokens, ntok - t0);
+                if (p.contiguous) {
+                    const int64_t off =
+                        (((int64_t)b * p.num_kv_heads + kvh) * p.L_pad + tok_begin + t0) * (int64_t)ROW_BYTES;
+                    const uint32_t bytes = (uint32_t)rows * ROW_BYTES;
+                    mbar_arrive_expect_tx(&full[slot], 2 * bytes);
+                    bulk_load(kdst, kbase + off, bytes, &full[slot], policy);
+                    bulk_load(vdst, vbase + off, bytes, &full[slot], policy);
+                } else {
+                    uint32_t bytes = 0;
+                    for (int r = 0; r < rows; r += bs) {
+                        const int32_t phys = tbl[(t0 + r) / bs];
+                        if (phys >= 0 && phys < p.num_blocks) bytes += (uint32_t)min(bs, rows - r) * ROW_BYTES;
+                    }
+                    mbar_arrive_expect_tx(&full[slot], 2 * bytes);
+                    for (int r = 0; r < rows; r += bs) {
+                        const int32_t phys = tbl[(t0 + r) / bs];
+                        if (phys < 0 || phys >= p.num_blocks) {
+                            record_error(p.err, PA_ERR_BAD_BLOCK_ID);
+                            continue;
+                        }
+                        const uint32_t nbytes = (uint32_t)min(bs, rows - r) * ROW_BYTES;
+                        const int64_t off = ((int64_t)phys * p.num_kv_heads + kvh) * bs * (int64_t)ROW_BYTES;
+                        bulk_load(kdst + r * ROW_BYTES, kbase + off, nbytes, &full[slot], policy);
+                        bulk_load(vdst + r * ROW_BYTES, vbase + off, nbytes, &full[slot], policy);
+                    }
+                }
+            }
+        }
+    } else {
+        // ---------------- consumers ----------------
+        const int cw = warp - 1;
+        float qf[G][VEC];
+        {
+            const T* qrow = static_cast<const T*>(p.q) + ((int64_t)b * p.num_q_heads + (int64_t)kvh * G) * D;
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const uint4 raw = *reinterpret_cast<const uint4*>(qrow + h * D + sub * VEC);
+                E::unpack(raw, qf[h]);
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) qf[h][v] *= p.scale_log2;
+            }
+        }
+        for (int j = cw; j < nstage; j += kConsumerWarps) {
+            const int slot = j % p.stages;
+            if (!mbar_wait(&full[slot], (j / p.stages) & 1, p.err)) {
+                s_abort = 1;
+                break;
+            }
+            const T* ks = reinterpret_cast<const T*>(ring + (size_t)slot * 2 * STAGE_BYTES);
+            const T* vs = ks + kStageTokens * D;
+            const int valid = min(kStageTokens, ntok - j * kStageTokens);
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
+                float s[PCH][G];
+#pragma unroll
+                for (int pp = 0; pp < PCH; ++pp) {
+                    const int t = (c * PCH + pp) * NG + grp;
+                    const uint4 raw = *reinterpret_cast<const uint4*>(ks + t * D + sub * VEC);
+                    float kf[VEC];
+                    E::unpack(raw, kf);
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        float acc = 0.f;
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v) acc = fmaf(qf[h][v], kf[v], acc);
+                        s[pp][h] = acc;
+                    }
+                }
+#pragma unroll
+                for (int off = TPT / 2; off >= 1; off >>= 1) {
+#pragma unroll
+                    for (int pp = 0; pp < PCH; ++pp)
+#pragma unroll
+                        for (int h = 0; h < G; ++h) s[pp][h] += __shfl_xor_sync(0xffffffffu, s[pp][h], off);
+                }
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    float mx = -INFINITY;
+#pragma unroll
+                    for (int pp = 0; pp < PCH; ++pp) {
+                        const int t = (c * PCH + pp) * NG + grp;
+                        if (t >= valid) s[pp][h] = -INFINITY;
+                        mx = fmaxf(mx, s[pp][h]);
+                    }
+                    const float m_new = fmaxf(m[h], mx);
+                    if (m_new == -INFINITY) {
+#pragma unroll
+                        for (int pp = 0; pp < PCH; ++pp) s[pp][h] = 0.f;
+                        continue;
+                    }
+                    const float alpha = exp2f(m[h] - m_new);
+                    m[h] = m_new;
+                    l[h] *= alpha;
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) o[h][v] *= alpha;
+#pragma unroll
+                    for (int pp = 0; pp < PCH; ++pp) {
+                        s[pp][h] = exp2f(s[pp][h] - m_new);
+                        l[h] += s[pp][h];
+                    }
+                }
+#pragma unroll
+                for (int pp = 0; pp < PCH; ++pp) {
+                    const int t = (c * PCH + pp) * NG + grp;
+                    if (t < valid) {
+                        const uint4 raw = *reinterpret_cast<const uint4*>(vs + t * D + sub * VEC);
+                        float vf[VEC];
+                        E::unpack(raw, vf);
+#pragma unroll
+                        for (int h = 0; h < G; ++h)
+#pragma unroll
+                            for (int v = 0; v < VEC; ++v) o[h][v] = fmaf(s[pp][h], vf[v], o[h][v]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
+        }
+        // merge the token groups of this warp
+#pragma unroll
+        for (int off = TPT; off < 32; off <<= 1) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float mo = __shfl_xor_sync(0xffffffffu, m[h], off);
+                const float lo = __shfl_xor_sync(0xffffffffu, l[h], off);
+                const float mn = fmaxf(m[h], mo);
+                const float a = m[h] == -INFINITY ? 0.f : exp2f(m[h] - mn);
+                const float a2 = mo == -INFINITY ? 0.f : exp2f(mo - mn);
+                l[h] = l[h] * a + lo * a2;
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, o[h][v], off);
+                    o[h][v] = o[h][v] * a + ov * a2;
+                }
+                m[h] = mn;
+            }
+        }
+    }
+    __syncthreads();  // pipeline drained: the ring is free for the merge scratch
+    if (s_abort) return;
+
+    float* sm_o = reinterpret_cast<float*>(ring);    // [4][G][D]
+    float* sm_m = sm_o + kConsumerWarps * G * D;      // [4][G]
+    float* sm_l = sm_m + kConsumerWarps * G;          // [4][G]
+    if (warp > 0 && grp == 0) {
+        const int cw = warp - 1;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) sm_o[(cw * G + h) * D + sub * VEC + v] = o[h][v];
+            if (sub == 0) {
+                sm_m[cw * G + h] = m[h];
+                sm_l[cw * G + h] = l[h];
+            }
+        }
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+        const int h = idx / D;
+        const int d = idx - h * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_m[w * G + h]);
+        float lt = 0.f, ot = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) {
+                const float mw = sm_m[w * G + h];
+                const float a = mw == -INFINITY ? 0.f : exp2f(mw - M);
+                lt += sm_l[w * G + h] * a;
+                ot += sm_o[(w * G + h) * D + d] * a;
+            }
+        }
+        const float val = lt > 0.f ? ot / lt : 0.f;
+        const int64_t qrow = (int64_t)b * p.num_q_heads + (int64_t)kvh * G + h;
+        if (num_splits_b == 1) {
+            store_out(p, qrow * D + d, val);
+        } else {
+            const int64_t r = qrow * p.max_splits + split;
+            p.part_o[r * D + d] = val;
+            if (d == 0) {
+                p.part_ml[2 * r] = M;
+                p.part_ml[2 * r + 1] = lt;
+            }
+        }
+    }
+}
+
+// Second pass: out = sum_s w_s o_s / sum_s w_s with w_s = l_s * 2^(m_s - max m),
+// for sequences that were cut into more than one split.  One CTA per
+// (sequence, query head), one thread per output element; fixed summation
+// order.
+template <int D>
+__global__ void __launch_bounds__(D) decode_merge_kernel(const DecodeParams p) {
+    extern __shared__ float wts[];  // [max_splits]
+    __shared__ float red[D / 32];
+    const int64_t row = blockIdx.x;  // b * Hq + h
+    const int b = (int)(row / p.num_q_heads);
+    const int L = clamp_len(p, b, false);
+    const int ns = L > 0 ? (L + p.partition - 1) / p.partition : 1;
+    if (ns <= 1) return;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const float* ml = p.part_ml + row * p.max_splits * 2;
+
+    float mx = -INFINITY;
+    for (int s = tid; s < ns; s += D) mx = fmaxf(mx, ml[2 * s]);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    if (lane == 0) red[warp] = mx;
+    __syncthreads();
+    float M = red[0];
+#pragma unroll
+    for (int w = 1; w < D / 32; ++w) M = fmaxf(M, red[w]);
+    __syncthreads();
+
+    float sum = 0.f;
+    for (int s = tid; s < ns; s += D) {
+        const float w = ml[2 * s + 1] * exp2f(ml[2 * s] - M);
+        wts[s] = w;
+        sum += w;
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane == 0) red[warp] = sum;
+    __syncthreads();
+    float W = 0.f;
+#pragma unroll
+    for (int w = 0; w < D / 32; ++w) W += red[w];
+
+    const float* po = p.part_o + row * p.max_splits * D;
+    float acc = 0.f;
+    for (int s = 0; s < ns; ++s) acc = fmaf(wts[s], po[(int64_t)s * D + tid], acc);
+    store_out(p, row * D + tid, W > 0.f ? acc / W : 0.f);
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+struct Plan {
+    int partition;
+    int max_splits;
+    size_t part_o_bytes;
+    size_t part_ml_bytes;
+    size_t workspace;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+int auto_partition(int batch, int num_kv_heads, int max_context_len) {
+    if (max_context_len <= 0) return kMinAutoPartition;
+    // About six work items per resident CTA slot (three CTAs per SM), assuming
+    // lengths spread evenly below max_context_len; long items are split so the
+    // tail of the grid stays short.
+    const double slots = (double)num_sms() * 3.0;
+    const double est_tokens = (double)batch * num_kv_heads * max_context_len * 0.5;
+    const double target = est_tokens / (slots * 6.0);
+    int P = kMinAutoPartition;
+    while (P < kMaxPartition && 2.0 * P <= target) P *= 2;
+    return P;
+}
+
+int make_plan(int batch, int num_q_heads, int num_kv_heads, int head_dim, int max_context_len, int partition_size,
+              Plan* plan) {
+    int P = partition_size;
+    if (P == 0) P = auto_partition(batch, num_kv_heads, max_context_len);
+    if (P < kStageTokens || P > kMaxPartition || P % kStageTokens != 0) return PA_ERR_INVALID_ARG;
+    const int L = max_context_len > 0 ? max_context_len : 1;
+    const int splits = (L + P - 1) / P;
+    plan->partition = P;
+    plan->max_splits = splits;
+    if (splits > 1) {
+        const size_t rows = (size_t)batch * num_q_heads * splits;
+        plan->part_o_bytes = align256(rows * head_dim * sizeof(float));
+        plan->part_ml_bytes = align256(rows * 2 * sizeof(float));
+    } else {
+        plan->part_o_bytes = plan->part_ml_bytes = 0;
+    }
+    plan->workspace = plan->part_o_bytes + plan->part_ml_bytes;
+    return PA_OK;
+}
+
+template <typename T, int D, int G>
+int launch_pass1(const DecodeParams& p, dim3 grid, size_t smem, cudaStream_t st) {
+    static std::atomic<unsigned long long> configured{0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(configured.load() & bit)) {
+        if (cudaFuncSetAttribute(decode_pass1_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 96 * 1024) != cudaSuccess)
+            return PA_ERR_CUDA;
+        configured.fetch_or(bit);
+    }
+    decode_pass1_kernel<T, D, G><<<grid, kDecodeThreads, smem, st>>>(p);
+    return launch_status();
+}
+
+template <typename T, int D>
+int dispatch_group(int G, const DecodeParams& p, dim3 grid, size_t smem, cudaStream_t st) {
+    switch (G) {
+        case 1: return launch_pass1<T, D, 1>(p, grid, smem, st);
+        case 2: return launch_pass1<T, D, 2>(p, grid, smem, st);
+        case 4: return launch_pass1<T, D, 4>(p, grid, smem, st);
+        case 8: return launch_pass1<T, D, 8>(p, grid, smem, st);
+        default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
+int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* workspace, size_t workspace_bytes,
+               int max_context_len, int partition_size, cudaStream_t st) {
+    const int G = p.num_q_heads / p.num_kv_heads;
+    Plan plan;
+    int rc = make_plan(batch, p.num_q_heads, p.num_kv_heads, head_dim, max_context_len, partition_size, &plan);
+    if (rc) return rc;
+    if (plan.workspace > 0) {
+        if (!workspace || workspace_bytes < plan.workspace || !aligned16(workspace)) return PA_ERR_WORKSPACE;
+        p.part_o = static_cast<float*>(workspace);
+        p.part_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + plan.part_o_bytes);
+    } else {
+        p.part_o = nullptr;
+        p.part_ml = nullptr;
+    }
+    p.partition = plan.partition;
+    p.max_splits = plan.max_splits;
+    p.err = error_word_ptr();
+    if (!p.err) return PA_ERR_CUDA;
+
+    const int stage_bytes = 2 * kStageTokens * head_dim * (int)dtype_bytes(kv_dtype);  // K + V
+    int stages = kRingTargetBytes / stage_bytes;
+    stages = stages < 2 ? 2 : (stages > 8 ? 8 : stages);
+    p.stages = stages;
+    const int table_bytes = p.contiguous ? 0 : (plan.partition / p.block_size) * 4;
+    p.ring_offset = (int)((16 * stages + table_bytes + 127) & ~127);
+    const size_t ring_bytes = (size_t)stages * stage_bytes;
+    const size_t merge_bytes = (size_t)kConsumerWarps * G * (head_dim + 2) * sizeof(float);
+    if (merge_bytes > ring_bytes) return PA_ERR_UNSUPPORTED;
+    const size_t smem = p.ring_offset + ring_bytes;
+
+    dim3 grid((unsigned)plan.max_splits, (unsigned)p.num_kv_heads, (unsigned)batch);
+    if (kv_dtype == PA_BF16) {
+        rc = head_dim == 128 ? dispatch_group<__nv_bfloat16, 128>(G, p, grid, smem, st)
+                             : dispatch_group<__nv_bfloat16, 64>(G, p, grid, smem, st);
+    } else {
+        rc = head_dim == 128 ? dispatch_group<float, 128>(G, p, grid, smem, st)
+                             : dispatch_group<float, 64>(G, p, grid, smem, st);
+    }
+    if (rc) return rc;
+    if (plan.max_splits > 1) {
+        const size_t msmem = (size_t)plan.max_splits * sizeof(float);
+        if (msmem > 48 * 1024) return PA_ERR_UNSUPPORTED;
+        const unsigned rows = (unsigned)((int64_t)batch * p.num_q_heads);
+        if (head_dim == 128)
+            decode_merge_kernel<128><<<rows, 128, msmem, st>>>(p);
+        else
+            decode_merge_kernel<64><<<rows, 64, msmem, st>>>(p);
+        rc = launch_status();
+    }
+    return rc;
+}
+
+int check_shapes(int batch, int num_q_heads, int num_kv_heads, int head_dim, int block_size, int kv_dtype,
+                 int out_dtype, int max_context_len) {
+    if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        max_context_len < 0 || !valid_dtype(kv_dtype) || !valid_dtype(out_dtype))
+        return PA_ERR_INVALID_ARG;
+    if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    if (!supported_head_dim(head_dim) || !supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
+    const int G = num_q_heads / num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
+    if (batch > 65535 || num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+    return PA_OK;
+}
+
+}  // namespace
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" int pa_paged_attention_partition_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                                                 int max_context_len, int block_size, int* partition_size) {
+    if (!partition_size) return PA_ERR_INVALID_ARG;
+    int rc = check_shapes(batch, num_q_heads, num_kv_heads, head_dim, block_size, PA_F32, PA_F32, max_context_len);
+    if (rc) return rc;
+    *partition_size = auto_partition(batch, num_kv_heads, max_context_len);
+    return PA_OK;
+}
+
+extern "C" int pa_paged_attention_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                                                 int max_context_len, int block_size, int partition_size,
+                                                 size_t* workspace_bytes) {
+    if (!workspace_bytes) return PA_ERR_INVALID_ARG;
+    int rc = check_shapes(batch, num_q_heads, num_kv_heads, head_dim, block_size, PA_F32, PA_F32, max_context_len);
+    if (rc) return rc;
+    Plan plan;
+    rc = make_plan(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, partition_size, &plan);
+    if (rc) return rc;
+    *workspace_bytes = plan.workspace;
+    return PA_OK;
+}
+
+extern "C" int pa_paged_attention_decode(const void* q, const void* k_pool, const void* v_pool,
+                                         const int32_t* block_tables, int max_blocks_per_seq,
+                                         const int32_t* context_lens, int max_context_len, float scale,
+                                         int block_size, void* out, int out_dtype, int batch, int num_q_heads,
+                                         int num_kv_heads, int head_dim, int64_t num_blocks, int kv_dtype,
+                                         int partition_size, void* workspace, size_t workspace_bytes,
+                                         void* stream) {
+    int rc = check_shapes(batch, num_q_heads, num_kv_heads, head_dim, block_size, kv_dtype, out_dtype,
+                          max_context_len);
+    if (rc) return rc;
+    if (max_blocks_per_seq < 0 || num_blocks < 0) return PA_ERR_INVALID_ARG;
+    if ((int64_t)max_context_len > (int64_t)max_blocks_per_seq * block_size) return PA_ERR_INVALID_ARG;
+    if (batch == 0) return PA_OK;
+    if (!q || !k_pool || !v_pool || !block_tables || !context_lens || !out) return PA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool)) return PA_ERR_INVALID_ARG;
+    DecodeParams p = {};
+    p.q = q;
+    p.k = k_pool;
+    p.v = v_pool;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.out = out;
+    p.num_blocks = num_blocks;
+    p.L_pad = 0;
+    p.max_len = max_context_len;  // validated <= max_blocks_per_seq * block_size
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.block_size = block_size;
+    p.out_bf16 = out_dtype == PA_BF16;
+    p.contiguous = 0;
+    p.scale_log2 = scale * kLog2e;
+    return run_decode(p, head_dim, kv_dtype, batch, workspace, workspace_bytes, max_context_len, partition_size,
+                      static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int pa_paged_attention_decode_contiguous(const void* q, const void* k_c, const void* v_c, int64_t L_pad,
+                                                    const int32_t* context_lens, int max_context_len, float scale,
+                                                    int block_size, void* out, int out_dtype, int batch,
+                                                    int num_q_heads, int num_kv_heads, int head_dim, int kv_dtype,
+                                                    int partition_size, void* workspace, size_t workspace_bytes,
+                                                    void* stream) {
+    int rc = check_shapes(batch, num_q_heads, num_kv_heads, head_dim, block_size, kv_dtype, out_dtype,
+                          max_context_len);
+    if (rc) return rc;
+    if (L_pad < 0 || (int64_t)max_context_len > L_pad) return PA_ERR_INVALID_ARG;
+    if (batch == 0) return PA_OK;
+    if (!q || !k_c || !v_c || !context_lens || !out) return PA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_c) || !aligned16(v_c)) return PA_ERR_INVALID_ARG;
+    DecodeParams p = {};
+    p.q = q;
+    p.k = k_c;
+    p.v = v_c;
+    p.block_tables = nullptr;
+    p.context_lens = context_lens;
+    p.out = out;
+    p.num_blocks = 0;
+    p.L_pad = L_pad;
+    p.max_len = max_context_len;  // validated <= L_pad
+    p.max_blocks_per_seq = 0;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.block_size = block_size;
+    p.out_bf16 = out_dtype == PA_BF16;
+    p.contiguous = 1;
+    p.scale_log2 = scale * kLog2e;
+    return run_decode(p, head_dim, kv_dtype, batch, workspace, workspace_bytes, max_context_len, partition_size,
+                      static_cast<cudaStream_t>(stream));
+}

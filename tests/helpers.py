@@ -66,3 +66,39 @@ def to_logical_lists(arr_list):
     """[array [L, Hkv, D]] -> nested python lists for the brute force."""
     return [[[list(map(float, arr[t, h])) for h in range(arr.shape[1])] for t in range(arr.shape[0])]
             for arr in arr_list]
+
+
+# ---------------------------------------------------------------------------
+# GPU-test helpers: hand tensors to the oracle, compare against it
+# ---------------------------------------------------------------------------
+def np_of(t):
+    """torch tensor (any device) -> numpy array in the oracle's conventions
+    (fp32 as float32, bf16 as its raw uint16 bits, integers as they are)."""
+    import torch
+
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.numpy()
+
+
+# Tolerances of paged decode attention against the fp64 oracle:
+# fp32 inputs: max |delta| <= 1e-5; bf16 inputs (fp32 accumulation):
+# max |delta| <= 2e-3 and every |delta| <= 2e-3 + 1e-2 * |oracle|.
+F32_ATOL = 1e-5
+BF16_ATOL, BF16_RTOL = 2e-3, 1e-2
+
+
+def assert_matches_oracle(got, ref, kv_is_bf16: bool, what: str = ""):
+    g = got.detach().float().cpu().double().numpy()
+    ref = np.asarray(ref, np.float64)
+    assert g.shape == ref.shape, (g.shape, ref.shape)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite output"
+    err = np.abs(g - ref)
+    if kv_is_bf16:
+        bad = err > BF16_ATOL + BF16_RTOL * np.abs(ref)
+        assert err.max() <= BF16_ATOL and not bad.any(), (
+            f"{what}: max|d|={err.max():.3e}, {int(bad.sum())} elements outside allclose(2e-3, 1e-2)")
+    else:
+        assert err.max() <= F32_ATOL, f"{what}: max|d|={err.max():.3e} > {F32_ATOL}"
+    return float(err.max())

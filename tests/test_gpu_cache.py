@@ -1,0 +1,118 @@
+"""GPU parity of the cache kernels: slot mapping, reshape_and_cache and
+copy_blocks must match the oracle bit for bit."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.helpers import np_of
+
+pytestmark = pytest.mark.gpu
+
+DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+@pytest.fixture(scope="module")
+def pa():
+    import paged_kv_cache_355_b200 as pa
+
+    assert torch.cuda.is_available()
+    pa.pa_read_error_flag()  # clear
+    return pa
+
+
+def test_slot_mapping_bit_exact(pa):
+    g = torch.Generator().manual_seed(5)
+    for bs in (8, 16, 32):
+        B, MBS = 37, 9
+        bt = torch.randperm(B * MBS + 11, generator=g)[: B * MBS].reshape(B, MBS).to(torch.int32)
+        T = 500
+        sid = torch.randint(0, B, (T,), generator=g, dtype=torch.int32)
+        pos = torch.randint(0, MBS * bs, (T,), generator=g, dtype=torch.int32)
+        want = oracle.slot_mapping(np_of(bt), np_of(sid), np_of(pos), bs)
+        got = torch.empty(T, dtype=torch.int64, device="cuda")
+        pa.pa_slot_mapping(bt.cuda(), sid.cuda(), pos.cuda(), bs, got)
+        assert np.array_equal(np_of(got), want)
+        # decode form: the last token of each sequence
+        lens = torch.randint(1, MBS * bs + 1, (B,), generator=g, dtype=torch.int32)
+        want = oracle.slot_mapping(np_of(bt), np.arange(B, dtype=np.int32), np_of(lens) - 1, bs)
+        got = torch.empty(B, dtype=torch.int64, device="cuda")
+        pa.pa_decode_slot_mapping(bt.cuda(), lens.cuda(), bs, got)
+        assert np.array_equal(np_of(got), want)
+    assert pa.pa_read_error_flag() == 0
+
+
+def test_slot_mapping_flags_unmapped_tokens(pa):
+    bt = torch.tensor([[4, -1], [7, 2]], dtype=torch.int32, device="cuda")
+    sid = torch.tensor([0, 0, 1, 3], dtype=torch.int32, device="cuda")
+    pos = torch.tensor([3, 20, 20, 0], dtype=torch.int32, device="cuda")
+    got = torch.empty(4, dtype=torch.int64, device="cuda")
+    pa.pa_slot_mapping(bt, sid, pos, 16, got)
+    assert got.tolist() == [4 * 16 + 3, -1, 2 * 16 + 4, -1]
+    assert pa.pa_read_error_flag() == 5
+    lens = torch.tensor([0, 17], dtype=torch.int32, device="cuda")
+    got = torch.empty(2, dtype=torch.int64, device="cuda")
+    pa.pa_decode_slot_mapping(bt, lens, 16, got)
+    assert got.tolist() == [-1, 2 * 16 + 0]
+    assert pa.pa_read_error_flag() == 0
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("bs", [8, 16, 32])
+def test_reshape_and_cache_bit_exact(pa, dtype, D, bs):
+    g = torch.Generator().manual_seed(D + bs)
+    NB, Hkv, T = 40, 4, 150
+    k_pool = torch.randn(NB, Hkv, bs, D, generator=g).to(DT[dtype])
+    v_pool = torch.randn(NB, Hkv, bs, D, generator=g).to(DT[dtype])
+    key = torch.randn(T, Hkv, D, generator=g).to(DT[dtype])
+    val = torch.randn(T, Hkv, D, generator=g).to(DT[dtype])
+    slots = torch.randperm(NB * bs, generator=g)[:T].to(torch.int64)
+    slots[::7] = -1
+    kp, vp = np_of(k_pool).copy(), np_of(v_pool).copy()
+    oracle.reshape_and_cache(np_of(key), np_of(val), kp, vp, np_of(slots))
+    gk, gv = k_pool.cuda(), v_pool.cuda()
+    pa.pa_reshape_and_cache(key.cuda(), val.cuda(), gk, gv, slots.cuda())
+    assert np_of(gk).tobytes() == kp.tobytes()
+    assert np_of(gv).tobytes() == vp.tobytes()
+    assert pa.pa_read_error_flag() == 0
+
+
+def test_reshape_and_cache_flags_slot_outside_pool(pa):
+    k_pool = torch.zeros(2, 1, 8, 64, device="cuda")
+    v_pool = torch.zeros_like(k_pool)
+    key = torch.ones(2, 1, 64, device="cuda")
+    slots = torch.tensor([3, 16], dtype=torch.int64, device="cuda")
+    pa.pa_reshape_and_cache(key, key, k_pool, v_pool, slots)
+    assert pa.pa_read_error_flag() == 5
+    assert k_pool[0, 0, 3].eq(1).all() and k_pool.sum().item() == 64
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("bs", [8, 16, 32])
+def test_copy_blocks_bit_exact(pa, dtype, bs):
+    g = torch.Generator().manual_seed(bs)
+    NB, Hkv, D = 64, 8, 128
+    k_pool = torch.randn(NB, Hkv, bs, D, generator=g).to(DT[dtype])
+    v_pool = torch.randn(NB, Hkv, bs, D, generator=g).to(DT[dtype])
+    perm = torch.randperm(NB, generator=g)
+    pairs = torch.stack([perm[:20], perm[20:40]], 1).to(torch.int64)  # distinct dsts, no dst is a src
+    kp, vp = np_of(k_pool).copy(), np_of(v_pool).copy()
+    oracle.copy_blocks(kp, vp, np_of(pairs))
+    gk, gv = k_pool.cuda(), v_pool.cuda()
+    pa.pa_copy_blocks(gk, gv, pairs.cuda())
+    assert np_of(gk).tobytes() == kp.tobytes()
+    assert np_of(gv).tobytes() == vp.tobytes()
+    assert pa.pa_read_error_flag() == 0
+
+
+def test_copy_blocks_flags_bad_pair(pa):
+    k_pool = torch.arange(4 * 64, dtype=torch.float32, device="cuda").reshape(4, 1, 1, 64).expand(4, 1, 8, 64)
+    k_pool = k_pool.contiguous()
+    v_pool = k_pool.clone()
+    before = k_pool.clone()
+    pa.pa_copy_blocks(k_pool, v_pool, torch.tensor([[0, 9], [1, 2]], dtype=torch.int64, device="cuda"))
+    assert pa.pa_read_error_flag() == 5
+    assert torch.equal(k_pool[2], before[1]) and torch.equal(k_pool[0], before[0])
