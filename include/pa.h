@@ -33,8 +33,8 @@
  *    tokens allocated at a time).
  *  * Grouped query heads: query head h reads kv head h / (Hq / Hkv).
  *  * Supported shapes: head_dim in {64, 128}; block_size in {8, 16, 32};
- *    Hq % Hkv == 0 with Hq / Hkv in {1, 2, 4, 8}.  Anything else returns
- *    PA_ERR_UNSUPPORTED without launching.
+ *    Hq % Hkv == 0 with Hq / Hkv in {1, 2, 4, 8}, or 16 for bf16.  Anything
+ *    else returns PA_ERR_UNSUPPORTED without launching.
  *  * Device-side checks: a block id outside [0, num_blocks), a negative or
  *    too-long context length, or a slot outside the pool is never
  *    dereferenced.  The kernel skips it and records the first such error in

@@ -37,12 +37,15 @@
 //
 // The contiguous-cache variant is the same kernel: only the producer's source
 // address differs (one bulk copy per 32-token stage instead of one per block).
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 #include <math.h>
 #include <stdint.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "pa.h"
 #include "pa_device.cuh"
@@ -55,8 +58,10 @@ constexpr int kConsumerWarps = 4;
 constexpr int kDecodeThreads = 32 * (1 + kConsumerWarps);
 constexpr int kStageTokens = 32;
 constexpr int kMaxPartition = 8192;
-constexpr int kMinAutoPartition = 512;
+constexpr int kMinAutoPartition = 256;
+constexpr int kDefaultPartition = 2048;
 constexpr int kRingTargetBytes = 64 * 1024;
+constexpr int kMaxDynamicSmem = 200 * 1024;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct DecodeParams {
@@ -131,6 +136,43 @@ __device__ __forceinline__ void store_out(const DecodeParams& p, int64_t idx, fl
         static_cast<float*>(p.out)[idx] = v;
 }
 
+// Combine the consumer warps' (m, l, o) states of one work item, held in
+// shared memory as o[w][h][d], m[w][h], l[w][h], and write the final row (one
+// split) or the normalised partial row plus (m, l) for the merge kernel.
+__device__ __forceinline__ void merge_warps_and_store(const DecodeParams& p, const float* sm_o, const float* sm_m,
+                                                      const float* sm_l, int G, int D, int b, int kvh, int split,
+                                                      int num_splits_b) {
+    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+        const int h = idx / D;
+        const int d = idx - h * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_m[w * G + h]);
+        float lt = 0.f, ot = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) {
+                const float mw = sm_m[w * G + h];
+                const float a = mw == -INFINITY ? 0.f : exp2f(mw - M);
+                lt += sm_l[w * G + h] * a;
+                ot += sm_o[(w * G + h) * D + d] * a;
+            }
+        }
+        const float val = lt > 0.f ? ot / lt : 0.f;
+        const int64_t qrow = (int64_t)b * p.num_q_heads + (int64_t)kvh * G + h;
+        if (num_splits_b == 1) {
+            store_out(p, qrow * D + d, val);
+        } else {
+            const int64_t r = qrow * p.max_splits + split;
+            p.part_o[r * D + d] = val;
+            if (d == 0) {
+                p.part_ml[2 * r] = M;
+                p.part_ml[2 * r + 1] = lt;
+            }
+        }
+    }
+}
+
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const DecodeParams p) {
     using E = Elt<T>;
@@ -196,47 +238,51 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const Deco
 
     if (warp == 0) {
         // ---------------- producer ----------------
-        if (lane == 0) {
-            const uint64_t policy = l2_policy_evict_first();
-            const char* kbase = static_cast<const char*>(p.k);
-            const char* vbase = static_cast<const char*>(p.v);
-            const int bs = p.block_size;
-            for (int j = 0; j < nstage; ++j) {
-                const int slot = j % p.stages;
-                if (j >= p.stages && !mbar_wait(&empty[slot], ((j / p.stages) - 1) & 1, p.err)) {
-                    s_abort = 1;
+        // Lane i issues the bulk copies of tile i of the stage (tile = one
+        // block of block_size tokens, or the same number of tokens of the
+        // contiguous cache), so the copies of a stage are issued in parallel.
+        const uint64_t policy = l2_policy_evict_first();
+        const char* kbase = static_cast<const char*>(p.k);
+        const char* vbase = static_cast<const char*>(p.v);
+        const int bs = p.block_size;
+        const int tiles = kStageTokens / bs;
+        for (int j = 0; j < nstage; ++j) {
+            const int slot = j % p.stages;
+            if (j >= p.stages) {
+                int ok = 1;
+                if (lane == 0) ok = mbar_wait(&empty[slot], ((j / p.stages) - 1) & 1, p.err);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                    if (lane == 0) s_abort = 1;
                     break;
                 }
-                uint8_t* kdst = ring + (size_t)slot * 2 * STAGE_BYTES;
-                uint8_t* vdst = kdst + STAGE_BYTES;
-                const int t0 = j * kStageTokens;
-                const int rows = min(kStageTokens, ntok - t0);
+            }
+            uint8_t* kdst = ring + (size_t)slot * 2 * STAGE_BYTES;
+            uint8_t* vdst = kdst + STAGE_BYTES;
+            const int t0 = j * kStageTokens;
+            const int rows = min(kStageTokens, ntok - t0);
+            const int r = lane * bs;
+            uint32_t nbytes = 0;
+            int64_t off = 0;
+            if (lane < tiles && r < rows) {
+                nbytes = (uint32_t)min(bs, rows - r) * ROW_BYTES;
                 if (p.contiguous) {
-                    const int64_t off =
-                        (((int64_t)b * p.num_kv_heads + kvh) * p.L_pad + tok_begin + t0) * (int64_t)ROW_BYTES;
-                    const uint32_t bytes = (uint32_t)rows * ROW_BYTES;
-                    mbar_arrive_expect_tx(&full[slot], 2 * bytes);
-                    bulk_load(kdst, kbase + off, bytes, &full[slot], policy);
-                    bulk_load(vdst, vbase + off, bytes, &full[slot], policy);
+                    off = (((int64_t)b * p.num_kv_heads + kvh) * p.L_pad + tok_begin + t0 + r) * (int64_t)ROW_BYTES;
                 } else {
-                    uint32_t bytes = 0;
-                    for (int r = 0; r < rows; r += bs) {
-                        const int32_t phys = tbl[(t0 + r) / bs];
-                        if (phys >= 0 && phys < p.num_blocks) bytes += (uint32_t)min(bs, rows - r) * ROW_BYTES;
-                    }
-                    mbar_arrive_expect_tx(&full[slot], 2 * bytes);
-                    for (int r = 0; r < rows; r += bs) {
-                        const int32_t phys = tbl[(t0 + r) / bs];
-                        if (phys < 0 || phys >= p.num_blocks) {
-                            record_error(p.err, PA_ERR_BAD_BLOCK_ID);
-                            continue;
-                        }
-                        const uint32_t nbytes = (uint32_t)min(bs, rows - r) * ROW_BYTES;
-                        const int64_t off = ((int64_t)phys * p.num_kv_heads + kvh) * bs * (int64_t)ROW_BYTES;
-                        bulk_load(kdst + r * ROW_BYTES, kbase + off, nbytes, &full[slot], policy);
-                        bulk_load(vdst + r * ROW_BYTES, vbase + off, nbytes, &full[slot], policy);
+                    const int32_t phys = tbl[(t0 + r) / bs];
+                    if (phys < 0 || phys >= p.num_blocks) {
+                        record_error(p.err, PA_ERR_BAD_BLOCK_ID);
+                        nbytes = 0;
+                    } else {
+                        off = ((int64_t)phys * p.num_kv_heads + kvh) * bs * (int64_t)ROW_BYTES;
                     }
                 }
+            }
+            const uint32_t total = __reduce_add_sync(0xffffffffu, nbytes);
+            if (lane == 0) mbar_arrive_expect_tx(&full[slot], 2 * total);
+            __syncwarp();
+            if (nbytes) {
+                bulk_load(kdst + r * ROW_BYTES, kbase + off, nbytes, &full[slot], policy);
+                bulk_load(vdst + r * ROW_BYTES, vbase + off, nbytes, &full[slot], policy);
             }
         }
     } else {
@@ -368,35 +414,345 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const Deco
         }
     }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-        const int h = idx / D;
-        const int d = idx - h * D;
-        float M = -INFINITY;
+    merge_warps_and_store(p, sm_o, sm_m, sm_l, G, D, b, kvh, split, num_splits_b);
+}
+
+// ---------------------------------------------------------------------------
+// bf16 pass 1 on the tensor cores.
+//
+// Same work decomposition, ring and producer/consumer roles as the kernel
+// above, with two differences:
+//  * K/V tiles are staged by tiled TMA (cp.async.bulk.tensor, 2-D tensor map
+//    over the pool viewed as [rows, head_dim]) with the 128-byte swizzle: a
+//    stage holds, per 64-element column slab, 32 token rows of 128 bytes in
+//    which 16-byte chunk c of row r sits at chunk c ^ (r & 7).  ldmatrix of 8
+//    token rows then touches 8 different bank groups.
+//  * The consumer warp does the two contractions with mma.sync m16n8k16
+//    (bf16 in, fp32 accumulate), tokens on the M side and the G query heads of
+//    the kv head on the N side:
+//        S^T[tokens, heads] = K[tokens, D] . Q^T[D, heads]
+//        O^T[D, heads]     += V^T[D, tokens] . P^T[tokens, heads]
+//    P^T comes from the S^T accumulator transposed in registers (movmatrix);
+//    P is split into a bf16 high part and a bf16 residual, both multiplied by
+//    V, so the weights keep ~16 significant bits instead of 8.
+// G <= 8 uses one 8-wide N tile (NT = 1), G == 16 two.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t swizzled(uint32_t slab, int row, int chunk) {
+    return slab + row * 128 + ((chunk ^ (row & 7)) << 4);
+}
+
+template <int D, int NT>
+__global__ void __launch_bounds__(kDecodeThreads)
+    decode_pass1_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
+                            const __grid_constant__ CUtensorMap tmv) {
+    constexpr int SLABS = D / 64;
+    constexpr int SLAB_BYTES = kStageTokens * 128;
+    constexpr int STAGE_BYTES = SLABS * SLAB_BYTES;  // K (or V) part of one stage
+    constexpr int KSTEPS = D / 16;
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + p.stages;
+    int32_t* tbl = reinterpret_cast<int32_t*>(empty + p.stages);
+    // the 128-byte swizzle pattern assumes 1024-byte aligned slabs: align the
+    // ring at run time (the launch reserves 1 KB of slack for this)
+    uint8_t* ring = smem + p.ring_offset + ((1024u - (smem_addr(smem) & 1023u)) & 1023u);
+    __shared__ int s_abort;
+
+    const int split = blockIdx.x;
+    const int kvh = blockIdx.y;
+    const int b = blockIdx.z;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int G = p.num_q_heads / p.num_kv_heads;
+
+    const int L = clamp_len(p, b, threadIdx.x == 0 && split == 0 && kvh == 0);
+    const int tok_begin = split * p.partition;
+    if (split > 0 && tok_begin >= L) return;
+    const int ntok = max(0, min(L, tok_begin + p.partition) - tok_begin);
+    const int nstage = (ntok + kStageTokens - 1) / kStageTokens;
+    const int num_splits_b = L > 0 ? (L + p.partition - 1) / p.partition : 1;
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        prefetch_tmap(&tmk);
+        prefetch_tmap(&tmv);
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        fence_barrier_init();
+    }
+    if (!p.contiguous) {
+        const int first_blk = tok_begin / p.block_size;
+        const int nblk = (ntok + p.block_size - 1) / p.block_size;
+        const int32_t* row = p.block_tables + (int64_t)b * p.max_blocks_per_seq + first_blk;
+        for (int i = threadIdx.x; i < nblk; i += blockDim.x) tbl[i] = row[i];
+    }
+    __syncthreads();
+
+    const int g = lane >> 2;  // fragment row group
+    const int t = lane & 3;   // fragment column pair
+    float o[KSTEPS][NT][4];
+    float m[NT][2], l[NT][2];
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_m[w * G + h]);
-        float lt = 0.f, ot = 0.f;
-        if (M != -INFINITY) {
+    for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) {
-                const float mw = sm_m[w * G + h];
-                const float a = mw == -INFINITY ? 0.f : exp2f(mw - M);
-                lt += sm_l[w * G + h] * a;
-                ot += sm_o[(w * G + h) * D + d] * a;
+        for (int i = 0; i < 2; ++i) {
+            m[nt][i] = -INFINITY;
+            l[nt][i] = 0.f;
+        }
+#pragma unroll
+        for (int mt = 0; mt < KSTEPS; ++mt)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) o[mt][nt][c] = 0.f;
+    }
+
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        // Lane i loads tile i of the stage (block_size rows) for every column
+        // slab of K and V; the box is always block_size full rows.
+        const uint64_t policy = l2_policy_evict_first();
+        const int bs = p.block_size;
+        const int tiles = kStageTokens / bs;
+        const uint32_t tile_bytes = (uint32_t)(SLABS * bs * 128);
+        for (int j = 0; j < nstage; ++j) {
+            const int slot = j % p.stages;
+            if (j >= p.stages) {
+                int ok = 1;
+                if (lane == 0) ok = mbar_wait(&empty[slot], ((j / p.stages) - 1) & 1, p.err);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                    if (lane == 0) s_abort = 1;
+                    break;
+                }
+            }
+            uint8_t* kdst = ring + (size_t)slot * 2 * STAGE_BYTES;
+            uint8_t* vdst = kdst + STAGE_BYTES;
+            const int t0 = j * kStageTokens;
+            const int rows = min(kStageTokens, ntok - t0);
+            const int r = lane * bs;
+            int y = 0;
+            uint32_t nbytes = 0;
+            if (lane < tiles && r < rows) {
+                nbytes = tile_bytes;
+                if (p.contiguous) {
+                    y = (int)(((int64_t)b * p.num_kv_heads + kvh) * p.L_pad + tok_begin + t0 + r);
+                } else {
+                    const int32_t phys = tbl[(t0 + r) / bs];
+                    if (phys < 0 || phys >= p.num_blocks) {
+                        record_error(p.err, PA_ERR_BAD_BLOCK_ID);
+                        nbytes = 0;
+                    } else {
+                        y = (phys * p.num_kv_heads + kvh) * bs;
+                    }
+                }
+            }
+            const uint32_t total = __reduce_add_sync(0xffffffffu, nbytes);
+            if (lane == 0) mbar_arrive_expect_tx(&full[slot], 2 * total);
+            __syncwarp();
+            if (nbytes) {
+#pragma unroll
+                for (int sl = 0; sl < SLABS; ++sl) {
+                    tma_load_2d(kdst + sl * SLAB_BYTES + r * 128, &tmk, sl * 64, y, &full[slot], policy);
+                    tma_load_2d(vdst + sl * SLAB_BYTES + r * 128, &tmv, sl * 64, y, &full[slot], policy);
+                }
             }
         }
-        const float val = lt > 0.f ? ot / lt : 0.f;
-        const int64_t qrow = (int64_t)b * p.num_q_heads + (int64_t)kvh * G + h;
-        if (num_splits_b == 1) {
-            store_out(p, qrow * D + d, val);
-        } else {
-            const int64_t r = qrow * p.max_splits + split;
-            p.part_o[r * D + d] = val;
-            if (d == 0) {
-                p.part_ml[2 * r] = M;
-                p.part_ml[2 * r + 1] = lt;
+    } else {
+        // ---------------- consumers ----------------
+        const int cw = warp - 1;
+        // Q^T fragments (k = head_dim, n = query head of the group), bf16 pairs
+        uint32_t qb[NT][KSTEPS][2];
+        {
+            const uint16_t* qbase = static_cast<const uint16_t*>(p.q) +
+                                    ((int64_t)b * p.num_q_heads + (int64_t)kvh * G) * D;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int head = nt * 8 + g;
+#pragma unroll
+                for (int kk = 0; kk < KSTEPS; ++kk) {
+                    if (head < G) {
+                        qb[nt][kk][0] = *reinterpret_cast<const uint32_t*>(qbase + head * D + kk * 16 + 2 * t);
+                        qb[nt][kk][1] = *reinterpret_cast<const uint32_t*>(qbase + head * D + kk * 16 + 8 + 2 * t);
+                    } else {
+                        qb[nt][kk][0] = qb[nt][kk][1] = 0u;
+                    }
+                }
             }
+        }
+        const int q4 = lane >> 3;  // which of the four ldmatrix matrices this lane addresses
+        const int r8 = lane & 7;   // which row of it
+        for (int j = cw; j < nstage; j += kConsumerWarps) {
+            const int slot = j % p.stages;
+            if (!mbar_wait(&full[slot], (j / p.stages) & 1, p.err)) {
+                s_abort = 1;
+                break;
+            }
+            uint8_t* kstage = ring + (size_t)slot * 2 * STAGE_BYTES;
+            uint8_t* vstage = kstage + STAGE_BYTES;
+            const uint32_t kst = smem_addr(kstage);
+            const uint32_t vst = smem_addr(vstage);
+            const int valid = min(kStageTokens, ntok - j * kStageTokens);
+            if (valid < kStageTokens) {
+                // rows past the sequence end may hold anything (NaN included):
+                // zero them so that 0-weight * V stays 0 in the MMA
+                const int nchunks = (kStageTokens - valid) * SLABS * 8;
+                for (int c = lane; c < nchunks; c += 32) {
+                    const int row = valid + c / (SLABS * 8);
+                    const int rem = c % (SLABS * 8);
+                    *reinterpret_cast<uint4*>(vstage + (rem >> 3) * SLAB_BYTES + row * 128 + (rem & 7) * 16) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+                __syncwarp();
+            }
+            // S^T = K . Q^T : two 16-token M tiles
+            float s[2][NT][4];
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) s[mt][nt][c] = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < KSTEPS; ++kk) {
+                const uint32_t slab = kst + (kk >> 2) * SLAB_BYTES;
+                const int chunk = (kk & 3) * 2 + (q4 >> 1);
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt) {
+                    uint32_t a[4];
+                    ldmatrix_x4(swizzled(slab, 16 * mt + r8 + 8 * (q4 & 1), chunk), a[0], a[1], a[2], a[3]);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[mt][nt], a, qb[nt][kk][0], qb[nt][kk][1]);
+                }
+            }
+            // online softmax, one column (query head) at a time; this lane holds
+            // tokens g, g + 8, 16 + g, 24 + g of columns 8 nt + 2 t + i
+            bool rescale = false;
+            float alpha[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    float v[4] = {s[0][nt][i], s[0][nt][2 + i], s[1][nt][i], s[1][nt][2 + i]};
+                    float mx = -INFINITY;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int tok = 16 * (k >> 1) + g + 8 * (k & 1);
+                        v[k] = tok < valid ? v[k] * p.scale_log2 : -INFINITY;
+                        mx = fmaxf(mx, v[k]);
+                    }
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                    const float m_new = fmaxf(m[nt][i], mx);
+                    float a = 1.f;
+                    if (m_new == -INFINITY) {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) v[k] = 0.f;
+                    } else {
+                        a = exp2f(m[nt][i] - m_new);
+                        float sum = 0.f;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            v[k] = exp2f(v[k] - m_new);
+                            sum += v[k];
+                        }
+                        l[nt][i] = l[nt][i] * a + sum;
+                        m[nt][i] = m_new;
+                    }
+                    alpha[nt][i] = a;
+                    rescale |= a != 1.f;
+                    s[0][nt][i] = v[0];
+                    s[0][nt][2 + i] = v[1];
+                    s[1][nt][i] = v[2];
+                    s[1][nt][2 + i] = v[3];
+                }
+            }
+            if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+                for (int mt = 0; mt < KSTEPS; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        o[mt][nt][0] *= alpha[nt][0];
+                        o[mt][nt][1] *= alpha[nt][1];
+                        o[mt][nt][2] *= alpha[nt][0];
+                        o[mt][nt][3] *= alpha[nt][1];
+                    }
+            }
+            // O^T += V^T . P^T, one 16-token K step per S^T M tile
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks) {
+                uint32_t bh[NT][2], bl[NT][2];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const float p0 = s[ks][nt][2 * half], p1 = s[ks][nt][2 * half + 1];
+                        const uint32_t hi = pack_bf16x2(p0, p1);
+                        const uint32_t lo = pack_bf16x2(p0 - bf16_lo_to_f32(hi), p1 - bf16_hi_to_f32(hi));
+                        bh[nt][half] = movmatrix_trans(hi);
+                        bl[nt][half] = movmatrix_trans(lo);
+                    }
+                }
+#pragma unroll
+                for (int mt = 0; mt < KSTEPS; ++mt) {
+                    const uint32_t slab = vst + (mt >> 2) * SLAB_BYTES;
+                    const int chunk = (mt & 3) * 2 + (q4 & 1);
+                    uint32_t a[4];
+                    ldmatrix_x4_trans(swizzled(slab, 16 * ks + r8 + 8 * (q4 >> 1), chunk), a[0], a[1], a[2], a[3]);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        mma_bf16_16816(o[mt][nt], a, bh[nt][0], bh[nt][1]);
+                        mma_bf16_16816(o[mt][nt], a, bl[nt][0], bl[nt][1]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
+        }
+        // l was summed per lane over its own tokens: add the 8 lanes of a column
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                l[nt][i] += __shfl_xor_sync(0xffffffffu, l[nt][i], 4);
+                l[nt][i] += __shfl_xor_sync(0xffffffffu, l[nt][i], 8);
+                l[nt][i] += __shfl_xor_sync(0xffffffffu, l[nt][i], 16);
+            }
+    }
+    __syncthreads();  // pipeline drained: the ring is free for the merge scratch
+    if (s_abort) return;
+
+    float* sm_o = reinterpret_cast<float*>(ring);  // [4][G][D]
+    float* sm_m = sm_o + kConsumerWarps * G * D;    // [4][G]
+    float* sm_l = sm_m + kConsumerWarps * G;        // [4][G]
+    if (warp > 0) {
+        const int cw = warp - 1;
+#pragma unroll
+        for (int mt = 0; mt < KSTEPS; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int head = nt * 8 + 2 * t + (c & 1);
+                    const int dim = 16 * mt + g + 8 * (c >> 1);
+                    if (head < G) sm_o[(cw * G + head) * D + dim] = o[mt][nt][c];
+                }
+        if (g == 0) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int head = nt * 8 + 2 * t + i;
+                    if (head < G) {
+                        sm_m[cw * G + head] = m[nt][i];
+                        sm_l[cw * G + head] = l[nt][i];
+                    }
+                }
         }
     }
+    __syncthreads();
+    merge_warps_and_store(p, sm_o, sm_m, sm_l, G, D, b, kvh, split, num_splits_b);
 }
 
 // Second pass: out = sum_s w_s o_s / sum_s w_s with w_s = l_s * 2^(m_s - max m),
@@ -460,15 +816,14 @@ struct Plan {
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 int auto_partition(int batch, int num_kv_heads, int max_context_len) {
-    if (max_context_len <= 0) return kMinAutoPartition;
-    // About six work items per resident CTA slot (three CTAs per SM), assuming
-    // lengths spread evenly below max_context_len; long items are split so the
-    // tail of the grid stays short.
-    const double slots = (double)num_sms() * 3.0;
-    const double est_tokens = (double)batch * num_kv_heads * max_context_len * 0.5;
-    const double target = est_tokens / (slots * 6.0);
-    int P = kMinAutoPartition;
-    while (P < kMaxPartition && 2.0 * P <= target) P *= 2;
+    // 2048 tokens per split (measured best on the B200 for batch >= 16 from
+    // 1k to 128k tokens: fewer, longer work items keep each CTA's TMA ring
+    // streaming and make the merge pass rare); halved while the grid would
+    // hold fewer than four work items per SM.
+    int P = kDefaultPartition;
+    const int64_t min_items = 4ll * num_sms();
+    const int64_t L = max_context_len > 0 ? max_context_len : 1;
+    while (P > kMinAutoPartition && (int64_t)batch * num_kv_heads * ((L + P - 1) / P) < min_items) P /= 2;
     return P;
 }
 
@@ -492,6 +847,53 @@ int make_plan(int batch, int num_q_heads, int num_kv_heads, int head_dim, int ma
     return PA_OK;
 }
 
+using TensorMapEncodeFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+TensorMapEncodeFn tensor_map_encoder() {
+    static TensorMapEncodeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<TensorMapEncodeFn>(ptr);
+    });
+    return fn;
+}
+
+// 2-D bf16 tensor map over `rows` rows of head_dim elements, boxes of 64
+// elements (128 bytes, the swizzle span) by box_rows rows, 128-byte swizzle.
+int encode_kv_map(CUtensorMap* map, const void* base, uint64_t rows, int head_dim, int box_rows) {
+    TensorMapEncodeFn enc = tensor_map_encoder();
+    if (!enc) return PA_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)head_dim, rows > 0 ? rows : 1};
+    cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
+    cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+    cuuint32_t elem_strides[2] = {1u, 1u};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                           elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+}
+
+template <int D, int NT>
+int launch_pass1_mma(const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, dim3 grid, size_t smem,
+                     cudaStream_t st) {
+    static std::atomic<unsigned long long> configured{0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(configured.load() & bit)) {
+        if (cudaFuncSetAttribute(decode_pass1_mma_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kMaxDynamicSmem) != cudaSuccess)
+            return PA_ERR_CUDA;
+        configured.fetch_or(bit);
+    }
+    decode_pass1_mma_kernel<D, NT><<<grid, kDecodeThreads, smem, st>>>(p, tmk, tmv);
+    return launch_status();
+}
+
 template <typename T, int D, int G>
 int launch_pass1(const DecodeParams& p, dim3 grid, size_t smem, cudaStream_t st) {
     static std::atomic<unsigned long long> configured{0};
@@ -500,7 +902,7 @@ int launch_pass1(const DecodeParams& p, dim3 grid, size_t smem, cudaStream_t st)
     const unsigned long long bit = 1ull << (dev & 63);
     if (!(configured.load() & bit)) {
         if (cudaFuncSetAttribute(decode_pass1_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 96 * 1024) != cudaSuccess)
+                                 kMaxDynamicSmem) != cudaSuccess)
             return PA_ERR_CUDA;
         configured.fetch_or(bit);
     }
@@ -539,8 +941,13 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
     if (!p.err) return PA_ERR_CUDA;
 
     const int stage_bytes = 2 * kStageTokens * head_dim * (int)dtype_bytes(kv_dtype);  // K + V
-    int stages = kRingTargetBytes / stage_bytes;
-    stages = stages < 2 ? 2 : (stages > 8 ? 8 : stages);
+    // Stage j lives in slot j % stages and is consumed by warp j % 4.  The
+    // stage count must be a multiple of the consumer-warp count: then the
+    // previous user of a slot is the same warp, so a warp never waits on a
+    // full-barrier phase more than one ahead of the barrier's current phase
+    // (a parity wait cannot tell phase k + 2 from phase k).
+    int stages = (kRingTargetBytes / stage_bytes) / kConsumerWarps * kConsumerWarps;
+    stages = stages < kConsumerWarps ? kConsumerWarps : (stages > 2 * kConsumerWarps ? 2 * kConsumerWarps : stages);
     p.stages = stages;
     const int table_bytes = p.contiguous ? 0 : (plan.partition / p.block_size) * 4;
     p.ring_offset = (int)((16 * stages + table_bytes + 127) & ~127);
@@ -548,11 +955,26 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
     const size_t merge_bytes = (size_t)kConsumerWarps * G * (head_dim + 2) * sizeof(float);
     if (merge_bytes > ring_bytes) return PA_ERR_UNSUPPORTED;
     const size_t smem = p.ring_offset + ring_bytes;
+    if (smem > (size_t)kMaxDynamicSmem) return PA_ERR_UNSUPPORTED;
 
     dim3 grid((unsigned)plan.max_splits, (unsigned)p.num_kv_heads, (unsigned)batch);
     if (kv_dtype == PA_BF16) {
-        rc = head_dim == 128 ? dispatch_group<__nv_bfloat16, 128>(G, p, grid, smem, st)
-                             : dispatch_group<__nv_bfloat16, 64>(G, p, grid, smem, st);
+        // tensor-core path: K/V tiles by tiled TMA, contractions by mma.sync
+        const uint64_t rows = p.contiguous ? (uint64_t)batch * p.num_kv_heads * (uint64_t)p.L_pad
+                                           : (uint64_t)p.num_blocks * p.num_kv_heads * (uint64_t)p.block_size;
+        if (rows >= (1ull << 31)) return PA_ERR_UNSUPPORTED;
+        CUtensorMap tmk, tmv;
+        if ((rc = encode_kv_map(&tmk, p.k, rows, head_dim, p.block_size))) return rc;
+        if ((rc = encode_kv_map(&tmv, p.v, rows, head_dim, p.block_size))) return rc;
+        p.ring_offset = (int)((16 * stages + table_bytes + 1023) & ~1023);
+        const size_t smem_mma = p.ring_offset + ring_bytes + 1024;
+        if (smem_mma > (size_t)kMaxDynamicSmem) return PA_ERR_UNSUPPORTED;
+        if (head_dim == 128)
+            rc = G <= 8 ? launch_pass1_mma<128, 1>(p, tmk, tmv, grid, smem_mma, st)
+                        : launch_pass1_mma<128, 2>(p, tmk, tmv, grid, smem_mma, st);
+        else
+            rc = G <= 8 ? launch_pass1_mma<64, 1>(p, tmk, tmv, grid, smem_mma, st)
+                        : launch_pass1_mma<64, 2>(p, tmk, tmv, grid, smem_mma, st);
     } else {
         rc = head_dim == 128 ? dispatch_group<float, 128>(G, p, grid, smem, st)
                              : dispatch_group<float, 64>(G, p, grid, smem, st);
@@ -579,7 +1001,7 @@ int check_shapes(int batch, int num_q_heads, int num_kv_heads, int head_dim, int
     if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
     if (!supported_head_dim(head_dim) || !supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
     const int G = num_q_heads / num_kv_heads;
-    if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
+    if (G != 1 && G != 2 && G != 4 && G != 8 && !(G == 16 && kv_dtype == PA_BF16)) return PA_ERR_UNSUPPORTED;
     if (batch > 65535 || num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
     return PA_OK;
 }
@@ -592,7 +1014,7 @@ using namespace pa;
 extern "C" int pa_paged_attention_partition_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
                                                  int max_context_len, int block_size, int* partition_size) {
     if (!partition_size) return PA_ERR_INVALID_ARG;
-    int rc = check_shapes(batch, num_q_heads, num_kv_heads, head_dim, block_size, PA_F32, PA_F32, max_context_len);
+    int rc = check_shapes(batch, num_q_heads, num_kv_heads, head_dim, block_size, PA_BF16, PA_F32, max_context_len);
     if (rc) return rc;
     *partition_size = auto_partition(batch, num_kv_heads, max_context_len);
     return PA_OK;
@@ -602,7 +1024,7 @@ extern "C" int pa_paged_attention_workspace_size(int batch, int num_q_heads, int
                                                  int max_context_len, int block_size, int partition_size,
                                                  size_t* workspace_bytes) {
     if (!workspace_bytes) return PA_ERR_INVALID_ARG;
-    int rc = check_shapes(batch, num_q_heads, num_kv_heads, head_dim, block_size, PA_F32, PA_F32, max_context_len);
+    int rc = check_shapes(batch, num_q_heads, num_kv_heads, head_dim, block_size, PA_BF16, PA_F32, max_context_len);
     if (rc) return rc;
     Plan plan;
     rc = make_plan(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, partition_size, &plan);

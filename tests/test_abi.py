@@ -66,7 +66,8 @@ def _decode(lib, **kw):
 
 def test_decode_rejects_bad_shapes(lib):
     assert _decode(lib, hq=6, hkv=4) == INVALID            # Hq % Hkv != 0
-    assert _decode(lib, hq=32, hkv=2) == UNSUPPORTED       # group of 16
+    assert _decode(lib, hq=64, hkv=2) == UNSUPPORTED       # group of 32
+    assert _decode(lib, hq=32, hkv=2, kv_dtype=0) == UNSUPPORTED  # group of 16 needs bf16
     assert _decode(lib, d=96) == UNSUPPORTED
     assert _decode(lib, bs=64) == UNSUPPORTED
     assert _decode(lib, kv_dtype=7) == INVALID
@@ -98,7 +99,7 @@ def test_workspace_size(lib):
     assert lib.pa_paged_attention_workspace_size(4, 8, 2, 128, 100, 16, 33, ctypes.byref(sz)) == INVALID
     part = ctypes.c_int(0)
     assert lib.pa_paged_attention_partition_size(64, 32, 32, 128, 2048, 16, ctypes.byref(part)) == OK
-    assert part.value % 32 == 0 and 512 <= part.value <= 8192
+    assert part.value % 32 == 0 and 256 <= part.value <= 8192
 
 
 def test_cache_kernels_reject_bad_arguments(lib):
