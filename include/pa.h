@@ -203,6 +203,45 @@ int pa_paged_attention_decode_contiguous(const void* q, const void* k_c, const v
                                          int partition_size, void* workspace,
                                          size_t workspace_bytes, void* stream);
 
+/*
+ * pa_paged_attention_decode_static_scratch -- pa_paged_attention_decode for
+ * callers that cannot allocate device memory.  The pages have no counterpart:
+ * this is a deployment convenience of this library.
+ *
+ * Some callers cannot call cudaMalloc (or any allocating routine) where they
+ * run decode attention: code inside a CUDA graph capture or a latency-bound
+ * serving loop that must not enter the allocator, or an embedder whose device
+ * memory belongs to another framework's pool.  This entry point takes the
+ * same arguments as pa_paged_attention_decode minus the workspace and uses
+ * instead a fixed scratch array of PA_STATIC_SCRATCH_BYTES that lives in the
+ * library itself (a file-scope __device__ array).  It calls no cudaMalloc,
+ * cudaFree or other allocating routine.  The caller still passes q, the
+ * pools, the tables and `out`, exactly as for pa_paged_attention_decode, and
+ * gets bit-identical results.
+ *
+ *  * Memory: every GPU that loads the library holds the PA_STATIC_SCRATCH_BYTES
+ *    array until the process exits, whether or not this entry point is used.
+ *  * Limit: a call whose split-KV scratch (pa_paged_attention_workspace_size)
+ *    exceeds PA_STATIC_SCRATCH_BYTES returns PA_ERR_WORKSPACE without
+ *    launching; a larger partition_size needs less scratch.
+ *  * Set-up: the first call on each device looks up the array's device
+ *    address (cudaGetSymbolAddress, with that device current) and caches it;
+ *    make that first call before any stream capture on the device.
+ *  * Sharing: every call uses the same array, which keeps the previous call's
+ *    contents (nothing in it needs to start at zero).  Calls that overlap on
+ *    the GPU, for example on two streams, race on it; calls ordered on one
+ *    stream are safe.
+ */
+#define PA_STATIC_SCRATCH_BYTES (16u << 20)
+
+int pa_paged_attention_decode_static_scratch(const void* q, const void* k_pool, const void* v_pool,
+                                             const int32_t* block_tables, int max_blocks_per_seq,
+                                             const int32_t* context_lens, int max_context_len,
+                                             float scale, int block_size, void* out, int out_dtype,
+                                             int batch, int num_q_heads, int num_kv_heads,
+                                             int head_dim, int64_t num_blocks, int kv_dtype,
+                                             int partition_size, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -43,6 +43,8 @@ _SIGS = {
                                    _SZ, _P], _I),
     "pa_paged_attention_decode_contiguous": ([_P, _P, _P, _I64, _P, _I, _F, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P,
                                               _SZ, _P], _I),
+    "pa_paged_attention_decode_static_scratch": ([_P, _P, _P, _P, _I, _P, _I, _F, _I, _P, _I, _I, _I, _I, _I, _I64,
+                                                  _I, _I, _P], _I),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -207,3 +209,28 @@ def pa_paged_attention_decode_contiguous(q, k_c, v_c, context_lens, max_context_
         _dev(q, "q"), k_c.data_ptr(), v_c.data_ptr(), L_pad, _dev(context_lens, "context_lens", torch.int32),
         int(max_context_len), float(scale), block_size, _dev(out, "out"), _kv_dtype(out), B, Hq, Hkv, D, dt,
         partition_size, ws, ws_bytes, _stream(stream)))
+
+
+STATIC_SCRATCH_BYTES = 16 << 20  # PA_STATIC_SCRATCH_BYTES in include/pa.h
+
+
+def pa_paged_attention_decode_static_scratch(q, k_pool, v_pool, block_tables, context_lens, max_context_len: int,
+                                             scale: float, out, partition_size: int = 0, stream=None) -> None:
+    """pa_paged_attention_decode without a workspace argument, for callers
+    that cannot allocate device memory: the split-KV scratch is a fixed array
+    of STATIC_SCRATCH_BYTES inside libpa, shared by all calls (calls that
+    overlap on the GPU race on it).  Raises PAError(PA_ERR_WORKSPACE) when the
+    sizes need more scratch than that.  The first call on a device looks up the
+    array's address and should come before any stream capture."""
+    B, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_pool.shape
+    if D2 != D or v_pool.shape != k_pool.shape or tuple(out.shape) != (B, Hq, D):
+        raise ValueError("q / pool / out shapes disagree")
+    MBS = block_tables.shape[1]
+    dt = _kv_dtype(q)
+    _dev(k_pool, "k_pool", q.dtype)
+    _dev(v_pool, "v_pool", q.dtype)
+    _check("pa_paged_attention_decode_static_scratch", _lib.pa_paged_attention_decode_static_scratch(
+        _dev(q, "q"), k_pool.data_ptr(), v_pool.data_ptr(), _dev(block_tables, "block_tables", torch.int32), MBS,
+        _dev(context_lens, "context_lens", torch.int32), int(max_context_len), float(scale), bs, _dev(out, "out"),
+        _kv_dtype(out), B, Hq, Hkv, D, NB, dt, partition_size, _stream(stream)))
