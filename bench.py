@@ -71,6 +71,8 @@ def parse():
     ap.add_argument("--workload", default="llama7b", choices=sorted(DESCRIPTIONS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--partition", type=int, default=0, help="tokens per KV split (0 = automatic)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (smaller cases for profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -189,11 +191,13 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank time over all ranks (the job is as slow as its slowest GPU)."""
     if world == 1:
         return x
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -293,7 +297,7 @@ def run_ours(args):
     from paged_kv_cache_355_b200.workloads import SEEDS, make_case
 
     dev = torch.device("cuda", local)
-    case = make_case(args.workload, device=dev, seed=SEEDS[args.workload] + 101 * rank)
+    case = make_case(args.workload, device=dev, seed=SEEDS[args.workload] + 101 * rank, batch=args.batch)
     w = case.workload
     B, Hq, Hkv, D, bs = w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size
     stream = torch.cuda.current_stream()
@@ -425,7 +429,8 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32", "data": "synthetic",
-        "config": {"workload": DESCRIPTIONS[args.workload], "batch_per_gpu": B, "partition_tokens": part,
+        "config": {"workload": DESCRIPTIONS[args.workload] + (f" (batch overridden to {B})" if args.batch else ""),
+                   "batch_per_gpu": B, "partition_tokens": part,
                    "max_splits": max_splits, "kv_bytes_per_step": kv_bytes,
                    "l2": "flushed between steps by a 256 MiB write outside the timed events; "
                          "K/V read per step also exceeds the 126 MB L2",

@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const Deco
     static_assert(TPT >= 1 && TPT <= 32 && NG * TPT == 32, "lane layout");
     static_assert(PASSES % PCH == 0, "chunking");
 
-    extern __shared__ __align__(128) uint8_t smem[];
+    extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + p.stages;
     int32_t* tbl = reinterpret_cast<int32_t*>(empty + p.stages);
