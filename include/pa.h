@@ -204,6 +204,66 @@ int pa_paged_attention_decode_contiguous(const void* q, const void* k_c, const v
                                          size_t workspace_bytes, void* stream);
 
 /*
+ * ------------------------------------------------------------------------
+ * Host-side block manager.
+ *
+ * The allocator the pages describe: fixed-size blocks, a per-sequence block
+ * table, one block taken at a time as a sequence grows ([P1] introduction;
+ * [P3] "Detail", "Key Technical Innovations" 1-2), a first-in first-out free
+ * list that starts as every block id in increasing order ([P3] "Example"),
+ * reference counts and copy-on-write for shared blocks ([P2] "Key terms in
+ * this lesson").  Unlike the kernels above it is stateful host code: the
+ * handle owns host memory until pa_bm_destroy.  Not thread-safe.  Every
+ * pointer argument here is a HOST pointer.
+ * ------------------------------------------------------------------------
+ */
+typedef struct pa_block_manager pa_block_manager;
+
+/* A manager for num_blocks blocks of block_size tokens; NULL on bad sizes or
+ * out of host memory.  Block ids are 0..num_blocks-1 (num_blocks < 2^31). */
+pa_block_manager* pa_bm_create(int64_t num_blocks, int block_size);
+void pa_bm_destroy(pa_block_manager* bm);
+
+/* Register an empty sequence (PA_ERR_INVALID_ARG if the id exists). */
+int pa_bm_add_sequence(pa_block_manager* bm, int64_t seq_id);
+
+/*
+ * Append one token to each seq_ids[i] in order (unknown ids start empty).
+ * slots[i] receives the token's slot.  A token at position pos takes a new
+ * block from the head of the free list when pos % block_size == 0.  A token
+ * written into a block shared with other sequences (refcount > 1) first moves
+ * its sequence onto a fresh block: the pair (shared, fresh) is appended to
+ * cow_pairs (int64 [2 * capacity], may be NULL to only count) and counted in
+ * *num_cow_pairs; the caller runs pa_copy_blocks on those pairs before
+ * writing the tokens.  Returns PA_ERR_WORKSPACE when the free list runs out;
+ * the tokens before the failing one stay appended.
+ */
+int pa_bm_append_tokens(pa_block_manager* bm, const int64_t* seq_ids, int64_t n, int64_t* slots,
+                        int64_t* cow_pairs, int64_t* num_cow_pairs);
+
+/* child shares every block of parent (reference counts + 1). */
+int pa_bm_fork(pa_block_manager* bm, int64_t parent, int64_t child);
+
+/* Drop a sequence; blocks whose count reaches 0 return to the free list's tail. */
+int pa_bm_free_sequence(pa_block_manager* bm, int64_t seq_id);
+
+/* Free blocks, a block's reference count, a sequence's length (-1 if unknown). */
+int64_t pa_bm_num_free(const pa_block_manager* bm);
+int pa_bm_refcount(const pa_block_manager* bm, int64_t block);
+int64_t pa_bm_length(const pa_block_manager* bm, int64_t seq_id);
+
+/* Dense block tables int32 [n][max_blocks_per_seq] (-1 past each sequence's
+ * blocks) and, if context_lens is not NULL, their lengths: the inputs of
+ * pa_paged_attention_decode once copied to the device.  PA_ERR_UNSUPPORTED if
+ * a table is wider than max_blocks_per_seq. */
+int pa_bm_block_tables(const pa_block_manager* bm, const int64_t* seq_ids, int64_t n,
+                       int max_blocks_per_seq, int32_t* tables, int32_t* context_lens);
+
+/* The free list in hand-out order: the first min(cap, free) ids into out,
+ * the number of free blocks into *n. */
+int pa_bm_free_list(const pa_block_manager* bm, int64_t* out, int64_t cap, int64_t* n);
+
+/*
  * pa_paged_attention_decode_static_scratch -- pa_paged_attention_decode for
  * callers that cannot allocate device memory.  The pages have no counterpart:
  * this is a deployment convenience of this library.

@@ -45,6 +45,18 @@ _SIGS = {
                                               _SZ, _P], _I),
     "pa_paged_attention_decode_static_scratch": ([_P, _P, _P, _P, _I, _P, _I, _F, _I, _P, _I, _I, _I, _I, _I, _I64,
                                                   _I, _I, _P], _I),
+    # host-side block manager (host pointers)
+    "pa_bm_create": ([_I64, _I], _P),
+    "pa_bm_destroy": ([_P], None),
+    "pa_bm_add_sequence": ([_P, _I64], _I),
+    "pa_bm_append_tokens": ([_P, _P, _I64, _P, _P, _P], _I),
+    "pa_bm_fork": ([_P, _I64, _I64], _I),
+    "pa_bm_free_sequence": ([_P, _I64], _I),
+    "pa_bm_num_free": ([_P], _I64),
+    "pa_bm_refcount": ([_P, _I64], _I),
+    "pa_bm_length": ([_P, _I64], _I64),
+    "pa_bm_block_tables": ([_P, _P, _I64, _I, _P, _P], _I),
+    "pa_bm_free_list": ([_P, _P, _I64, _P], _I),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)

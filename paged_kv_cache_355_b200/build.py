@@ -2,7 +2,7 @@
 
     python -m paged_kv_cache_355_b200.build [--force] [--verbose]
 
-Each csrc/*.cu is compiled separately (in parallel) with
+Each csrc/*.cu (and host-only csrc/*.cpp) is compiled separately (in parallel) with
 ``-gencode arch=compute_100a,code=sm_100a -O3 -lineinfo`` into _build/, then
 linked into paged_kv_cache_355_b200/libpa.so with the CUDA runtime linked
 statically, so the library does not depend on which libcudart the host
@@ -37,7 +37,7 @@ def _nvcc() -> str:
 
 
 def _sources():
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
 def _headers():

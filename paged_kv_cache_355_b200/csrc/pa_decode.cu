@@ -19,7 +19,7 @@
 //    gathers 32 / block_size physical blocks into one contiguous 32-token
 //    tile, so the math never depends on block_size.  Full/empty mbarriers
 //    hand stages to the consumers and back.
-//  * Warps 1..4 are consumers.  Stage j goes to consumer warp j % 4, which
+//  * Warps 1..2 are consumers.  Stage j goes to consumer warp j % 2, which
 //    keeps its own fp32 online-softmax state (running max m, running sum l,
 //    output accumulator o) for all G = Hq / Hkv query heads of the kv head:
 //    every K and V element loaded from shared memory is used by all G heads.
@@ -54,13 +54,13 @@
 namespace pa {
 namespace {
 
-constexpr int kConsumerWarps = 4;
+constexpr int kConsumerWarps = 2;
 constexpr int kDecodeThreads = 32 * (1 + kConsumerWarps);
 constexpr int kStageTokens = 32;
 constexpr int kMaxPartition = 8192;
 constexpr int kMinAutoPartition = 256;
-constexpr int kDefaultPartition = 2048;
-constexpr int kRingTargetBytes = 64 * 1024;
+constexpr int kBasePartition = 512;
+constexpr int kRingTargetBytes = 32 * 1024;
 constexpr int kMaxDynamicSmem = 200 * 1024;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -398,9 +398,9 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const Deco
     __syncthreads();  // pipeline drained: the ring is free for the merge scratch
     if (s_abort) return;
 
-    float* sm_o = reinterpret_cast<float*>(ring);    // [4][G][D]
-    float* sm_m = sm_o + kConsumerWarps * G * D;      // [4][G]
-    float* sm_l = sm_m + kConsumerWarps * G;          // [4][G]
+    float* sm_o = reinterpret_cast<float*>(ring);    // [warps][G][D]
+    float* sm_m = sm_o + kConsumerWarps * G * D;      // [warps][G]
+    float* sm_l = sm_m + kConsumerWarps * G;          // [warps][G]
     if (warp > 0 && grp == 0) {
         const int cw = warp - 1;
 #pragma unroll
@@ -723,9 +723,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
     __syncthreads();  // pipeline drained: the ring is free for the merge scratch
     if (s_abort) return;
 
-    float* sm_o = reinterpret_cast<float*>(ring);  // [4][G][D]
-    float* sm_m = sm_o + kConsumerWarps * G * D;    // [4][G]
-    float* sm_l = sm_m + kConsumerWarps * G;        // [4][G]
+    float* sm_o = reinterpret_cast<float*>(ring);  // [warps][G][D]
+    float* sm_m = sm_o + kConsumerWarps * G * D;    // [warps][G]
+    float* sm_l = sm_m + kConsumerWarps * G;        // [warps][G]
     if (warp > 0) {
         const int cw = warp - 1;
 #pragma unroll
@@ -815,12 +815,16 @@ struct Plan {
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-int auto_partition(int batch, int num_kv_heads, int max_context_len) {
-    // 2048 tokens per split (measured best on the B200 for batch >= 16 from
-    // 1k to 128k tokens: fewer, longer work items keep each CTA's TMA ring
-    // streaming and make the merge pass rare); halved while the grid would
-    // hold fewer than four work items per SM.
-    int P = kDefaultPartition;
+int auto_partition(int batch, int num_q_heads, int num_kv_heads, int max_context_len) {
+    // 512 tokens per split for groups of up to 4 query heads, 1024 for 8,
+    // 2048 for 16: each split of a kv head writes and re-reads G partial rows
+    // of (D + 2) fp32 values, about G / partition of the K/V bytes it reads,
+    // so larger groups want longer splits (measured on the B200 over batch
+    // 16..256 and lengths 128..128k).  Halved while the grid would hold fewer
+    // than four work items per SM.
+    const int G = num_q_heads / num_kv_heads;
+    int P = kBasePartition * (G > 4 ? G / 4 : 1);
+    if (P > kMaxPartition) P = kMaxPartition;
     const int64_t min_items = 4ll * num_sms();
     const int64_t L = max_context_len > 0 ? max_context_len : 1;
     while (P > kMinAutoPartition && (int64_t)batch * num_kv_heads * ((L + P - 1) / P) < min_items) P /= 2;
@@ -830,7 +834,7 @@ int auto_partition(int batch, int num_kv_heads, int max_context_len) {
 int make_plan(int batch, int num_q_heads, int num_kv_heads, int head_dim, int max_context_len, int partition_size,
               Plan* plan) {
     int P = partition_size;
-    if (P == 0) P = auto_partition(batch, num_kv_heads, max_context_len);
+    if (P == 0) P = auto_partition(batch, num_q_heads, num_kv_heads, max_context_len);
     if (P < kStageTokens || P > kMaxPartition || P % kStageTokens != 0) return PA_ERR_INVALID_ARG;
     const int L = max_context_len > 0 ? max_context_len : 1;
     const int splits = (L + P - 1) / P;
@@ -941,13 +945,13 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
     if (!p.err) return PA_ERR_CUDA;
 
     const int stage_bytes = 2 * kStageTokens * head_dim * (int)dtype_bytes(kv_dtype);  // K + V
-    // Stage j lives in slot j % stages and is consumed by warp j % 4.  The
+    // Stage j lives in slot j % stages and is consumed by warp j % 2.  The
     // stage count must be a multiple of the consumer-warp count: then the
     // previous user of a slot is the same warp, so a warp never waits on a
     // full-barrier phase more than one ahead of the barrier's current phase
     // (a parity wait cannot tell phase k + 2 from phase k).
     int stages = (kRingTargetBytes / stage_bytes) / kConsumerWarps * kConsumerWarps;
-    stages = stages < kConsumerWarps ? kConsumerWarps : (stages > 2 * kConsumerWarps ? 2 * kConsumerWarps : stages);
+    stages = stages < kConsumerWarps ? kConsumerWarps : (stages > 4 * kConsumerWarps ? 4 * kConsumerWarps : stages);
     p.stages = stages;
     const int table_bytes = p.contiguous ? 0 : (plan.partition / p.block_size) * 4;
     p.ring_offset = (int)((16 * stages + table_bytes + 127) & ~127);
@@ -1016,7 +1020,7 @@ extern "C" int pa_paged_attention_partition_size(int batch, int num_q_heads, int
     if (!partition_size) return PA_ERR_INVALID_ARG;
     int rc = check_shapes(batch, num_q_heads, num_kv_heads, head_dim, block_size, PA_BF16, PA_F32, max_context_len);
     if (rc) return rc;
-    *partition_size = auto_partition(batch, num_kv_heads, max_context_len);
+    *partition_size = auto_partition(batch, num_q_heads, num_kv_heads, max_context_len);
     return PA_OK;
 }
 

@@ -1,0 +1,67 @@
+"""The capacity/waste simulation on the native block manager, checked
+against the oracle's allocator model and against closed forms."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+from oracle.block_manager import BlockManager as RefManager
+from oracle.block_manager import OutOfBlocks as RefOut
+
+
+@pytest.fixture(scope="module")
+def cap():
+    from paged_kv_cache_355_b200 import build
+
+    build.build()
+    from paged_kv_cache_355_b200 import capacity
+
+    return capacity
+
+
+def _ref_paged(lengths, pool_tokens, bs):
+    bm = RefManager(pool_tokens // bs, bs)
+    admitted = used = 0
+    for i, L in enumerate(lengths):
+        if -(-int(L) // bs) > len(bm.free):
+            break
+        try:
+            for _ in range(int(L)):
+                bm.append_token(i)
+        except RefOut:
+            bm.free_sequence(i)
+            break
+        admitted += 1
+        used += int(L)
+    reserved = (bm.num_blocks - len(bm.free)) * bs
+    return admitted, used, reserved
+
+
+@pytest.mark.parametrize("bs", [8, 16, 32])
+def test_paged_admission_matches_oracle_model(cap, bs):
+    lengths = cap.lognormal_lengths(300, 200.0, 0.8, 16, 1024, seed=bs)
+    got = cap.paged(lengths, 40000, bs)
+    assert (got["admitted"], got["used_tokens"], got["reserved_tokens"]) == _ref_paged(lengths, 40000, bs)
+
+
+def test_closed_forms(cap):
+    # one request of 100 tokens in a 4096-token reservation wastes 3996 / 4096
+    assert cap.contiguous([100], 4096, 4096)["waste"] == 3996 / 4096
+    # paging wastes less than one block per admitted sequence
+    lengths = cap.lognormal_lengths(2000, 1000.0, 0.8, 16, 4096, seed=3)
+    p = cap.paged(lengths, 1 << 20, 16)
+    assert p["reserved_tokens"] - p["used_tokens"] <= 15 * p["admitted"]
+    # contiguous admits exactly pool // max_model_len requests (when enough arrive)
+    assert cap.contiguous(lengths, 1 << 20, 4096)["admitted"] == (1 << 20) // 4096
+    # n samples without sharing hold the prompt n times
+    shared = cap.parallel_sampling_blocks(1000, 8, 16, True)
+    private = cap.parallel_sampling_blocks(1000, 8, 16, False)
+    assert shared == -(-1000 // 16) and private == 8 * shared
+
+
+def test_report_reproduces_the_pages_ranges(cap):
+    r = cap.report()
+    assert 0.6 <= r["contiguous"]["waste"] <= 0.8      # "~60-80 %" wasted by max-length reservation
+    assert r["paged"]["waste"] < 0.04                   # "under 4 %"
+    assert 2.0 <= r["batch_gain"] <= 4.0                # "2-4x larger batches"
+    assert r["prompt_blocks_n8_private"] == 8 * r["prompt_blocks_n8_shared"]
