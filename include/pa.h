@@ -139,6 +139,29 @@ int pa_copy_blocks(void* k_pool, void* v_pool, const int64_t* block_mapping, int
                    void* stream);
 
 /*
+ * pa_swap_blocks -- move whole blocks between two pools of the same shape
+ * except their block counts, typically a device pool and a pinned host pool
+ * (swap-out and swap-in when the scheduler preempts a sequence by swapping,
+ * [P1] "Key takeaways": the scheduler preempts by swapping or recomputing,
+ * and paging makes both finer-grained).
+ * For every pair p: dst block block_mapping[p][1] := src block
+ * block_mapping[p][0], K and V, bit-exact.
+ *   src_k, src_v  [src_num_blocks][num_kv_heads][block_size][head_dim]
+ *   dst_k, dst_v  [dst_num_blocks][...same...]
+ * Each pool pointer is device memory or pinned host memory that the device
+ * can address (cudaHostAlloc / torch pin_memory under unified addressing);
+ * one kernel moves all pairs, so a host-side pool is read or written across
+ * the host link without per-block copy calls.  block_mapping (int64
+ * [num_pairs][2]) must be device-addressable too.  Destinations must be
+ * distinct.  Ids outside their pool skip the pair and record
+ * PA_ERR_BAD_BLOCK_ID.
+ */
+int pa_swap_blocks(const void* src_k, const void* src_v, void* dst_k, void* dst_v,
+                   const int64_t* block_mapping, int64_t num_pairs, int num_kv_heads, int head_dim,
+                   int block_size, int64_t src_num_blocks, int64_t dst_num_blocks, int dtype,
+                   void* stream);
+
+/*
  * pa_paged_attention_partition_size -- tokens per KV split that
  * pa_paged_attention_decode uses for these sizes when called with
  * partition_size == 0 (a multiple of 32, at most 8192).  Sequences longer

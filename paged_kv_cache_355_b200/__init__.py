@@ -11,7 +11,8 @@ not been built (build it with ``python -m paged_kv_cache_355_b200.build``);
 there is no fallback implementation.
 """
 _BINDING_NAMES = (
-    "EXPORTED", "LIB_PATH", "PA_BF16", "PA_F32", "PAError", "pa_copy_blocks", "pa_decode_slot_mapping",
+    "EXPORTED", "LIB_PATH", "PA_BF16", "PA_F32", "PAError", "pa_copy_blocks", "pa_swap_blocks",
+    "pa_decode_slot_mapping",
     "pa_paged_attention_decode", "pa_paged_attention_decode_contiguous", "pa_paged_attention_partition_size",
     "pa_paged_attention_workspace_size", "pa_read_error_flag", "pa_reshape_and_cache", "pa_slot_mapping",
     "pa_status_string", "pa_version", "pa_paged_attention_decode_static_scratch", "STATIC_SCRATCH_BYTES",

@@ -37,6 +37,7 @@ _SIGS = {
     "pa_decode_slot_mapping": ([_P, _I, _P, _I, _I, _P, _P], _I),
     "pa_reshape_and_cache": ([_P, _P, _P, _P, _P, _I64, _I, _I, _I, _I64, _I, _P], _I),
     "pa_copy_blocks": ([_P, _P, _P, _I64, _I, _I, _I, _I64, _I, _P], _I),
+    "pa_swap_blocks": ([_P, _P, _P, _P, _P, _I64, _I, _I, _I, _I64, _I64, _I, _P], _I),
     "pa_paged_attention_partition_size": ([_I, _I, _I, _I, _I, _I, ctypes.POINTER(_I)], _I),
     "pa_paged_attention_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
     "pa_paged_attention_decode": ([_P, _P, _P, _P, _I, _P, _I, _F, _I, _P, _I, _I, _I, _I, _I, _I64, _I, _I, _P,
@@ -150,6 +151,32 @@ def pa_copy_blocks(k_pool, v_pool, block_mapping, stream=None) -> None:
     _check("pa_copy_blocks", _lib.pa_copy_blocks(
         _dev(k_pool, "k_pool"), v_pool.data_ptr(), _dev(block_mapping, "block_mapping", torch.int64), P, Hkv, D, bs,
         NB, _kv_dtype(k_pool), _stream(stream)))
+
+
+def _addr(t: torch.Tensor, name: str, dtype=None) -> int:
+    """Pointer of a CUDA tensor or of a pinned host tensor (device-addressable)."""
+    if not isinstance(t, torch.Tensor) or not (t.is_cuda or t.is_pinned()):
+        raise TypeError(f"{name} must be a CUDA tensor or a pinned host tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def pa_swap_blocks(src_k, src_v, dst_k, dst_v, block_mapping, stream=None) -> None:
+    """dst block m[p][1] := src block m[p][0] (K and V); pools on the device or
+    in pinned host memory, block_mapping likewise."""
+    sNB, Hkv, bs, D = src_k.shape
+    dNB = dst_k.shape[0]
+    if tuple(dst_k.shape[1:]) != (Hkv, bs, D) or src_v.shape != src_k.shape or dst_v.shape != dst_k.shape:
+        raise ValueError("pool shapes disagree")
+    for t, n in ((src_v, "src_v"), (dst_k, "dst_k"), (dst_v, "dst_v")):
+        _addr(t, n, src_k.dtype)
+    _check("pa_swap_blocks", _lib.pa_swap_blocks(
+        _addr(src_k, "src_k"), src_v.data_ptr(), dst_k.data_ptr(), dst_v.data_ptr(),
+        _addr(block_mapping, "block_mapping", torch.int64), block_mapping.numel() // 2, Hkv, D, bs, sNB, dNB,
+        _kv_dtype(src_k), _stream(stream)))
 
 
 def pa_paged_attention_partition_size(batch, num_q_heads, num_kv_heads, head_dim, max_context_len,

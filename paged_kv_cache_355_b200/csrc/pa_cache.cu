@@ -1,9 +1,10 @@
 // pa_cache.cu -- the kernels that feed the KV pool: slot mapping,
-// reshape_and_cache (write a new token's K/V into its slot) and copy_blocks
-// (copy-on-write duplication of a shared block).
+// reshape_and_cache (write a new token's K/V into its slot), copy_blocks
+// (copy-on-write duplication of a shared block) and swap_blocks (whole blocks
+// between a device pool and a pinned host pool, for preemption by swapping).
 //
-// All three are bit copies or integer index work, bound by latency (tiny
-// per-step sizes) or by HBM bandwidth (copy_blocks).  Each moves 16-byte
+// All are bit copies or integer index work, bound by latency (tiny per-step
+// sizes), by HBM bandwidth (copy_blocks) or by the host link (swap_blocks).  Each moves 16-byte
 // vectors: one (token, kv head) row of head_dim elements is head_dim *
 // elt / 16 vectors (8 to 32), contiguous in both source and destination.
 #include <cuda_runtime.h>
@@ -87,27 +88,61 @@ __global__ void reshape_and_cache_kernel(const uint4* __restrict__ key, const ui
 }
 
 // blockIdx.x = pair; blockIdx.y strides over the block's 16-byte vectors.
-__global__ void copy_blocks_kernel(uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
-                                   const int64_t* __restrict__ block_mapping, int64_t num_blocks,
-                                   int64_t block_vecs, int* err) {
+// Source and destination pools may be the same pool (copy-on-write) or two
+// pools, one of them in pinned host memory mapped into the device address
+// space (swap).  Each thread keeps four 16-byte loads in flight so that a
+// source across PCIe still sees enough outstanding requests.
+__global__ void copy_blocks_kernel(const uint4* src_k, const uint4* src_v, uint4* dst_k, uint4* dst_v,
+                                   const int64_t* __restrict__ block_mapping, int64_t src_num_blocks,
+                                   int64_t dst_num_blocks, int64_t block_vecs, int* err) {
+    constexpr int kUnroll = 4;
     const int64_t p = blockIdx.x;
     const int64_t src = block_mapping[2 * p];
     const int64_t dst = block_mapping[2 * p + 1];
-    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+    if (src < 0 || src >= src_num_blocks || dst < 0 || dst >= dst_num_blocks) {
         if (threadIdx.x == 0 && blockIdx.y == 0) record_error(err, PA_ERR_BAD_BLOCK_ID);
         return;
     }
-    const uint4* ks = k_pool + src * block_vecs;
-    const uint4* vs = v_pool + src * block_vecs;
-    uint4* kd = k_pool + dst * block_vecs;
-    uint4* vd = v_pool + dst * block_vecs;
-    for (int64_t i = blockIdx.y * (int64_t)blockDim.x + threadIdx.x; i < block_vecs;
-         i += (int64_t)gridDim.y * blockDim.x) {
-        const uint4 a = ks[i];
-        const uint4 b = vs[i];
-        kd[i] = a;
-        vd[i] = b;
+    const uint4* ks = src_k + src * block_vecs;
+    const uint4* vs = src_v + src * block_vecs;
+    uint4* kd = dst_k + dst * block_vecs;
+    uint4* vd = dst_v + dst * block_vecs;
+    const int64_t step = (int64_t)gridDim.y * blockDim.x;
+    for (int64_t i0 = blockIdx.y * (int64_t)blockDim.x + threadIdx.x; i0 < block_vecs; i0 += step * kUnroll) {
+        uint4 a[kUnroll], b[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t i = i0 + u * step;
+            if (i < block_vecs) {
+                a[u] = ks[i];
+                b[u] = vs[i];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t i = i0 + u * step;
+            if (i < block_vecs) {
+                kd[i] = a[u];
+                vd[i] = b[u];
+            }
+        }
     }
+}
+
+int launch_copy(const void* src_k, const void* src_v, void* dst_k, void* dst_v, const int64_t* block_mapping,
+                int64_t num_pairs, int num_kv_heads, int head_dim, int block_size, int64_t src_num_blocks,
+                int64_t dst_num_blocks, int dtype, void* stream) {
+    int* err = error_word_ptr();
+    if (!err) return PA_ERR_CUDA;
+    const int64_t block_vecs = (int64_t)num_kv_heads * block_size * head_dim * (int64_t)dtype_bytes(dtype) / 16;
+    int64_t slices = (block_vecs + kThreads * 4 - 1) / (kThreads * 4);
+    if (slices > 64) slices = 64;
+    if (slices < 1) slices = 1;
+    dim3 grid((unsigned)num_pairs, (unsigned)slices);
+    copy_blocks_kernel<<<grid, kThreads, 0, (cudaStream_t)stream>>>(
+        static_cast<const uint4*>(src_k), static_cast<const uint4*>(src_v), static_cast<uint4*>(dst_k),
+        static_cast<uint4*>(dst_v), block_mapping, src_num_blocks, dst_num_blocks, block_vecs, err);
+    return launch_status();
 }
 
 inline int grid_for(int64_t work) {
@@ -180,14 +215,22 @@ extern "C" int pa_copy_blocks(void* k_pool, void* v_pool, const int64_t* block_m
     if (num_pairs == 0) return PA_OK;
     if (num_pairs > 0x7fffffff) return PA_ERR_INVALID_ARG;
     if (!k_pool || !v_pool || !block_mapping || !aligned16(k_pool) || !aligned16(v_pool)) return PA_ERR_INVALID_ARG;
-    int* err = error_word_ptr();
-    if (!err) return PA_ERR_CUDA;
-    const int64_t block_vecs = (int64_t)num_kv_heads * block_size * head_dim * (int64_t)dtype_bytes(dtype) / 16;
-    int64_t slices = (block_vecs + kThreads * 4 - 1) / (kThreads * 4);
-    if (slices > 64) slices = 64;
-    if (slices < 1) slices = 1;
-    dim3 grid((unsigned)num_pairs, (unsigned)slices);
-    copy_blocks_kernel<<<grid, kThreads, 0, (cudaStream_t)stream>>>(
-        static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), block_mapping, num_blocks, block_vecs, err);
-    return launch_status();
+    return launch_copy(k_pool, v_pool, k_pool, v_pool, block_mapping, num_pairs, num_kv_heads, head_dim, block_size,
+                       num_blocks, num_blocks, dtype, stream);
+}
+
+extern "C" int pa_swap_blocks(const void* src_k, const void* src_v, void* dst_k, void* dst_v,
+                              const int64_t* block_mapping, int64_t num_pairs, int num_kv_heads, int head_dim,
+                              int block_size, int64_t src_num_blocks, int64_t dst_num_blocks, int dtype,
+                              void* stream) {
+    if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || src_num_blocks < 0 ||
+        dst_num_blocks < 0 || !valid_dtype(dtype))
+        return PA_ERR_INVALID_ARG;
+    if (!supported_head_dim(head_dim) || !supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
+    if (num_pairs == 0) return PA_OK;
+    if (num_pairs > 0x7fffffff) return PA_ERR_INVALID_ARG;
+    if (!src_k || !src_v || !dst_k || !dst_v || !block_mapping) return PA_ERR_INVALID_ARG;
+    if (!aligned16(src_k) || !aligned16(src_v) || !aligned16(dst_k) || !aligned16(dst_v)) return PA_ERR_INVALID_ARG;
+    return launch_copy(src_k, src_v, dst_k, dst_v, block_mapping, num_pairs, num_kv_heads, head_dim, block_size,
+                       src_num_blocks, dst_num_blocks, dtype, stream);
 }

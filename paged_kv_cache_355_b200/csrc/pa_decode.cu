@@ -58,8 +58,10 @@ constexpr int kConsumerWarps = 2;
 constexpr int kDecodeThreads = 32 * (1 + kConsumerWarps);
 constexpr int kStageTokens = 32;
 constexpr int kMaxPartition = 8192;
-constexpr int kMinAutoPartition = 256;
-constexpr int kBasePartition = 512;
+constexpr int kMinAutoPartition = 512;
+constexpr int kMaxAutoPartition = 4096;
+constexpr int kCtasPerSmEstimate = 6;  // resident pass-1 CTAs per SM (34 KB of shared memory each)
+constexpr int kLongestFirstMaxBatch = 2048;  // O(batch) per CTA for the launch order
 constexpr int kRingTargetBytes = 32 * 1024;
 constexpr int kMaxDynamicSmem = 200 * 1024;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -87,6 +89,8 @@ struct DecodeParams {
     int ring_offset;
     int out_bf16;
     int contiguous;
+    int batch;
+    int longest_first;  // blockIdx.z is a rank in decreasing-length order
     float scale_log2;
 };
 
@@ -173,6 +177,67 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeParams& p, con
     }
 }
 
+// Longest-first launch order.  The hardware dispatches CTAs in the order of
+// their linear index, so the grid's z coordinate is used as a rank: the CTA
+// works on the sequence with that rank when sequences are ordered by
+// decreasing length (64 length buckets, ties by index).  This is
+// longest-processing-time-first list scheduling; it keeps the tail of the
+// grid short when lengths vary.  All threads read each length once into a
+// shared-memory key and a bucket histogram; then one warp walks the keys in
+// index order, placing each lane among equal keys with match_any (a counting
+// sort, O(batch) shared-memory work).  `scratch` is shared memory that is
+// free at this point (at least 512 + batch bytes).  With longest_first == 0
+// the rank is the sequence index.
+__device__ __forceinline__ int schedule_sequence(const DecodeParams& p, uint8_t* scratch) {
+    const int rank = blockIdx.z;
+    if (!p.longest_first) return rank;
+    __shared__ int s_seq;
+    int* hist = reinterpret_cast<int*>(scratch);  // [64], then running positions [64]
+    int* run = hist + 64;
+    uint8_t* key = scratch + 512;                 // [batch]
+    const int tid = threadIdx.x;
+    for (int k = tid; k < 64; k += blockDim.x) hist[k] = 0;
+    if (tid == 0) s_seq = rank;
+    __syncthreads();
+    for (int b = tid; b < p.batch; b += blockDim.x) {
+        int L = p.context_lens[b];
+        L = L < 0 ? 0 : ((int64_t)L > p.max_len ? (int)p.max_len : L);
+        int k = (int)(((int64_t)L * 64) / (p.max_len + 1));
+        k = 63 - (k > 63 ? 63 : k);  // longer sequences get lower keys
+        key[b] = (uint8_t)k;
+        atomicAdd(&hist[k], 1);
+    }
+    __syncthreads();
+    if (tid < 32) {
+        const int lane = tid;
+        const int a0 = hist[2 * lane], a1 = hist[2 * lane + 1];
+        int incl = a0 + a1;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        const int excl = incl - a0 - a1;
+        run[2 * lane] = excl;
+        run[2 * lane + 1] = excl + a0;
+        __syncwarp();
+        for (int c = 0; c < p.batch; c += 32) {
+            const int b = c + lane;
+            const bool valid = b < p.batch;
+            const int k = valid ? key[b] : 64 + lane;
+            const unsigned peers = __match_any_sync(0xffffffffu, k);
+            const int before = __popc(peers & ((1u << lane) - 1u));
+            const int pos = valid ? run[k] + before : -1;
+            __syncwarp();
+            if (valid && before == 0) run[k] += __popc(peers);
+            if (pos == rank) s_seq = b;
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+    return s_seq;
+}
+
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const DecodeParams p) {
     using E = Elt<T>;
@@ -196,7 +261,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const Deco
 
     const int split = blockIdx.x;
     const int kvh = blockIdx.y;
-    const int b = blockIdx.z;
+    const int b = schedule_sequence(p, ring);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
@@ -461,7 +526,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
 
     const int split = blockIdx.x;
     const int kvh = blockIdx.y;
-    const int b = blockIdx.z;
+    const int b = schedule_sequence(p, ring);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int G = p.num_q_heads / p.num_kv_heads;
@@ -756,50 +821,60 @@ __global__ void __launch_bounds__(kDecodeThreads)
 }
 
 // Second pass: out = sum_s w_s o_s / sum_s w_s with w_s = l_s * 2^(m_s - max m),
-// for sequences that were cut into more than one split.  One CTA per
-// (sequence, query head), one thread per output element; fixed summation
-// order.
+// for sequences that were cut into more than one split.  One warp per
+// (sequence, query head) row, eight rows per CTA: lane s loads split s's
+// (m, l), the max and the sum are warp shuffles, and lane i accumulates
+// output elements [i * D / 32, (i + 1) * D / 32) over the splits in order
+// (deterministic, no shared memory, no block barrier).
+constexpr int kMergeWarps = 8;
+
 template <int D>
-__global__ void __launch_bounds__(D) decode_merge_kernel(const DecodeParams p) {
-    extern __shared__ float wts[];  // [max_splits]
-    __shared__ float red[D / 32];
-    const int64_t row = blockIdx.x;  // b * Hq + h
+__global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(const DecodeParams p, int64_t rows) {
+    constexpr int VPL = D / 32;  // output elements per lane
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);  // b * Hq + h
+    if (row >= rows) return;
     const int b = (int)(row / p.num_q_heads);
     const int L = clamp_len(p, b, false);
     const int ns = L > 0 ? (L + p.partition - 1) / p.partition : 1;
     if (ns <= 1) return;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const float* ml = p.part_ml + row * p.max_splits * 2;
+    const float* po = p.part_o + row * p.max_splits * D + lane * VPL;
 
-    float mx = -INFINITY;
-    for (int s = tid; s < ns; s += D) mx = fmaxf(mx, ml[2 * s]);
+    float M = -INFINITY;
+    for (int s = lane; s < ns; s += 32) M = fmaxf(M, ml[2 * s]);
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    if (lane == 0) red[warp] = mx;
-    __syncthreads();
-    float M = red[0];
-#pragma unroll
-    for (int w = 1; w < D / 32; ++w) M = fmaxf(M, red[w]);
-    __syncthreads();
+    for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
 
-    float sum = 0.f;
-    for (int s = tid; s < ns; s += D) {
-        const float w = ml[2 * s + 1] * exp2f(ml[2 * s] - M);
-        wts[s] = w;
-        sum += w;
+    float acc[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
+    float W = 0.f;
+    for (int s0 = 0; s0 < ns; s0 += 32) {
+        const int s = s0 + lane;
+        const float w = s < ns ? ml[2 * s + 1] * exp2f(ml[2 * s] - M) : 0.f;
+        W += w;
+        const int n = min(32, ns - s0);
+        for (int k = 0; k < n; ++k) {
+            const float wk = __shfl_sync(0xffffffffu, w, k);
+            const float* src = po + (int64_t)(s0 + k) * D;
+            if constexpr (VPL == 4) {
+                const float4 v = *reinterpret_cast<const float4*>(src);
+                acc[0] = fmaf(wk, v.x, acc[0]);
+                acc[1] = fmaf(wk, v.y, acc[1]);
+                acc[2] = fmaf(wk, v.z, acc[2]);
+                acc[3] = fmaf(wk, v.w, acc[3]);
+            } else {
+                const float2 v = *reinterpret_cast<const float2*>(src);
+                acc[0] = fmaf(wk, v.x, acc[0]);
+                acc[1] = fmaf(wk, v.y, acc[1]);
+            }
+        }
     }
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-    if (lane == 0) red[warp] = sum;
-    __syncthreads();
-    float W = 0.f;
+    for (int off = 16; off >= 1; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
 #pragma unroll
-    for (int w = 0; w < D / 32; ++w) W += red[w];
-
-    const float* po = p.part_o + row * p.max_splits * D;
-    float acc = 0.f;
-    for (int s = 0; s < ns; ++s) acc = fmaf(wts[s], po[(int64_t)s * D + tid], acc);
-    store_out(p, row * D + tid, W > 0.f ? acc / W : 0.f);
+    for (int i = 0; i < VPL; ++i) store_out(p, row * D + lane * VPL + i, W > 0.f ? acc[i] / W : 0.f);
 }
 
 // ---------------------------------------------------------------------------
@@ -816,18 +891,17 @@ struct Plan {
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 int auto_partition(int batch, int num_q_heads, int num_kv_heads, int max_context_len) {
-    // 512 tokens per split for groups of up to 4 query heads, 1024 for 8,
-    // 2048 for 16: each split of a kv head writes and re-reads G partial rows
-    // of (D + 2) fp32 values, about G / partition of the K/V bytes it reads,
-    // so larger groups want longer splits (measured on the B200 over batch
-    // 16..256 and lengths 128..128k).  Halved while the grid would hold fewer
-    // than four work items per SM.
-    const int G = num_q_heads / num_kv_heads;
-    int P = kBasePartition * (G > 4 ? G / 4 : 1);
-    if (P > kMaxPartition) P = kMaxPartition;
-    const int64_t min_items = 4ll * num_sms();
+    // With longest-first launch order, long work items cost nothing in the
+    // tail while each split adds a CTA start-up and G partial rows to write
+    // and merge; so the partition is as long as possible (4096 tokens) while
+    // the grid still holds two waves of work items (counted as if every
+    // sequence had max_context_len tokens), halved down to 512 otherwise.
+    // Measured on the B200 over batch 1..256, groups 1..8, lengths 128..128k.
+    (void)num_q_heads;
+    int P = kMaxAutoPartition;
+    const int64_t waves = 2ll * num_sms() * kCtasPerSmEstimate;
     const int64_t L = max_context_len > 0 ? max_context_len : 1;
-    while (P > kMinAutoPartition && (int64_t)batch * num_kv_heads * ((L + P - 1) / P) < min_items) P /= 2;
+    while (P > kMinAutoPartition && (int64_t)batch * num_kv_heads * ((L + P - 1) / P) < waves) P /= 2;
     return P;
 }
 
@@ -941,6 +1015,8 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
     }
     p.partition = plan.partition;
     p.max_splits = plan.max_splits;
+    p.batch = batch;
+    p.longest_first = batch <= kLongestFirstMaxBatch;
     p.err = error_word_ptr();
     if (!p.err) return PA_ERR_CUDA;
 
@@ -985,13 +1061,12 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
     }
     if (rc) return rc;
     if (plan.max_splits > 1) {
-        const size_t msmem = (size_t)plan.max_splits * sizeof(float);
-        if (msmem > 48 * 1024) return PA_ERR_UNSUPPORTED;
-        const unsigned rows = (unsigned)((int64_t)batch * p.num_q_heads);
+        const int64_t rows = (int64_t)batch * p.num_q_heads;
+        const unsigned blocks = (unsigned)((rows + kMergeWarps - 1) / kMergeWarps);
         if (head_dim == 128)
-            decode_merge_kernel<128><<<rows, 128, msmem, st>>>(p);
+            decode_merge_kernel<128><<<blocks, 32 * kMergeWarps, 0, st>>>(p, rows);
         else
-            decode_merge_kernel<64><<<rows, 64, msmem, st>>>(p);
+            decode_merge_kernel<64><<<blocks, 32 * kMergeWarps, 0, st>>>(p, rows);
         rc = launch_status();
     }
     return rc;

@@ -116,3 +116,54 @@ def test_copy_blocks_flags_bad_pair(pa):
     pa.pa_copy_blocks(k_pool, v_pool, torch.tensor([[0, 9], [1, 2]], dtype=torch.int64, device="cuda"))
     assert pa.pa_read_error_flag() == 5
     assert torch.equal(k_pool[2], before[1]) and torch.equal(k_pool[0], before[0])
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_swap_out_and_in_through_pinned_host_memory(pa, dtype):
+    """Blocks swapped to a pinned host pool and back are bit-identical, and the
+    host pool holds exactly the swapped blocks (oracle: a numpy copy)."""
+    g = torch.Generator().manual_seed(7)
+    NB, HNB, Hkv, bs, D = 64, 24, 8, 16, 128
+    k = torch.randn(NB, Hkv, bs, D, generator=g).to(DT[dtype]).cuda()
+    v = torch.randn(NB, Hkv, bs, D, generator=g).to(DT[dtype]).cuda()
+    hk = torch.zeros(HNB, Hkv, bs, D, dtype=DT[dtype]).pin_memory()
+    hv = torch.zeros(HNB, Hkv, bs, D, dtype=DT[dtype]).pin_memory()
+    src = torch.randperm(NB, generator=g)[:20]
+    dst = torch.randperm(HNB, generator=g)[:20]
+    out_map = torch.stack([src, dst], 1).to(torch.int64)
+    k0, v0 = k.clone(), v.clone()
+    pa.pa_swap_blocks(k, v, hk, hv, out_map.cuda())  # swap out: device -> host
+    torch.cuda.synchronize()
+    want_k, want_v = np.zeros_like(np_of(hk)), np.zeros_like(np_of(hv))
+    want_k[np_of(dst)] = np_of(k0)[np_of(src)]
+    want_v[np_of(dst)] = np_of(v0)[np_of(src)]
+    assert np_of(hk).tobytes() == want_k.tobytes() and np_of(hv).tobytes() == want_v.tobytes()
+    k[src] = 0  # the device blocks are reused by someone else meanwhile
+    v[src] = 0
+    new_home = torch.randperm(NB, generator=g)[:20]
+    in_map = torch.stack([dst, new_home], 1).to(torch.int64).pin_memory()  # mapping read from host memory too
+    pa.pa_swap_blocks(hk, hv, k, v, in_map)  # swap in: host -> device, to new block ids
+    torch.cuda.synchronize()
+    assert torch.equal(k[new_home].cpu(), k0[src].cpu()) and torch.equal(v[new_home].cpu(), v0[src].cpu())
+    assert pa.pa_read_error_flag() == 0
+
+
+def test_swap_bandwidth_is_reported(pa):
+    """Swap 2048 blocks (256 MiB of K+V at 8 heads, bs 16, D 128, bf16) each
+    way and print the achieved host-link bandwidth (no bound asserted)."""
+    NB, Hkv, bs, D = 2048, 8, 16, 128
+    k = torch.empty(NB, Hkv, bs, D, dtype=torch.bfloat16, device="cuda").normal_()
+    v = torch.empty_like(k).normal_()
+    hk = torch.empty(NB, Hkv, bs, D, dtype=torch.bfloat16).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    m = torch.stack([torch.arange(NB), torch.randperm(NB)], 1).to(torch.int64).cuda()
+    nbytes = 2 * k.numel() * k.element_size()
+    for name, args in (("device->host", (k, v, hk, hv)), ("host->device", (hk, hv, k, v))):
+        pa.pa_swap_blocks(*args, m)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        pa.pa_swap_blocks(*args, m)
+        e1.record()
+        torch.cuda.synchronize()
+        print(f"swap {name}: {nbytes / e0.elapsed_time(e1) / 1e6:.1f} GB/s")
+    assert pa.pa_read_error_flag() == 0
