@@ -63,6 +63,7 @@ def _load():
             lib.oracle_paged_decode.argtypes = [P, P, P, P, i32, P, f32, i32, i32, i32, i32, i32, i64, i32, P]
             lib.oracle_paged_decode_rows.argtypes = [P, P, P, P, i32, P, f32, i32, i32, i32, i32, i32, i64, i32, P, P, i64, P]
             lib.oracle_contiguous_decode.argtypes = [P, P, P, i32, P, f32, i32, i32, i32, i32, i32, P]
+            lib.oracle_paged_prefill.argtypes = [P, P, P, P, i32, P, P, f32, i32, i32, i32, i32, i32, i64, i32, P]
             lib.oracle_slot_mapping.argtypes = [P, i32, i32, P, P, i64, i32, P]
             lib.oracle_reshape_and_cache.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i32]
             lib.oracle_copy_blocks.argtypes = [P, P, P, i64, i32, i32, i32, i64, i32]
@@ -70,6 +71,7 @@ def _load():
             lib.oracle_round_bf16.restype = None
             lib.oracle_num_threads.argtypes = []
             for name in ("oracle_paged_decode", "oracle_paged_decode_rows", "oracle_contiguous_decode",
+                         "oracle_paged_prefill",
                          "oracle_slot_mapping", "oracle_reshape_and_cache", "oracle_copy_blocks",
                          "oracle_num_threads"):
                 getattr(lib, name).restype = ctypes.c_int
@@ -131,6 +133,23 @@ def paged_decode_rows(q, k_pool, v_pool, block_tables, context_lens, scale, bloc
                                           _ptr(rb), _ptr(rh), rb.shape[0], _ptr(out))
     if rc:
         raise ValueError("oracle_paged_decode_rows rejected its arguments")
+    return out
+
+
+def paged_prefill(q, k_pool, v_pool, block_tables, context_lens, query_start, scale, block_size):
+    """Causal multi-query attention, float64 [T, Hq, D]; sequence b owns query
+    rows query_start[b] .. query_start[b + 1] - 1, its last tokens."""
+    q, k_pool, v_pool = _c(q), _c(k_pool), _c(v_pool)
+    bt, lens, qs = _c(block_tables, np.int32), _c(context_lens, np.int32), _c(query_start, np.int32)
+    dt = _dtype_code(q)
+    T, Hq, D = q.shape
+    NB, Hkv, bs, _ = k_pool.shape
+    assert bs == block_size and qs.shape[0] == lens.shape[0] + 1 and qs[-1] == T
+    out = np.zeros((T, Hq, D), np.float64)
+    rc = _load().oracle_paged_prefill(_ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(bt), bt.shape[1], _ptr(lens), _ptr(qs),
+                                      float(np.float32(scale)), block_size, lens.shape[0], Hq, Hkv, D, NB, dt, _ptr(out))
+    if rc:
+        raise ValueError("oracle_paged_prefill rejected its arguments")
     return out
 
 

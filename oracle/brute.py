@@ -61,3 +61,26 @@ def decode_logical(q, keys, values, scale: float):
             rows.append(attend_logical(q_b[h], ks, vs, scale))
         out.append(rows)
     return out
+
+
+def prefill_logical(q, keys, values, scale: float):
+    """Causal multi-query attention over logical lists.
+
+    q[b] is a list of query tokens, each a list over query heads of D floats;
+    they are the last len(q[b]) tokens of sequence b (whose keys/values are
+    keys[b][t][kvh]).  Query i sits at position L - n + i and sees tokens
+    0..that position.  Returns out[b][i][h].
+    """
+    out = []
+    for b, qb in enumerate(q):
+        L, n = len(keys[b]), len(qb)
+        rows = []
+        for i, qtok in enumerate(qb):
+            pos = L - n + i
+            Hq = len(qtok)
+            Hkv = len(keys[b][0])
+            G = Hq // Hkv
+            rows.append([attend_logical(qtok[h], [tok[h // G] for tok in keys[b][: pos + 1]],
+                                        [tok[h // G] for tok in values[b][: pos + 1]], scale) for h in range(Hq)])
+        out.append(rows)
+    return out

@@ -25,6 +25,12 @@
  *      heads share a kv head; the pages are silent on grouped heads).
  *      A sequence of length 0 yields a zero row.
  *
+ *  - oracle_paged_prefill
+ *      several new query tokens per sequence over the same paged cache
+ *      (chunked prefill): a sequence of length L with n new queries has query
+ *      i (0-based) at position p = L - n + i, attending keys 0..p (causal);
+ *      each query row is the attention above with the first p + 1 tokens.
+ *
  *  - oracle_contiguous_decode
  *      the same attention over a contiguous [B, Hkv, L_pad, D] cache, the
  *      "ideal contiguous attention" the same section compares against.
@@ -212,6 +218,54 @@ int oracle_paged_decode(const void* q, const void* k_pool, const void* v_pool,
                 const int h = kvh * G + g;
                 for (int d = 0; d < D; ++d) qrow[d] = widen(q, ((int64_t)b * Hq + h) * D + d, dtype);
                 bad |= attend(qrow, Kc, Vc, L, D, (double)scale, out + ((int64_t)b * Hq + h) * D);
+            }
+        }
+        free(Kc);
+        free(Vc);
+        free(qrow);
+    }
+    return bad;
+}
+
+/* Causal multi-query attention.  q and out rows: [T, Hq, D] with sequence b
+ * owning rows query_start[b] .. query_start[b + 1] - 1, its last n_b tokens. */
+int oracle_paged_prefill(const void* q, const void* k_pool, const void* v_pool,
+                         const int32_t* block_tables, int max_blocks_per_seq,
+                         const int32_t* context_lens, const int32_t* query_start, float scale,
+                         int block_size, int batch, int Hq, int Hkv, int D, int64_t num_blocks,
+                         int dtype, double* out) {
+    if (check_common(batch, Hq, Hkv, D, dtype) || block_size <= 0 || max_blocks_per_seq < 0)
+        return 1;
+    for (int b = 0; b < batch; ++b) {
+        const int64_t L = context_lens[b];
+        const int64_t n = (int64_t)query_start[b + 1] - query_start[b];
+        if (L < 0 || L > (int64_t)max_blocks_per_seq * block_size || n < 0 || n > L) return 1;
+    }
+    const int G = Hq / Hkv;
+    const int64_t tasks = (int64_t)batch * Hkv;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int64_t task = 0; task < tasks; ++task) {
+        const int b = (int)(task / Hkv), kvh = (int)(task % Hkv);
+        const int64_t L = context_lens[b];
+        const int64_t n = (int64_t)query_start[b + 1] - query_start[b];
+        double* Kc = (double*)malloc((size_t)(L > 0 ? L : 1) * D * sizeof(double));
+        double* Vc = (double*)malloc((size_t)(L > 0 ? L : 1) * D * sizeof(double));
+        double* qrow = (double*)malloc((size_t)D * sizeof(double));
+        if (!Kc || !Vc || !qrow) {
+            bad |= 1;
+        } else if (gather_paged(k_pool, v_pool, block_tables + (int64_t)b * max_blocks_per_seq,
+                                L, kvh, Hkv, block_size, D, num_blocks, dtype, Kc, Vc)) {
+            bad |= 1;
+        } else {
+            for (int64_t i = 0; i < n; ++i) {
+                const int64_t pos = L - n + i;
+                const int64_t row = query_start[b] + i;
+                for (int g = 0; g < G; ++g) {
+                    const int h = kvh * G + g;
+                    for (int d = 0; d < D; ++d) qrow[d] = widen(q, (row * Hq + h) * D + d, dtype);
+                    bad |= attend(qrow, Kc, Vc, pos + 1, D, (double)scale, out + (row * Hq + h) * D);
+                }
             }
         }
         free(Kc);

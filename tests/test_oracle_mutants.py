@@ -33,6 +33,9 @@ MUTANTS = {
                                    "memcpy((char*)v_pool + dst * row_bytes, (const char*)key + src * row_bytes, row_bytes);"),
     "copy_blocks_skips_v": ("memmove((char*)v_pool + dst * block_bytes, (const char*)v_pool + src * block_bytes, block_bytes);", ""),
     "bf16_rounds_one_bit_short": ("int qexp = e - 8;", "int qexp = e - 7;"),
+    "prefill_causal_excludes_self": ("bad |= attend(qrow, Kc, Vc, pos + 1, D,", "bad |= attend(qrow, Kc, Vc, pos, D,"),
+    "prefill_causal_sees_one_ahead": ("bad |= attend(qrow, Kc, Vc, pos + 1, D,", "bad |= attend(qrow, Kc, Vc, pos + 2 > L ? L : pos + 2, D,"),
+    "prefill_query_position_from_start": ("const int64_t pos = L - n + i;", "const int64_t pos = i;"),
 }
 
 
@@ -47,7 +50,8 @@ def test_pins_catch_planted_mistake(name, tmp_path):
     subprocess.run(["gcc", "-O2", "-ffp-contract=off", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", str(lib),
                     str(mutant), "-lm"], check=True)
     env = dict(os.environ, PA_ORACLE_LIB=str(lib), OMP_NUM_THREADS="2")
-    pins = [os.path.join(ROOT, "tests", f) for f in ("test_oracle_pins.py", "test_oracle_cache_ops.py")]
+    pins = [os.path.join(ROOT, "tests", f) for f in ("test_oracle_pins.py", "test_oracle_cache_ops.py",
+                                                      "test_oracle_prefill.py")]
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider", *pins],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
