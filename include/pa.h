@@ -212,6 +212,34 @@ int pa_paged_attention_decode(const void* q, const void* k_pool, const void* v_p
                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * pa_paged_attention_prefill -- causal attention for several new query
+ * tokens per sequence over the paged cache (chunked prefill, or speculative
+ * tokens): the multi-query form of pa_paged_attention_decode, reading K and V
+ * through the block table in the same way ([P1] "The kernel side").
+ * Sequence b of length L = context_lens[b] (counting its new tokens, whose
+ * K/V must already be in the pool) owns query rows query_start[b] ..
+ * query_start[b + 1] - 1, its last n = query_start[b + 1] - query_start[b]
+ * tokens; row i sits at position p = L - n + i and attends keys 0..p:
+ *   out[r][h] = sum_{t <= p} softmax_t(scale * <q[r][h], K_t>) V_t.
+ *   q             [num_tokens][num_q_heads][head_dim] bf16
+ *   query_start   int32 [batch + 1], non-decreasing, query_start[0] = 0,
+ *                 query_start[batch] = num_tokens
+ *   max_query_len host-side upper bound of the n (sizes the grid)
+ *   out           [num_tokens][num_q_heads][head_dim], out_dtype PA_F32 or PA_BF16
+ * bf16 only (kv_dtype PA_BF16, else PA_ERR_UNSUPPORTED); head_dim 64 or 128;
+ * Hq / Hkv in {1, 2, 4, 8, 16}.  Runs on the 5th-generation tensor cores
+ * (tcgen05 with tensor-memory accumulators).  A sequence with n > L or a
+ * length beyond its table is skipped and records PA_ERR_BAD_BLOCK_ID.
+ */
+int pa_paged_attention_prefill(const void* q, const void* k_pool, const void* v_pool,
+                               const int32_t* block_tables, int max_blocks_per_seq,
+                               const int32_t* context_lens, const int32_t* query_start,
+                               int max_query_len, float scale, int block_size, void* out,
+                               int out_dtype, int batch, int num_q_heads, int num_kv_heads,
+                               int head_dim, int64_t num_tokens, int64_t num_blocks, int kv_dtype,
+                               void* stream);
+
+/*
  * pa_paged_attention_decode_contiguous -- the same attention over a
  * contiguous cache, the "ideal contiguous attention" [P1] "The kernel side"
  * measures the paged kernel against.  Same kernel, same tiling and staging

@@ -44,6 +44,8 @@ _SIGS = {
                                    _SZ, _P], _I),
     "pa_paged_attention_decode_contiguous": ([_P, _P, _P, _I64, _P, _I, _F, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P,
                                               _SZ, _P], _I),
+    "pa_paged_attention_prefill": ([_P, _P, _P, _P, _I, _P, _P, _I, _F, _I, _P, _I, _I, _I, _I, _I, _I64, _I64, _I,
+                                    _P], _I),
     "pa_paged_attention_decode_static_scratch": ([_P, _P, _P, _P, _I, _P, _I, _F, _I, _P, _I, _I, _I, _I, _I, _I64,
                                                   _I, _I, _P], _I),
     # host-side block manager (host pointers)
@@ -273,3 +275,23 @@ def pa_paged_attention_decode_static_scratch(q, k_pool, v_pool, block_tables, co
         _dev(q, "q"), k_pool.data_ptr(), v_pool.data_ptr(), _dev(block_tables, "block_tables", torch.int32), MBS,
         _dev(context_lens, "context_lens", torch.int32), int(max_context_len), float(scale), bs, _dev(out, "out"),
         _kv_dtype(out), B, Hq, Hkv, D, NB, dt, partition_size, _stream(stream)))
+
+
+def pa_paged_attention_prefill(q, k_pool, v_pool, block_tables, context_lens, query_start, max_query_len: int,
+                               scale: float, out, stream=None) -> None:
+    """Causal multi-query attention: q rows query_start[b]..query_start[b+1]-1
+    are the last tokens of sequence b (lengths context_lens, counting them)."""
+    T, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_pool.shape
+    if D2 != D or v_pool.shape != k_pool.shape or tuple(out.shape) != (T, Hq, D):
+        raise ValueError("q / pool / out shapes disagree")
+    B = context_lens.numel()
+    if query_start.numel() != B + 1:
+        raise ValueError("query_start needs batch + 1 entries")
+    _dev(k_pool, "k_pool", q.dtype)
+    _dev(v_pool, "v_pool", q.dtype)
+    _check("pa_paged_attention_prefill", _lib.pa_paged_attention_prefill(
+        _dev(q, "q"), k_pool.data_ptr(), v_pool.data_ptr(), _dev(block_tables, "block_tables", torch.int32),
+        block_tables.shape[1], _dev(context_lens, "context_lens", torch.int32),
+        _dev(query_start, "query_start", torch.int32), int(max_query_len), float(scale), bs, _dev(out, "out"),
+        _kv_dtype(out), B, Hq, Hkv, D, T, NB, _kv_dtype(q), _stream(stream)))

@@ -1,0 +1,551 @@
+// pa_prefill.cu -- causal multi-query attention over the paged cache
+// (several new tokens per sequence, as in chunked prefill), on the 5th-
+// generation tensor cores (tcgen05, accumulators in tensor memory).
+//
+// What it computes: sequence b of length L has n new query tokens, its last
+// n; query i sits at position p = L - n + i and attends keys 0..p.  K and V
+// are read from the block pool through the block table ("PagedAttention and
+// KV memory management", "The kernel side"), never gathered.
+//
+// Work item = 128 query rows of one (sequence, kv head): 128 / G query tokens
+// x the G query heads that share the kv head, one CTA each.  Per CTA:
+//  * warp 0 loads the Q tile once (tiled TMA, 3-D map over q [T, Hq, D]) and
+//    streams K/V tiles of 64 tokens through a 2-stage ring (tiled TMA boxes
+//    of block_size rows from the pool, 128-byte swizzle);
+//  * warp 1 allocates tensor memory and issues the MMAs from one thread:
+//        S_j = Q . K_j^T        (M = 128 rows, N = 64 keys, K = D)
+//        O  += P_j . V_j        (M = 128 rows, N = D, K = 64 keys)
+//    S is double-buffered in TMEM so S_{j+1} runs while the softmax works on
+//    S_j; O accumulates in TMEM across tiles;
+//  * warps 2..5 (128 threads, one query row each: TMEM lane = row) load S_j,
+//    apply the causal mask and scale, keep the row's running max and sum in
+//    registers, rescale O in TMEM when the max grows, and write P_j to shared
+//    memory as a bf16 high part plus a bf16 residual (both multiplied by V,
+//    so the weights keep ~16 significant bits).  At the end they read O,
+//    divide by the row sum and store the row.
+// Every wait is a bounded mbarrier wait; on expiry the CTA records
+// PA_ERR_TIMEOUT and winds down (tensor memory is always released).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "pa.h"
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+namespace {
+
+constexpr int kRows = 128;    // query rows per CTA (TMEM lanes)
+constexpr int kKeys = 64;     // keys per tile
+constexpr int kThreads = 192;  // producer, MMA, 4 softmax warps
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct PrefillParams {
+    const void* q;
+    void* out;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    const int32_t* query_start;
+    int* err;
+    int64_t num_blocks;
+    int max_blocks_per_seq;
+    int num_q_heads;
+    int num_kv_heads;
+    int block_size;
+    int out_bf16;
+    float scale_log2;
+};
+
+// ---- tcgen05 helpers -------------------------------------------------------
+__device__ __forceinline__ uint64_t umma_desc(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+    // shared-memory matrix descriptor: start, leading / stride byte offsets
+    // (16-byte units), descriptor version 1, 128-byte swizzle
+    uint64_t d = (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// instruction descriptor: fp32 accumulate, bf16 A and B, A K-major, B K- or
+// MN-major, shape M x N
+__host__ __device__ constexpr uint32_t umma_idesc(int M, int N, bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn_major ? (1u << 16) : 0u) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(da), "l"(db), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 consecutive fp32 columns of this warp's 32 TMEM lanes (one per thread)
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+        "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+        "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+        "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+        "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])),
+        "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+        "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])),
+        "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
+        "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
+        "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, int x, int y, int z, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// ---- the kernel ------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmq,
+                      const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
+    constexpr int SLABS = D / 64;
+    constexpr int Q_BYTES = SLABS * kRows * 128;     // 128 rows x D
+    constexpr int KV_SLAB = kKeys * 128;             // 64 rows x 64 elements
+    constexpr int KV_BYTES = SLABS * KV_SLAB;        // one of K or V for one tile
+    constexpr int P_BYTES = kRows * 128;             // 128 rows x 64 keys (bf16)
+    constexpr int S_COLS = kKeys;                    // TMEM columns of one S buffer
+    constexpr uint32_t O_COL = 2 * S_COLS;           // O after the two S buffers
+    constexpr uint32_t TMEM_COLS = 2 * S_COLS + D <= 256 ? 256 : 512;
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    uint8_t* sQ = smem;
+    uint8_t* sK = sQ + Q_BYTES;            // [2][KV_BYTES]
+    uint8_t* sV = sK + 2 * KV_BYTES;       // [2][KV_BYTES]
+    uint8_t* sPh = sV + 2 * KV_BYTES;      // P high part
+    uint8_t* sPl = sPh + P_BYTES;          // P residual
+
+    __shared__ uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], s_free[2], p_full, o_done;
+    __shared__ uint32_t tmem_base;
+    __shared__ int s_abort;
+
+    const int qtile = blockIdx.x;
+    const int kvh = blockIdx.y;
+    const int b = blockIdx.z;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int G = p.num_q_heads / p.num_kv_heads;
+    const int TQ = kRows / G;  // query tokens per tile
+
+    const int q0 = p.query_start[b];
+    const int n = p.query_start[b + 1] - q0;
+    const int L = p.context_lens[b];
+    const int t0 = qtile * TQ;
+    if (t0 >= n) return;  // uniform over the CTA
+    if (n > L || (int64_t)L > (int64_t)p.max_blocks_per_seq * p.block_size) {
+        if (threadIdx.x == 0 && qtile == 0 && kvh == 0) record_error(p.err, PA_ERR_BAD_BLOCK_ID);
+        return;
+    }
+    const int nq = min(TQ, n - t0);
+    const int pos_first = L - n + t0;        // position of the tile's first query token
+    const int n_kv = pos_first + nq;         // keys the tile needs: 0 .. pos_first + nq - 1
+    const int nt = (n_kv + kKeys - 1) / kKeys;
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        prefetch_tmap(&tmq);
+        prefetch_tmap(&tmk);
+        prefetch_tmap(&tmv);
+        mbar_init(&q_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+            mbar_init(&s_full[s], 1);
+            mbar_init(&s_free[s], 4);
+        }
+        mbar_init(&p_full, 128);
+        mbar_init(&o_done, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&tmem_base)),
+                     "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base;
+
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        const int bs = p.block_size;
+        const int boxes = kKeys / bs;  // pool boxes per tile and slab
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&q_full, (uint32_t)Q_BYTES);
+#pragma unroll
+            for (int sl = 0; sl < SLABS; ++sl)
+                tma_load_3d(sQ + sl * kRows * 128, &tmq, sl * 64, kvh * G, q0 + t0, &q_full);
+        }
+        const int32_t* table = p.block_tables + (int64_t)b * p.max_blocks_per_seq;
+        for (int j = 0; j < nt; ++j) {
+            const int s = j & 1;
+            if (j >= 2) {
+                int ok = 1;
+                if (lane == 0) ok = mbar_wait(&kv_empty[s], ((j >> 1) - 1) & 1, p.err);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                    if (lane == 0) s_abort = 1;
+                    break;
+                }
+            }
+            // lane i loads pool block i of the tile (if it holds keys < n_kv)
+            const int key0 = j * kKeys + lane * bs;
+            uint32_t bytes = 0;
+            int y = 0;
+            if (lane < boxes && key0 < n_kv) {
+                const int32_t phys = table[key0 / bs];
+                if (phys < 0 || phys >= p.num_blocks) {
+                    record_error(p.err, PA_ERR_BAD_BLOCK_ID);
+                } else {
+                    bytes = (uint32_t)(2 * SLABS * bs * 128);
+                    y = (phys * p.num_kv_heads + kvh) * bs;
+                }
+            }
+            const uint32_t total = __reduce_add_sync(0xffffffffu, bytes);
+            if (lane == 0) mbar_arrive_expect_tx(&kv_full[s], total);
+            __syncwarp();
+            if (bytes) {
+                const uint64_t policy = l2_policy_evict_first();
+#pragma unroll
+                for (int sl = 0; sl < SLABS; ++sl) {
+                    tma_load_2d(sK + s * KV_BYTES + sl * KV_SLAB + lane * bs * 128, &tmk, sl * 64, y, &kv_full[s],
+                                policy);
+                    tma_load_2d(sV + s * KV_BYTES + sl * KV_SLAB + lane * bs * 128, &tmv, sl * 64, y, &kv_full[s],
+                                policy);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            constexpr uint32_t IDESC_S = umma_idesc(kRows, kKeys, false);
+            constexpr uint32_t IDESC_O = umma_idesc(kRows, D, true);
+            const uint32_t q_base = smem_addr(sQ);
+            bool ok = mbar_wait(&q_full, 0, p.err);
+            auto issue_s = [&](int j) -> bool {
+                const int s = j & 1;
+                if (!mbar_wait(&kv_full[s], (j >> 1) & 1, p.err)) return false;
+                if (j >= 2 && !mbar_wait(&s_free[s], ((j >> 1) - 1) & 1, p.err)) return false;
+                tc_fence_after();
+                const uint32_t k_base = smem_addr(sK + s * KV_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk & 3) * 32;
+                    const uint64_t da = umma_desc(q_base + (kk >> 2) * (kRows * 128) + off, 16, 1024);
+                    const uint64_t db = umma_desc(k_base + (kk >> 2) * KV_SLAB + off, 16, 1024);
+                    umma(tmem + s * S_COLS, da, db, IDESC_S, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&s_full[s]);
+                return true;
+            };
+            if (ok) ok = issue_s(0);
+            for (int j = 0; ok && j < nt; ++j) {
+                if (j + 1 < nt && !(ok = issue_s(j + 1))) break;
+                if (!(ok = mbar_wait(&p_full, j & 1, p.err))) break;
+                tc_fence_after();
+                const uint32_t v_base = smem_addr(sV + (j & 1) * KV_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < kKeys / 16; ++kk) {
+                    const uint64_t db = umma_desc(v_base + kk * 2048, KV_SLAB, 1024);
+                    const uint64_t dh = umma_desc(smem_addr(sPh) + kk * 32, 16, 1024);
+                    const uint64_t dl = umma_desc(smem_addr(sPl) + kk * 32, 16, 1024);
+                    umma(tmem + O_COL, dh, db, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+                    umma(tmem + O_COL, dl, db, IDESC_O, 1u);
+                }
+                umma_commit(&o_done);
+                umma_commit(&kv_empty[j & 1]);
+            }
+            if (!ok) s_abort = 1;
+        }
+    } else {
+        // ---------------- softmax / epilogue: one query row per thread ----------------
+        const int quarter = warp & 3;                 // TMEM lane quarter this warp may access
+        const int row = quarter * 32 + lane;          // query row of the tile = TMEM lane
+        const int tq = row / G;                       // query token within the tile
+        const bool valid = tq < nq;
+        const int limit = valid ? pos_first + tq : -1;  // last key this row may see
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        float m = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nt; ++j) {
+            const int s = j & 1;
+            if (!(ok = mbar_wait(&s_full[s], (j >> 1) & 1, p.err))) break;
+            tc_fence_after();
+            float sv[kKeys];
+            tmem_ld32(lane_base + s * S_COLS, sv);
+            tmem_ld32(lane_base + s * S_COLS + 32, sv + 32);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_free[s]);
+            const int kbase = j * kKeys;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < kKeys; ++c) {
+                sv[c] = kbase + c <= limit ? sv[c] * p.scale_log2 : -INFINITY;
+                mx = fmaxf(mx, sv[c]);
+            }
+            const float m_new = fmaxf(m, mx);
+            float alpha = 1.f, sum = 0.f;
+            if (m_new != -INFINITY) {
+                alpha = exp2f(m - m_new);
+#pragma unroll
+                for (int c = 0; c < kKeys; ++c) {
+                    sv[c] = exp2f(sv[c] - m_new);
+                    sum += sv[c];
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < kKeys; ++c) sv[c] = 0.f;
+            }
+            l = l * alpha + sum;
+            m = m_new;
+            // P_j and the O rescale must wait until PV_{j-1} has finished with
+            // the P buffer and with O
+            if (j > 0) {
+                if (!(ok = mbar_wait(&o_done, (j - 1) & 1, p.err))) break;
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+                    for (int c0 = 0; c0 < D; c0 += 32) {
+                        float ov[32];
+                        tmem_ld32(lane_base + O_COL + c0, ov);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+                        tmem_st32(lane_base + O_COL + c0, ov);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            // P row: 64 keys = one 128-byte row per part, 8 chunks of 8 keys
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float a = sv[8 * c + 2 * e], bb = sv[8 * c + 2 * e + 1];
+                    hi[e] = pack_bf16x2(a, bb);
+                    lo[e] = pack_bf16x2(a - bf16_lo_to_f32(hi[e]), bb - bf16_hi_to_f32(hi[e]));
+                }
+                const int pc = (c ^ (row & 7)) << 4;
+                *reinterpret_cast<uint4*>(sPh + row * 128 + pc) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4*>(sPl + row * 128 + pc) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+            // keys past the sequence end carry weight 0, but 0 * NaN is NaN in
+            // the MMA: zero those V rows of the last tile
+            if (j == nt - 1 && n_kv < nt * kKeys) {
+                uint8_t* vs = sV + s * KV_BYTES;
+                const int first = n_kv - j * kKeys;
+                const int nch = (kKeys - first) * SLABS * 8;
+                for (int c = threadIdx.x - 64; c < nch; c += 128) {
+                    const int r = first + c / (SLABS * 8);
+                    const int rem = c % (SLABS * 8);
+                    *reinterpret_cast<uint4*>(vs + (rem >> 3) * KV_SLAB + r * 128 + (rem & 7) * 16) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+            // every softmax thread signals its own P row (and V zeroing) to the
+            // MMA thread; no named barrier, so a timed-out warp cannot strand
+            // the others
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tc_fence_before();
+            mbar_arrive(&p_full);
+        }
+        // epilogue: O / l for this row
+        if (ok && (ok = mbar_wait(&o_done, (nt - 1) & 1, p.err))) {
+            tc_fence_after();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const int64_t orow = ((int64_t)(q0 + t0 + tq) * p.num_q_heads + (int64_t)kvh * G + (row % G)) * D;
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                float ov[32];
+                tmem_ld32(lane_base + O_COL + c0, ov);
+                tmem_wait_ld();
+                if (valid) {
+                    if (p.out_bf16) {
+                        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + orow + c0;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] = __float2bfloat16_rn(ov[i] * inv);
+                    } else {
+                        float* o = static_cast<float*>(p.out) + orow + c0;
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4)
+                            *reinterpret_cast<float4*>(o + i) =
+                                make_float4(ov[i] * inv, ov[i + 1] * inv, ov[i + 2] * inv, ov[i + 3] * inv);
+                    }
+                }
+            }
+        }
+        if (!ok) s_abort = 1;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+    }
+}
+
+// ---- host side -------------------------------------------------------------
+using TensorMapEncodeFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+TensorMapEncodeFn encoder() {
+    static TensorMapEncodeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<TensorMapEncodeFn>(ptr);
+    });
+    return fn;
+}
+
+int encode(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+           const cuuint32_t* box) {
+    TensorMapEncodeFn enc = encoder();
+    if (!enc) return PA_ERR_CUDA;
+    cuuint32_t es[3] = {1u, 1u, 1u};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, es,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+}
+
+template <int D>
+size_t prefill_smem_bytes() {
+    constexpr int SLABS = D / 64;
+    return 1024 + SLABS * kRows * 128 + 4 * SLABS * kKeys * 128 + 2 * kRows * 128;
+}
+
+template <int D>
+int launch_prefill(const PrefillParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                   dim3 grid, cudaStream_t st) {
+    static std::atomic<unsigned long long> configured{0};
+    const size_t smem = prefill_smem_bytes<D>();
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(configured.load() & bit)) {
+        if (cudaFuncSetAttribute(prefill_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return PA_ERR_CUDA;
+        configured.fetch_or(bit);
+    }
+    prefill_tc_kernel<D><<<grid, kThreads, smem, st>>>(p, tq, tk, tv);
+    return launch_status();
+}
+
+}  // namespace
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" int pa_paged_attention_prefill(const void* q, const void* k_pool, const void* v_pool,
+                                          const int32_t* block_tables, int max_blocks_per_seq,
+                                          const int32_t* context_lens, const int32_t* query_start,
+                                          int max_query_len, float scale, int block_size, void* out,
+                                          int out_dtype, int batch, int num_q_heads, int num_kv_heads,
+                                          int head_dim, int64_t num_tokens, int64_t num_blocks, int kv_dtype,
+                                          void* stream) {
+    if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        max_query_len < 0 || num_tokens < 0 || num_blocks < 0 || max_blocks_per_seq < 0 || !valid_dtype(kv_dtype) ||
+        !valid_dtype(out_dtype) || num_q_heads % num_kv_heads != 0)
+        return PA_ERR_INVALID_ARG;
+    const int G = num_q_heads / num_kv_heads;
+    if (kv_dtype != PA_BF16 || !supported_head_dim(head_dim) || !supported_block_size(block_size) ||
+        (G != 1 && G != 2 && G != 4 && G != 8 && G != 16))
+        return PA_ERR_UNSUPPORTED;
+    if (batch == 0 || num_tokens == 0 || max_query_len == 0) return PA_OK;
+    if (batch > 65535 || num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+    if (!q || !k_pool || !v_pool || !block_tables || !context_lens || !query_start || !out) return PA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out)) return PA_ERR_INVALID_ARG;
+    const uint64_t pool_rows = (uint64_t)num_blocks * num_kv_heads * (uint64_t)block_size;
+    if (pool_rows >= (1ull << 31) || num_tokens >= (1ll << 31)) return PA_ERR_UNSUPPORTED;
+    int* err = error_word_ptr();
+    if (!err) return PA_ERR_CUDA;
+
+    CUtensorMap tq, tk, tv;
+    const int TQ = kRows / G;
+    {
+        cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_q_heads, (cuuint64_t)num_tokens};
+        cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2, (cuuint64_t)num_q_heads * head_dim * 2};
+        cuuint32_t box[3] = {64u, (cuuint32_t)G, (cuuint32_t)TQ};
+        int rc = encode(&tq, q, 3, dims, strides, box);
+        if (rc) return rc;
+    }
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)head_dim, pool_rows > 0 ? pool_rows : 1};
+        cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
+        cuuint32_t box[2] = {64u, (cuuint32_t)block_size};
+        int rc = encode(&tk, k_pool, 2, dims, strides, box);
+        if (!rc) rc = encode(&tv, v_pool, 2, dims, strides, box);
+        if (rc) return rc;
+    }
+    PrefillParams p = {};
+    p.q = q;
+    p.out = out;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.query_start = query_start;
+    p.err = err;
+    p.num_blocks = num_blocks;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.block_size = block_size;
+    p.out_bf16 = out_dtype == PA_BF16;
+    p.scale_log2 = scale * kLog2e;
+    dim3 grid((unsigned)((max_query_len + TQ - 1) / TQ), (unsigned)num_kv_heads, (unsigned)batch);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return head_dim == 128 ? launch_prefill<128>(p, tq, tk, tv, grid, st) : launch_prefill<64>(p, tq, tk, tv, grid, st);
+}

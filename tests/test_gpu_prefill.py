@@ -1,0 +1,99 @@
+"""GPU parity of causal multi-query paged attention (tcgen05 kernel) against
+the fp64 oracle: chunks that are whole sequences or their tails, every group
+size and block size, ragged lengths across tile boundaries, NaN-poisoned
+slots past each sequence, and the single-token case against decode."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_355_b200.workloads import custom_case
+from tests.helpers import assert_matches_oracle, np_of
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def pa():
+    import paged_kv_cache_355_b200 as pa
+
+    assert torch.cuda.is_available()
+    pa.pa_read_error_flag()
+    return pa
+
+
+def _run(pa, case, news, out_dtype=torch.float32, k_pool=None, v_pool=None):
+    """Prefill with news[b] query tokens at the end of each sequence."""
+    Hq, D = case.q.shape[1], case.q.shape[2]
+    qs = np.concatenate([[0], np.cumsum(news)]).astype(np.int32)
+    T = int(qs[-1])
+    g = torch.Generator().manual_seed(T + Hq)
+    q = torch.randn(T, Hq, D, generator=g).to(torch.bfloat16)
+    kp = case.k_pool if k_pool is None else k_pool
+    vp = case.v_pool if v_pool is None else v_pool
+    out = torch.full((T, Hq, D), float("nan"), dtype=out_dtype, device="cuda")
+    pa.pa_paged_attention_prefill(q.cuda(), kp.cuda(), vp.cuda(), case.block_tables.cuda(), case.lengths.cuda(),
+                                  torch.from_numpy(qs).cuda(), int(max(news)), case.scale, out)
+    torch.cuda.synchronize()
+    ref = oracle.paged_prefill(np_of(q), np_of(kp), np_of(vp), np_of(case.block_tables), np_of(case.lengths), qs,
+                               case.scale, case.workload.block_size)
+    return out, ref
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("bs", [8, 16, 32])
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
+def test_prefill_sweep(pa, D, bs, G):
+    Hkv = 2
+    lengths = [1, 63, 64, 65, 200, 300]
+    news = [1, 63, 10, 65, 130, 1]
+    case = custom_case(lengths, Hkv * G, Hkv, D, bs, torch.bfloat16, seed=D + bs + G)
+    out, ref = _run(pa, case, news)
+    assert_matches_oracle(out, ref, True, f"prefill D{D} bs{bs} G{G}")
+    assert pa.pa_read_error_flag() == 0
+
+
+def test_prefill_long_chunk_and_bf16_out(pa):
+    case = custom_case([1500, 700, 2048], 32, 8, 128, 16, torch.bfloat16, seed=5)
+    out, ref = _run(pa, case, [1500, 256, 129], out_dtype=torch.bfloat16)
+    assert_matches_oracle(out, ref, True, "prefill long")
+
+
+def test_prefill_single_token_equals_decode(pa):
+    case = custom_case([5, 77, 300, 1], 16, 4, 128, 16, torch.bfloat16, seed=6)
+    out, ref = _run(pa, case, [1, 1, 1, 1])
+    dec = torch.empty_like(out)
+    qs = np.arange(5, dtype=np.int32)
+    g = torch.Generator().manual_seed(4 + 16)
+    q = torch.randn(4, 16, 128, generator=g).to(torch.bfloat16)
+    pa.pa_paged_attention_decode(q.cuda(), case.k_pool.cuda(), case.v_pool.cuda(), case.block_tables.cuda(),
+                                 case.lengths.cuda(), case.max_len, case.scale, dec)
+    torch.cuda.synchronize()
+    assert_matches_oracle(out, ref, True, "prefill n=1")
+    assert_matches_oracle(dec, ref, True, "decode vs prefill oracle")
+
+
+def test_prefill_never_reads_past_the_sequence(pa):
+    lengths = [40, 129, 17]
+    case = custom_case(lengths, 8, 2, 128, 16, torch.bfloat16, seed=7, extra_blocks=6)
+    kp, vp = case.k_pool.clone(), case.v_pool.clone()
+    used = torch.zeros(case.num_blocks, 16, dtype=torch.bool)
+    for b, L in enumerate(lengths):
+        for t in range(L):
+            used[case.block_tables[b, t // 16], t % 16] = True
+    kp.permute(0, 2, 1, 3)[~used] = float("nan")
+    vp.permute(0, 2, 1, 3)[~used] = float("nan")
+    out, ref = _run(pa, case, [40, 70, 3], k_pool=kp, v_pool=vp)
+    assert_matches_oracle(out, ref, True, "poisoned slots")
+    assert pa.pa_read_error_flag() == 0
+
+
+def test_prefill_rejects_fp32(pa):
+    case = custom_case([8], 4, 4, 64, 16, torch.float32, seed=8)
+    q = torch.zeros(8, 4, 64, device="cuda")
+    with pytest.raises(pa.PAError, match="UNSUPPORTED"):
+        pa.pa_paged_attention_prefill(q, case.k_pool.cuda(), case.v_pool.cuda(), case.block_tables.cuda(),
+                                      case.lengths.cuda(), torch.tensor([0, 8], dtype=torch.int32, device="cuda"), 8,
+                                      case.scale, torch.empty(8, 4, 64, device="cuda"))
