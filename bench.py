@@ -74,6 +74,9 @@ def parse():
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", default="decode", choices=["decode", "prefill"],
+                    help="decode: the decode step (default); prefill: causal multi-query paged attention "
+                         "on a chunked-prefill workload, in TFLOP/s")
     return ap.parse_args()
 
 
@@ -452,10 +455,68 @@ def run_ours(args):
     print(json.dumps(line), flush=True)
 
 
+PREFILL_WORKLOAD = ("chunked prefill: batch 8, 32 q / 8 kv heads, head_dim 128, block_size 16, bf16, "
+                    "context 4096 of which the last 2048 tokens are the new chunk, blocks scattered")
+
+
+def run_prefill(args):
+    """Causal multi-query paged attention on one GPU: useful FLOPs (4 * D per
+    (query, visible key, query head)) / CUDA-event time."""
+    import paged_kv_cache_355_b200 as pa
+    from paged_kv_cache_355_b200.workloads import custom_case
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    B, Hq, Hkv, D, bs, L, n = 8, 32, 8, 128, 16, 4096, 2048
+    case = custom_case([L] * B, Hq, Hkv, D, bs, torch.bfloat16, seed=2001, device=dev)
+    qs = torch.arange(0, (B + 1) * n, n, dtype=torch.int32, device=dev)
+    g = torch.Generator(device=dev).manual_seed(2002)
+    q = torch.randn(B * n, Hq, D, generator=g, device=dev).to(torch.bfloat16)
+    out = torch.empty(B * n, Hq, D, dtype=torch.bfloat16, device=dev)
+    bt, lens = case.block_tables.to(dev), case.lengths.to(dev)
+    pairs = sum(n * (L - n) + n * (n + 1) // 2 for _ in range(B))  # visible (query, key) pairs per head
+    flops = 4.0 * D * Hq * pairs
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    run = lambda: pa.pa_paged_attention_prefill(q, case.k_pool, case.v_pool, bt, lens, qs, n, case.scale, out)
+    for _ in range(args.warmup):
+        run()
+    evs = []
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clocks:
+        for _ in range(args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            run()
+            e1.record()
+            evs.append((e0, e1))
+        torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b_) for a, b_ in evs) / len(evs)
+    assert pa.pa_read_error_flag() == 0
+    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    peak = float(peaks.get("bf16_tflops", 1590.0))
+    tflops = flops / (ms * 1e-3) / 1e12
+    print(json.dumps({
+        "metric": "Paged prefill attn (causal, multi-query): achieved TFLOP/s vs bf16 peak", "value": tflops,
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic", "config": {"workload": PREFILL_WORKLOAD},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
+                     "traffic": None, "kernel": "prefill_tc_kernel (tcgen05)",
+                     "peak_source": "measured (MEASURED_PEAKS.json bf16_tflops, cuBLAS burst)" if peaks
+                     else "fallback"},
+        "note": "useful FLOPs only; the kernel multiplies P by V twice (bf16 high part and residual), "
+                "so the tensor pipe executes 1.5x these FLOPs",
+        "clocks": clocks.summary()}), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.op == "prefill":
+        run_prefill(args)
         return
     run_ours(args)
     if int(os.environ.get("WORLD_SIZE", "1")) > 1:

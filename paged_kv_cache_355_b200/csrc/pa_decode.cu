@@ -855,6 +855,7 @@ __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(const De
         const float w = s < ns ? ml[2 * s + 1] * exp2f(ml[2 * s] - M) : 0.f;
         W += w;
         const int n = min(32, ns - s0);
+#pragma unroll 8
         for (int k = 0; k < n; ++k) {
             const float wk = __shfl_sync(0xffffffffu, w, k);
             const float* src = po + (int64_t)(s0 + k) * D;
