@@ -10,7 +10,7 @@
 // Work item = 128 query rows of one (sequence, kv head): 128 / G query tokens
 // x the G query heads that share the kv head, one CTA each.  Per CTA:
 //  * warp 0 loads the Q tile once (tiled TMA, 3-D map over q [T, Hq, D]) and
-//    streams K/V tiles of 64 tokens through a 2-stage ring (tiled TMA boxes
+//    streams K/V tiles of 64 tokens through a 4-stage ring (tiled TMA boxes
 //    of block_size rows from the pool, 128-byte swizzle);
 //  * warp 1 allocates tensor memory and issues the MMAs from one thread:
 //        S_j = Q . K_j^T        (M = 128 rows, N = 64 keys, K = D)
@@ -19,10 +19,12 @@
 //    S_j; O accumulates in TMEM across tiles;
 //  * warps 2..5 (128 threads, one query row each: TMEM lane = row) load S_j,
 //    apply the causal mask and scale, keep the row's running max and sum in
-//    registers, rescale O in TMEM when the max grows, and write P_j to shared
-//    memory as a bf16 high part plus a bf16 residual (both multiplied by V,
-//    so the weights keep ~16 significant bits).  At the end they read O,
-//    divide by the row sum and store the row.
+//    registers, rescale O in TMEM only when the max has grown by more than
+//    2^8 (lazy rescale), and write P_j to one of two shared-memory buffers as
+//    a bf16 high part plus a bf16 residual (both multiplied by V, so the
+//    weights keep ~16 significant bits); the softmax of tile j + 1 thus runs
+//    while the tensor core does P_j . V_j.  At the end they read O, divide by
+//    the row sum and store the row.
 // Every wait is a bounded mbarrier wait; on expiry the CTA records
 // PA_ERR_TIMEOUT and winds down (tensor memory is always released).
 #include <cuda.h>
@@ -45,7 +47,9 @@ namespace {
 constexpr int kRows = 128;    // query rows per CTA (TMEM lanes)
 constexpr int kKeys = 64;     // keys per tile
 constexpr int kThreads = 192;  // producer, MMA, 4 softmax warps
+constexpr int kStages = 4;     // K/V ring depth
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleLog2 = 8.f;  // lazy-rescale threshold of the running max (log2 units)
 
 struct PrefillParams {
     const void* q;
@@ -92,6 +96,14 @@ __device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t da, uint64_t db, 
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
                  : "memory");
+}
+
+// 2^x with the hardware's approximate exp2 instruction (ex2.approx.ftz,
+// relative error ~2^-22; 2^-inf = 0)
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -157,12 +169,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     uint8_t* sQ = smem;
-    uint8_t* sK = sQ + Q_BYTES;            // [2][KV_BYTES]
-    uint8_t* sV = sK + 2 * KV_BYTES;       // [2][KV_BYTES]
-    uint8_t* sPh = sV + 2 * KV_BYTES;      // P high part
-    uint8_t* sPl = sPh + P_BYTES;          // P residual
+    uint8_t* sK = sQ + Q_BYTES;                  // [kStages][KV_BYTES]
+    uint8_t* sV = sK + kStages * KV_BYTES;       // [kStages][KV_BYTES]
+    uint8_t* sPh = sV + kStages * KV_BYTES;      // P high part, [2][P_BYTES]
+    uint8_t* sPl = sPh + 2 * P_BYTES;      // P residual,  [2][P_BYTES]
 
-    __shared__ uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], s_free[2], p_full, o_done;
+    __shared__ uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[2], s_free[2], p_full[2], pv_done[2];
     __shared__ uint32_t tmem_base;
     __shared__ int s_abort;
 
@@ -194,14 +206,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
         mbar_init(&q_full, 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kStages; ++s) {
             mbar_init(&kv_full[s], 1);
             mbar_init(&kv_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
             mbar_init(&s_full[s], 1);
             mbar_init(&s_free[s], 4);
+            mbar_init(&p_full[s], 128);
+            mbar_init(&pv_done[s], 1);
         }
-        mbar_init(&p_full, 128);
-        mbar_init(&o_done, 1);
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -226,10 +240,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int32_t* table = p.block_tables + (int64_t)b * p.max_blocks_per_seq;
         for (int j = 0; j < nt; ++j) {
-            const int s = j & 1;
-            if (j >= 2) {
+            const int s = j % kStages;
+            if (j >= kStages) {
                 int ok = 1;
-                if (lane == 0) ok = mbar_wait(&kv_empty[s], ((j >> 1) - 1) & 1, p.err);
+                if (lane == 0) ok = mbar_wait(&kv_empty[s], ((j / kStages) - 1) & 1, p.err);
                 if (!__shfl_sync(0xffffffffu, ok, 0)) {
                     if (lane == 0) s_abort = 1;
                     break;
@@ -270,11 +284,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t q_base = smem_addr(sQ);
             bool ok = mbar_wait(&q_full, 0, p.err);
             auto issue_s = [&](int j) -> bool {
-                const int s = j & 1;
-                if (!mbar_wait(&kv_full[s], (j >> 1) & 1, p.err)) return false;
+                const int s = j & 1;  // S buffer
+                const int ks = j % kStages;
+                if (!mbar_wait(&kv_full[ks], (j / kStages) & 1, p.err)) return false;
                 if (j >= 2 && !mbar_wait(&s_free[s], ((j >> 1) - 1) & 1, p.err)) return false;
                 tc_fence_after();
-                const uint32_t k_base = smem_addr(sK + s * KV_BYTES);
+                const uint32_t k_base = smem_addr(sK + ks * KV_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk & 3) * 32;
@@ -288,19 +303,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok) ok = issue_s(0);
             for (int j = 0; ok && j < nt; ++j) {
                 if (j + 1 < nt && !(ok = issue_s(j + 1))) break;
-                if (!(ok = mbar_wait(&p_full, j & 1, p.err))) break;
+                if (!(ok = mbar_wait(&p_full[j & 1], (j >> 1) & 1, p.err))) break;
                 tc_fence_after();
-                const uint32_t v_base = smem_addr(sV + (j & 1) * KV_BYTES);
+                const uint32_t v_base = smem_addr(sV + (j % kStages) * KV_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < kKeys / 16; ++kk) {
                     const uint64_t db = umma_desc(v_base + kk * 2048, KV_SLAB, 1024);
-                    const uint64_t dh = umma_desc(smem_addr(sPh) + kk * 32, 16, 1024);
-                    const uint64_t dl = umma_desc(smem_addr(sPl) + kk * 32, 16, 1024);
+                    const uint64_t dh = umma_desc(smem_addr(sPh + (j & 1) * P_BYTES) + kk * 32, 16, 1024);
+                    const uint64_t dl = umma_desc(smem_addr(sPl + (j & 1) * P_BYTES) + kk * 32, 16, 1024);
                     umma(tmem + O_COL, dh, db, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
                     umma(tmem + O_COL, dl, db, IDESC_O, 1u);
                 }
-                umma_commit(&o_done);
-                umma_commit(&kv_empty[j & 1]);
+                umma_commit(&pv_done[j & 1]);
+                umma_commit(&kv_empty[j % kStages]);
             }
             if (!ok) s_abort = 1;
         }
@@ -327,18 +342,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(&s_free[s]);
             const int kbase = j * kKeys;
             float mx = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < kKeys; ++c) {
-                sv[c] = kbase + c <= limit ? sv[c] * p.scale_log2 : -INFINITY;
-                mx = fmaxf(mx, sv[c]);
-            }
-            const float m_new = fmaxf(m, mx);
-            float alpha = 1.f, sum = 0.f;
-            if (m_new != -INFINITY) {
-                alpha = exp2f(m - m_new);
+            if (__all_sync(0xffffffffu, kbase + kKeys - 1 <= limit)) {
+                // every key of the tile is visible to every row of this warp
 #pragma unroll
                 for (int c = 0; c < kKeys; ++c) {
-                    sv[c] = exp2f(sv[c] - m_new);
+                    sv[c] *= p.scale_log2;
+                    mx = fmaxf(mx, sv[c]);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < kKeys; ++c) {
+                    sv[c] = kbase + c <= limit ? sv[c] * p.scale_log2 : -INFINITY;
+                    mx = fmaxf(mx, sv[c]);
+                }
+            }
+            // Lazy rescale: the weights are exp2(s - m) against a reference max
+            // m that only moves when the row's max exceeds it by more than
+            // kRescaleLog2 (weights stay <= 2^kRescaleLog2, far inside fp32 and
+            // bf16 range); the result O / l does not depend on m.  Most tiles
+            // then leave O alone and need not wait for the previous P.V.
+            const bool grow = mx > m + kRescaleLog2;
+            float alpha = 1.f;
+            if (grow) {
+                alpha = m == -INFINITY ? 0.f : exp2f(m - mx);
+                m = mx;
+            }
+            float sum = 0.f;
+            if (m != -INFINITY) {
+#pragma unroll
+                for (int c = 0; c < kKeys; ++c) {
+                    sv[c] = ex2_approx(sv[c] - m);
                     sum += sv[c];
                 }
             } else {
@@ -346,25 +379,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < kKeys; ++c) sv[c] = 0.f;
             }
             l = l * alpha + sum;
-            m = m_new;
-            // P_j and the O rescale must wait until PV_{j-1} has finished with
-            // the P buffer and with O
-            if (j > 0) {
-                if (!(ok = mbar_wait(&o_done, (j - 1) & 1, p.err))) break;
+            if (j > 0 && __any_sync(0xffffffffu, grow)) {
+                // O holds P.V of tiles < j: wait for the last of them, then rescale
+                if (!(ok = mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, p.err))) break;
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-                    for (int c0 = 0; c0 < D; c0 += 32) {
-                        float ov[32];
-                        tmem_ld32(lane_base + O_COL + c0, ov);
-                        tmem_wait_ld();
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    float ov[32];
+                    tmem_ld32(lane_base + O_COL + c0, ov);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-                        tmem_st32(lane_base + O_COL + c0, ov);
-                    }
-                    tmem_wait_st();
+                    for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+                    tmem_st32(lane_base + O_COL + c0, ov);
                 }
+                tmem_wait_st();
             }
+            // the P buffer of tile j was read by P.V of tile j - 2
+            if (j >= 2) {
+                if (!(ok = mbar_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1, p.err))) break;
+            }
+            uint8_t* ph = sPh + (j & 1) * P_BYTES;
+            uint8_t* pl = sPl + (j & 1) * P_BYTES;
             // P row: 64 keys = one 128-byte row per part, 8 chunks of 8 keys
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -376,13 +411,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     lo[e] = pack_bf16x2(a - bf16_lo_to_f32(hi[e]), bb - bf16_hi_to_f32(hi[e]));
                 }
                 const int pc = (c ^ (row & 7)) << 4;
-                *reinterpret_cast<uint4*>(sPh + row * 128 + pc) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4*>(sPl + row * 128 + pc) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                *reinterpret_cast<uint4*>(ph + row * 128 + pc) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4*>(pl + row * 128 + pc) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
             }
             // keys past the sequence end carry weight 0, but 0 * NaN is NaN in
             // the MMA: zero those V rows of the last tile
             if (j == nt - 1 && n_kv < nt * kKeys) {
-                uint8_t* vs = sV + s * KV_BYTES;
+                uint8_t* vs = sV + (j % kStages) * KV_BYTES;
                 const int first = n_kv - j * kKeys;
                 const int nch = (kKeys - first) * SLABS * 8;
                 for (int c = threadIdx.x - 64; c < nch; c += 128) {
@@ -397,10 +432,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the others
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc_fence_before();
-            mbar_arrive(&p_full);
+            mbar_arrive(&p_full[j & 1]);
         }
         // epilogue: O / l for this row
-        if (ok && (ok = mbar_wait(&o_done, (nt - 1) & 1, p.err))) {
+        if (ok && (ok = mbar_wait(&pv_done[(nt - 1) & 1], ((nt - 1) >> 1) & 1, p.err))) {
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             const int64_t orow = ((int64_t)(q0 + t0 + tq) * p.num_q_heads + (int64_t)kvh * G + (row % G)) * D;
@@ -464,7 +499,7 @@ int encode(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
 template <int D>
 size_t prefill_smem_bytes() {
     constexpr int SLABS = D / 64;
-    return 1024 + SLABS * kRows * 128 + 4 * SLABS * kKeys * 128 + 2 * kRows * 128;
+    return 1024 + SLABS * kRows * 128 + 2 * kStages * SLABS * kKeys * 128 + 4 * kRows * 128;
 }
 
 template <int D>
