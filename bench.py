@@ -9,10 +9,12 @@ decode attention over every sequence (pa_paged_attention_decode, pass 1 plus
 the split-KV merge when a sequence is split).  Inputs are seeded synthetic
 tensors shaped like the named workload, resident in HBM before timing.
 
-Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
-on the launching stream, with a 256 MiB write between steps (outside the
-events) to flush the 126 MB L2; the region is bracketed by a barrier and
-torch.cuda.synchronize(); the reported time is the max over ranks.
+Timing: W untimed warm-up steps, then the step is captured into CUDA graphs
+(the cache kernels, the decode call) and K replays are timed, each bracketed
+by CUDA events on the launching stream, with a 256 MiB write between steps
+(outside the events) to flush the 126 MB L2; the region is bracketed by a
+barrier and torch.cuda.synchronize(); the reported time is the max over
+ranks.  The end-to-end figure goes through the plain Python API instead.
 
 value  = K/V bytes attention reads (tokens < length, K and V) / step time,
          summed over ranks (each rank runs its own batch: weak scaling, no
@@ -335,10 +337,31 @@ def run_ours(args):
     launches_per_step = (1 if pairs.numel() else 0) + 2 + 1 + (1 if max_splits > 1 else 0)
 
     # ---- device-resident timed region
+    # The step is captured once into two CUDA graphs (cache kernels; decode
+    # call) and replayed, as a serving engine runs its decode step: this
+    # keeps Python's launch overhead out of the device timeline, so the
+    # events between the two replays time the decode kernels themselves.
     for _ in range(args.warmup):
         flush.zero_()
         cache_part()
         decode_part()
+    torch.cuda.synchronize()
+    graphs = None
+    try:
+        g_cache, g_decode = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_cache):
+            cache_part()
+        with torch.cuda.graph(g_decode):
+            decode_part()
+        torch.cuda.synchronize()
+        graphs = (g_cache, g_decode)
+        run_cache, run_decode = g_cache.replay, g_decode.replay
+        for _ in range(2):
+            run_cache()
+            run_decode()
+    except Exception as exc:  # capture unavailable: time the direct calls
+        print(f"bench: CUDA graph capture failed ({exc}); timing direct calls", file=sys.stderr)
+        run_cache, run_decode = cache_part, decode_part
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     torch.cuda.synchronize()
     barrier(world)
@@ -349,9 +372,9 @@ def run_ours(args):
         for i in range(args.steps):
             flush.zero_()
             ev[i][0].record(stream)
-            cache_part()
+            run_cache()
             ev[i][1].record(stream)
-            decode_part()
+            run_decode()
             ev[i][2].record(stream)
         torch.cuda.synchronize()
         barrier(world)
@@ -362,18 +385,28 @@ def run_ours(args):
     ms_dec = max_over_ranks(sum(dec_ms) / len(dec_ms), world)
     assert pa.pa_read_error_flag() == 0, "device error during the timed steps"
 
-    # ---- contiguous-cache variant of the same kernel on the same lengths (paging overhead)
+    # ---- contiguous-cache variant of the same kernel on the same lengths (paging overhead),
+    # timed the same way (graph replay)
     L_pad = -(-max_len // 32) * 32
     k_c = torch.empty(B, Hkv, L_pad, D, dtype=w.dtype, device=dev).normal_()
     v_c = torch.empty_like(k_c).normal_()
     out_c = torch.empty_like(out)
+    contig = lambda: pa.pa_paged_attention_decode_contiguous(case.q, k_c, v_c, lens, max_len, case.scale, out_c,
+                                                             block_size=bs, partition_size=part, workspace=ws)
+    contig()
+    torch.cuda.synchronize()
+    run_contig = contig
+    if graphs is not None:
+        g_contig = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_contig):
+            contig()
+        run_contig = g_contig.replay
     contig_ms = []
     for i in range(args.warmup + min(args.steps, 200)):
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        pa.pa_paged_attention_decode_contiguous(case.q, k_c, v_c, lens, max_len, case.scale, out_c, block_size=bs,
-                                                partition_size=part, workspace=ws)
+        run_contig()
         e1.record(stream)
         if i >= args.warmup:
             contig_ms.append((e0, e1))
@@ -381,7 +414,9 @@ def run_ours(args):
     ms_contig = max_over_ranks(sum(a.elapsed_time(b_) for a, b_ in contig_ms) / len(contig_ms), world)
     paged_med = statistics.median(dec_ms)
     contig_med = statistics.median(a.elapsed_time(b_) for a, b_ in contig_ms)
-    del k_c, v_c
+    del k_c, v_c, run_contig
+    if graphs is not None:
+        del g_contig
 
     # ---- end to end through the public API with host buffers
     pin = lambda t: t.detach().to("cpu").pin_memory()
@@ -448,6 +483,8 @@ def run_ours(args):
         "e2e": {"value": world * kv_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
         "gpu_launches": launches_per_step * args.steps,
+        "timing": "CUDA graph replay of the step (cache kernels, decode call), events between the replays"
+                  if graphs is not None else "direct calls",
         "clocks": clk,
         "wall_s_timed_region": t_wall,
         "cpu_baseline": cpu,
