@@ -3,18 +3,22 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 A step is one decode step of one attention layer over one batch: the new
-token's slot (pa_decode_slot_mapping), its K/V write (pa_reshape_and_cache),
-copy-on-write copies when the workload has them (pa_copy_blocks), and paged
-decode attention over every sequence (pa_paged_attention_decode, pass 1 plus
-the split-KV merge when a sequence is split).  Inputs are seeded synthetic
-tensors shaped like the named workload, resident in HBM before timing.
+token's slot and its K/V write (pa_reshape_and_cache_decode, one launch; the
+workloads that append several tokens per sequence use pa_slot_mapping and
+pa_reshape_and_cache), copy-on-write copies when the workload has them
+(pa_copy_blocks), and paged decode attention over every sequence
+(pa_paged_attention_decode, pass 1 plus the split-KV merge when a sequence is
+split).  Inputs are seeded synthetic tensors shaped like the named workload,
+resident in HBM before timing.
 
-Timing: W untimed warm-up steps, then the step is captured into CUDA graphs
-(the cache kernels, the decode call) and K replays are timed, each bracketed
-by CUDA events on the launching stream, with a 256 MiB write between steps
-(outside the events) to flush the 126 MB L2; the region is bracketed by a
-barrier and torch.cuda.synchronize(); the reported time is the max over
-ranks.  The end-to-end figure goes through the plain Python API instead.
+Timing: W untimed warm-up steps, then the step is captured into a CUDA graph
+and K replays are timed, each bracketed by CUDA events on the launching
+stream; then the decode call alone, captured into its own graph, is timed the
+same way for the roofline.  Between replays (outside the events) 256 MiB are
+written and another 256 MiB read, which leaves the 126 MB L2 holding none of
+the step's data and no dirty lines.  The region is bracketed by a barrier and
+torch.cuda.synchronize(); the reported time is the max over ranks.  The
+end-to-end figure goes through the plain Python API instead.
 
 value  = K/V bytes attention reads (tokens < length, K and V) / step time,
          summed over ranks (each rank runs its own batch: weak scaling, no
@@ -318,51 +322,65 @@ def run_ours(args):
     ws_bytes = pa.pa_paged_attention_workspace_size(B, Hq, Hkv, D, max_len, bs, part)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    clean = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     plain_decode = pairs.numel() == 0 and case.new_seq_ids.numel() == B
 
     def cache_part():
         if pairs.numel():
             pa.pa_copy_blocks(case.k_pool, case.v_pool, pairs)
         if plain_decode:
-            pa.pa_decode_slot_mapping(bt, lens, bs, slots)
+            # slot mapping and cache write of the step's one token per sequence, one launch
+            pa.pa_reshape_and_cache_decode(case.k_new, case.v_new, case.k_pool, case.v_pool, bt, lens, slots)
         else:
             pa.pa_slot_mapping(bt, sid, pos, bs, slots)
-        pa.pa_reshape_and_cache(case.k_new, case.v_new, case.k_pool, case.v_pool, slots)
+            pa.pa_reshape_and_cache(case.k_new, case.v_new, case.k_pool, case.v_pool, slots)
 
     def decode_part():
         pa.pa_paged_attention_decode(case.q, case.k_pool, case.v_pool, bt, lens, max_len, case.scale, out,
                                      partition_size=part, workspace=ws)
 
-    max_splits = -(-max(max_len, 1) // part)
-    launches_per_step = (1 if pairs.numel() else 0) + 2 + 1 + (1 if max_splits > 1 else 0)
-
-    # ---- device-resident timed region
-    # The step is captured once into two CUDA graphs (cache kernels; decode
-    # call) and replayed, as a serving engine runs its decode step: this
-    # keeps Python's launch overhead out of the device timeline, so the
-    # events between the two replays time the decode kernels themselves.
-    for _ in range(args.warmup):
-        flush.zero_()
+    def step():
         cache_part()
         decode_part()
+
+    def flush_l2():
+        # write a buffer twice the L2, then read another one, so that the
+        # step starts with the L2 holding none of its inputs and no dirty
+        # lines whose write-back it would pay for
+        flush.zero_()
+        clean.sum()
+
+    max_splits = -(-max(max_len, 1) // part)
+    cache_launches = (1 if pairs.numel() else 0) + (1 if plain_decode else 2)
+    decode_launches = 1 + (1 if max_splits > 1 else 0)
+
+    # ---- device-resident timed region
+    # The step is captured once into a CUDA graph and replayed, as a serving
+    # engine runs its decode step: Python's launch overhead stays out of the
+    # device timeline and the kernels' programmatic launches overlap each
+    # kernel's start with the previous one's drain.  The decode call alone is
+    # captured into a second graph and timed the same way, for the roofline.
+    for _ in range(args.warmup):
+        flush_l2()
+        step()
     torch.cuda.synchronize()
     graphs = None
     try:
-        g_cache, g_decode = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_cache):
-            cache_part()
+        g_step, g_decode = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_step):
+            step()
         with torch.cuda.graph(g_decode):
             decode_part()
         torch.cuda.synchronize()
-        graphs = (g_cache, g_decode)
-        run_cache, run_decode = g_cache.replay, g_decode.replay
+        graphs = (g_step, g_decode)
+        run_step, run_decode = g_step.replay, g_decode.replay
         for _ in range(2):
-            run_cache()
+            run_step()
             run_decode()
     except Exception as exc:  # capture unavailable: time the direct calls
         print(f"bench: CUDA graph capture failed ({exc}); timing direct calls", file=sys.stderr)
-        run_cache, run_decode = cache_part, decode_part
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+        run_step, run_decode = step, decode_part
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     torch.cuda.synchronize()
     barrier(world)
     with ClockSampler(torch.cuda.current_device()) as clocks:
@@ -370,17 +388,20 @@ def run_ours(args):
         barrier(world)
         t_wall = time.perf_counter()
         for i in range(args.steps):
-            flush.zero_()
+            flush_l2()
             ev[i][0].record(stream)
-            run_cache()
+            run_step()
             ev[i][1].record(stream)
-            run_decode()
+        for i in range(args.steps):
+            flush_l2()
             ev[i][2].record(stream)
+            run_decode()
+            ev[i][3].record(stream)
         torch.cuda.synchronize()
         barrier(world)
         t_wall = time.perf_counter() - t_wall
-    step_ms = [a.elapsed_time(c) for a, _, c in ev]
-    dec_ms = [b_.elapsed_time(c) for _, b_, c in ev]
+    step_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    dec_ms = [e[2].elapsed_time(e[3]) for e in ev]
     ms_step = max_over_ranks(sum(step_ms) / len(step_ms), world)
     ms_dec = max_over_ranks(sum(dec_ms) / len(dec_ms), world)
     assert pa.pa_read_error_flag() == 0, "device error during the timed steps"
@@ -403,7 +424,7 @@ def run_ours(args):
         run_contig = g_contig.replay
     contig_ms = []
     for i in range(args.warmup + min(args.steps, 200)):
-        flush.zero_()
+        flush_l2()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         run_contig()
@@ -429,7 +450,7 @@ def run_ours(args):
     d2h = h_out.numel() * h_out.element_size()
     e2e_ev = []
     for i in range(args.warmup + args.steps):
-        flush.zero_()
+        flush_l2()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for dst, src in ((d_q, h_q), (d_kn, h_kn), (d_vn, h_vn), (d_bt, h_bt), (d_lens, h_lens)):
@@ -470,8 +491,9 @@ def run_ours(args):
         "config": {"workload": DESCRIPTIONS[args.workload] + (f" (batch overridden to {B})" if args.batch else ""),
                    "batch_per_gpu": B, "partition_tokens": part,
                    "max_splits": max_splits, "kv_bytes_per_step": kv_bytes,
-                   "l2": "flushed between steps by a 256 MiB write outside the timed events; "
-                         "K/V read per step also exceeds the 126 MB L2",
+                   "l2": "flushed between steps outside the timed events (256 MiB written, then another "
+                         "256 MiB read, so no dirty line is written back inside the step); K/V read per "
+                         "step also exceeds the 126 MB L2",
                    "parallelism": f"{world} independent replicas (sequences sharded, no collective)"},
         "tokens_per_s": world * B / (ms_step * 1e-3),
         "decode_attention_ms": ms_dec,
@@ -482,9 +504,10 @@ def run_ours(args):
                             "overhead": paged_med / contig_med - 1.0, "contiguous_ms_mean_max_ranks": ms_contig},
         "e2e": {"value": world * kv_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
-        "gpu_launches": launches_per_step * args.steps,
-        "timing": "CUDA graph replay of the step (cache kernels, decode call), events between the replays"
-                  if graphs is not None else "direct calls",
+        "gpu_launches": (cache_launches + decode_launches) * args.steps,
+        "gpu_launches_decode_roofline_loop": decode_launches * args.steps,
+        "timing": ("K replays of the step's CUDA graph (value), then K replays of the decode call's graph "
+                   "(roofline), each bracketed by events" if graphs is not None else "direct calls"),
         "clocks": clk,
         "wall_s_timed_region": t_wall,
         "cpu_baseline": cpu,

@@ -123,6 +123,29 @@ int pa_reshape_and_cache(const void* key, const void* value, void* k_pool, void*
                          void* stream);
 
 /*
+ * pa_reshape_and_cache_decode -- pa_decode_slot_mapping and
+ * pa_reshape_and_cache of one decode step in a single launch ([P3] "Detail"
+ * for the slot, "Key Technical Innovations" item 2 for the write): token b
+ * is position context_lens[b] - 1 of sequence b, its slot is
+ * block_tables[b][pos / bs] * bs + pos % bs, and its K and V rows go there.
+ *   key, value    [batch][num_kv_heads][head_dim]   (dtype)
+ *   block_tables  int32 [batch][max_blocks_per_seq]
+ *   context_lens  int32 [batch], lengths INCLUDING the token being written
+ *   slot_mapping  int64 [batch] output, or NULL: the slot each token got,
+ *                 exactly as pa_decode_slot_mapping computes it
+ * Length 0 writes nothing (slot -1).  A negative length, an unmapped
+ * position or a block outside [0, num_blocks) writes nothing and records
+ * PA_ERR_BAD_BLOCK_ID.  Pool contents after the call are bit-identical to
+ * the two-call sequence.  Launched with programmatic stream serialisation,
+ * so a following pa_paged_attention_decode can be scheduled while it drains.
+ */
+int pa_reshape_and_cache_decode(const void* key, const void* value, void* k_pool, void* v_pool,
+                                const int32_t* block_tables, int max_blocks_per_seq,
+                                const int32_t* context_lens, int batch, int num_kv_heads,
+                                int head_dim, int block_size, int64_t num_blocks, int dtype,
+                                int64_t* slot_mapping, void* stream);
+
+/*
  * pa_copy_blocks -- copy-on-write duplication of shared blocks ([P2] "Key
  * terms in this lesson", Copy-on-write: a block is shared until someone
  * writes to it, and the writer then gets a private copy; [P1] "Myths and

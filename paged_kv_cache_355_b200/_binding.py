@@ -36,6 +36,7 @@ _SIGS = {
     "pa_slot_mapping": ([_P, _I, _I, _P, _P, _I64, _I, _P, _P], _I),
     "pa_decode_slot_mapping": ([_P, _I, _P, _I, _I, _P, _P], _I),
     "pa_reshape_and_cache": ([_P, _P, _P, _P, _P, _I64, _I, _I, _I, _I64, _I, _P], _I),
+    "pa_reshape_and_cache_decode": ([_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I64, _I, _P, _P], _I),
     "pa_copy_blocks": ([_P, _P, _P, _I64, _I, _I, _I, _I64, _I, _P], _I),
     "pa_swap_blocks": ([_P, _P, _P, _P, _P, _I64, _I, _I, _I, _I64, _I64, _I, _P], _I),
     "pa_paged_attention_partition_size": ([_I, _I, _I, _I, _I, _I, ctypes.POINTER(_I)], _I),
@@ -144,6 +145,24 @@ def pa_reshape_and_cache(key, value, k_pool, v_pool, slot_mapping, stream=None) 
     _check("pa_reshape_and_cache", _lib.pa_reshape_and_cache(
         _dev(key, "key"), value.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
         _dev(slot_mapping, "slot_mapping", torch.int64), T, Hkv, D, bs, NB, dt, _stream(stream)))
+
+
+def pa_reshape_and_cache_decode(key, value, k_pool, v_pool, block_tables, context_lens, slot_mapping=None,
+                                stream=None) -> None:
+    B, Hkv, D = key.shape
+    NB, Hkv2, bs, D2 = k_pool.shape
+    if (Hkv2, D2) != (Hkv, D) or value.shape != key.shape or v_pool.shape != k_pool.shape:
+        raise ValueError("key/value and pool shapes disagree")
+    if block_tables.shape[0] != B or context_lens.numel() != B:
+        raise ValueError("block_tables / context_lens do not match the batch of key")
+    dt = _kv_dtype(key)
+    for t, n in ((value, "value"), (k_pool, "k_pool"), (v_pool, "v_pool")):
+        _dev(t, n, key.dtype)
+    slots = 0 if slot_mapping is None else _dev(slot_mapping, "slot_mapping", torch.int64)
+    _check("pa_reshape_and_cache_decode", _lib.pa_reshape_and_cache_decode(
+        _dev(key, "key"), value.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
+        _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+        _dev(context_lens, "context_lens", torch.int32), B, Hkv, D, bs, NB, dt, slots or None, _stream(stream)))
 
 
 def pa_copy_blocks(k_pool, v_pool, block_mapping, stream=None) -> None:

@@ -87,6 +87,49 @@ __global__ void reshape_and_cache_kernel(const uint4* __restrict__ key, const ui
     }
 }
 
+// Decode step, slot mapping and cache write in one pass: token b is position
+// context_lens[b] - 1 of sequence b; every thread of its rows derives the slot
+// from the table itself, so no slot array has to round-trip through memory
+// between two launches.  The thread owning vector 0 of token b stores the
+// slot (if asked) and records a bad table entry.
+__global__ void decode_append_kernel(const uint4* __restrict__ key, const uint4* __restrict__ value,
+                                     uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
+                                     const int32_t* __restrict__ block_tables, int max_blocks_per_seq,
+                                     const int32_t* __restrict__ context_lens, int batch, int num_kv_heads,
+                                     int row_vecs, int block_size, int64_t num_blocks, int64_t* __restrict__ slots,
+                                     int* err) {
+    griddep_wait();
+    griddep_launch_dependents();
+    const int64_t per_token = (int64_t)num_kv_heads * row_vecs;
+    const int64_t total = (int64_t)batch * per_token;
+    for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int b = (int)(idx / per_token);
+        const int64_t rem = idx - (int64_t)b * per_token;
+        const int L = context_lens[b];
+        int64_t blk = -1;
+        int off = 0;
+        if (L > 0 && (L - 1) / block_size < max_blocks_per_seq) {
+            const int pos = L - 1;
+            blk = block_tables[(int64_t)b * max_blocks_per_seq + pos / block_size];
+            off = pos % block_size;
+        }
+        // the slot as pa_decode_slot_mapping gives it; the write also needs
+        // the block inside the pool
+        const bool ok = blk >= 0 && blk < num_blocks;
+        if (rem == 0) {
+            if (slots) slots[b] = blk >= 0 ? blk * block_size + off : -1;
+            if (!ok && L != 0) record_error(err, PA_ERR_BAD_BLOCK_ID);
+        }
+        if (!ok) continue;
+        const int h = (int)(rem / row_vecs);
+        const int c = (int)(rem - (int64_t)h * row_vecs);
+        const int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * row_vecs + c;
+        k_pool[dst] = key[idx];
+        v_pool[dst] = value[idx];
+    }
+}
+
 // blockIdx.x = pair; blockIdx.y strides over the block's 16-byte vectors.
 // Source and destination pools may be the same pool (copy-on-write) or two
 // pools, one of them in pinned host memory mapped into the device address
@@ -203,6 +246,28 @@ extern "C" int pa_reshape_and_cache(const void* key, const void* value, void* k_
         static_cast<const uint4*>(key), static_cast<const uint4*>(value), static_cast<uint4*>(k_pool),
         static_cast<uint4*>(v_pool), slot_mapping, num_tokens, num_kv_heads, row_vecs, block_size, num_blocks, err);
     return launch_status();
+}
+
+extern "C" int pa_reshape_and_cache_decode(const void* key, const void* value, void* k_pool, void* v_pool,
+                                           const int32_t* block_tables, int max_blocks_per_seq,
+                                           const int32_t* context_lens, int batch, int num_kv_heads, int head_dim,
+                                           int block_size, int64_t num_blocks, int dtype, int64_t* slot_mapping,
+                                           void* stream) {
+    if (batch < 0 || max_blocks_per_seq < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        num_blocks < 0 || !valid_dtype(dtype))
+        return PA_ERR_INVALID_ARG;
+    if (!supported_head_dim(head_dim) || !supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
+    if (batch == 0) return PA_OK;
+    if (!key || !value || !k_pool || !v_pool || !block_tables || !context_lens) return PA_ERR_INVALID_ARG;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(k_pool) || !aligned16(v_pool))
+        return PA_ERR_INVALID_ARG;
+    int* err = error_word_ptr();
+    if (!err) return PA_ERR_CUDA;
+    const int row_vecs = (int)(head_dim * dtype_bytes(dtype) / 16);
+    return launch_pdl(decode_append_kernel, dim3(grid_for((int64_t)batch * num_kv_heads * row_vecs)), dim3(kThreads),
+                      0, (cudaStream_t)stream, static_cast<const uint4*>(key), static_cast<const uint4*>(value),
+                      static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), block_tables, max_blocks_per_seq,
+                      context_lens, batch, num_kv_heads, row_vecs, block_size, num_blocks, slot_mapping, err);
 }
 
 extern "C" int pa_copy_blocks(void* k_pool, void* v_pool, const int64_t* block_mapping, int64_t num_pairs,

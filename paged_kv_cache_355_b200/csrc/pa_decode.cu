@@ -259,6 +259,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const Deco
     uint8_t* ring = smem + p.ring_offset;
     __shared__ int s_abort;
 
+    griddep_wait();  // q, lengths, tables and the pool may come from the kernel before
+    griddep_launch_dependents();
     const int split = blockIdx.x;
     const int kvh = blockIdx.y;
     const int b = schedule_sequence(p, ring);
@@ -524,6 +526,12 @@ __global__ void __launch_bounds__(kDecodeThreads)
     uint8_t* ring = smem + p.ring_offset + ((1024u - (smem_addr(smem) & 1023u)) & 1023u);
     __shared__ int s_abort;
 
+    if (threadIdx.x == 0) {
+        prefetch_tmap(&tmk);
+        prefetch_tmap(&tmv);
+    }
+    griddep_wait();  // q, lengths, tables and the pool may come from the kernel before
+    griddep_launch_dependents();
     const int split = blockIdx.x;
     const int kvh = blockIdx.y;
     const int b = schedule_sequence(p, ring);
@@ -540,8 +548,6 @@ __global__ void __launch_bounds__(kDecodeThreads)
 
     if (threadIdx.x == 0) {
         s_abort = 0;
-        prefetch_tmap(&tmk);
-        prefetch_tmap(&tmv);
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
@@ -832,6 +838,7 @@ template <int D>
 __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(const DecodeParams p, int64_t rows) {
     constexpr int VPL = D / 32;  // output elements per lane
     const int lane = threadIdx.x & 31;
+    griddep_wait();  // the partial rows come from pass 1
     const int64_t row = (int64_t)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);  // b * Hq + h
     if (row >= rows) return;
     const int b = (int)(row / p.num_q_heads);
@@ -969,8 +976,7 @@ int launch_pass1_mma(const DecodeParams& p, const CUtensorMap& tmk, const CUtens
             return PA_ERR_CUDA;
         configured.fetch_or(bit);
     }
-    decode_pass1_mma_kernel<D, NT><<<grid, kDecodeThreads, smem, st>>>(p, tmk, tmv);
-    return launch_status();
+    return launch_pdl(decode_pass1_mma_kernel<D, NT>, grid, dim3(kDecodeThreads), smem, st, p, tmk, tmv);
 }
 
 template <typename T, int D, int G>
@@ -985,8 +991,7 @@ int launch_pass1(const DecodeParams& p, dim3 grid, size_t smem, cudaStream_t st)
             return PA_ERR_CUDA;
         configured.fetch_or(bit);
     }
-    decode_pass1_kernel<T, D, G><<<grid, kDecodeThreads, smem, st>>>(p);
-    return launch_status();
+    return launch_pdl(decode_pass1_kernel<T, D, G>, grid, dim3(kDecodeThreads), smem, st, p);
 }
 
 template <typename T, int D>
@@ -1064,11 +1069,8 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
     if (plan.max_splits > 1) {
         const int64_t rows = (int64_t)batch * p.num_q_heads;
         const unsigned blocks = (unsigned)((rows + kMergeWarps - 1) / kMergeWarps);
-        if (head_dim == 128)
-            decode_merge_kernel<128><<<blocks, 32 * kMergeWarps, 0, st>>>(p, rows);
-        else
-            decode_merge_kernel<64><<<blocks, 32 * kMergeWarps, 0, st>>>(p, rows);
-        rc = launch_status();
+        rc = head_dim == 128 ? launch_pdl(decode_merge_kernel<128>, dim3(blocks), dim3(32 * kMergeWarps), 0, st, p, rows)
+                             : launch_pdl(decode_merge_kernel<64>, dim3(blocks), dim3(32 * kMergeWarps), 0, st, p, rows);
     }
     return rc;
 }

@@ -33,6 +33,18 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
 }
 
+// Programmatic dependent launch.  A kernel launched with the programmatic
+// stream-serialisation attribute may be scheduled while the kernel before it
+// on the stream is still finishing; griddep_wait() blocks until that kernel
+// has completed and its writes are visible, so every global read and write of
+// such a kernel comes after it (only shared-memory set-up may precede it).
+// Without the attribute griddep_wait() returns at once.
+// griddep_launch_dependents() lets the next such kernel be scheduled early.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Make barrier initialisation visible to the async (bulk-copy) proxy.
 __device__ __forceinline__ void fence_barrier_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");

@@ -7,24 +7,30 @@
 // are read from the block pool through the block table ("PagedAttention and
 // KV memory management", "The kernel side"), never gathered.
 //
-// Work item = 128 query rows of one (sequence, kv head): 128 / G query tokens
-// x the G query heads that share the kv head, one CTA each.  Per CTA:
-//  * warp 0 loads the Q tile once (tiled TMA, 3-D map over q [T, Hq, D]) and
-//    streams K/V tiles of 64 tokens through a 4-stage ring (tiled TMA boxes
-//    of block_size rows from the pool, 128-byte swizzle);
-//  * warp 1 allocates tensor memory and issues the MMAs from one thread:
-//        S_j = Q . K_j^T        (M = 128 rows, N = 64 keys, K = D)
-//        O  += P_j . V_j        (M = 128 rows, N = D, K = 64 keys)
-//    S is double-buffered in TMEM so S_{j+1} runs while the softmax works on
-//    S_j; O accumulates in TMEM across tiles;
-//  * warps 2..5 (128 threads, one query row each: TMEM lane = row) load S_j,
-//    apply the causal mask and scale, keep the row's running max and sum in
-//    registers, rescale O in TMEM only when the max has grown by more than
-//    2^8 (lazy rescale), and write P_j to one of two shared-memory buffers as
-//    a bf16 high part plus a bf16 residual (both multiplied by V, so the
-//    weights keep ~16 significant bits); the softmax of tile j + 1 thus runs
-//    while the tensor core does P_j . V_j.  At the end they read O, divide by
-//    the row sum and store the row.
+// Query tile = 128 query rows of one (sequence, kv head): 128 / G query
+// tokens x the G query heads that share the kv head.  One CTA takes two
+// neighbouring tiles, which need (almost) the same keys:
+//  * warp 0 loads both Q tiles once (tiled TMA, 3-D map over q [T, Hq, D])
+//    and streams K/V tiles of 64 tokens through a 4-stage ring (tiled TMA
+//    boxes of block_size rows from the pool, 128-byte swizzle), each tile
+//    used by both query tiles;
+//  * warp 1 allocates all 512 tensor-memory columns and issues the MMAs from
+//    one thread, per query tile t:
+//        S_tj = Q_t . K_j^T       (M = 128 rows, N = 64 keys, K = D)
+//        O_t += P_tj . V_j        (M = 128 rows, N = D, K = 64 keys)
+//    S is double-buffered in tensor memory, so S_t,j+1 runs while the
+//    softmax works on S_tj, and P_tj is written back over S_tj's columns and
+//    read by the P.V MMA straight from tensor memory;
+//  * warps 2..5 and 6..9 are the two tiles' softmax warpgroups (one query
+//    row per thread: TMEM lane = row).  Each loads S_tj, applies the causal
+//    mask and scale, keeps its row's running max and sum in registers,
+//    rescales O in tensor memory only when the max has grown by more than
+//    2^8 (lazy rescale), and stores P as a bf16 high part plus a bf16
+//    residual (both multiplied by V, so the weights keep ~16 significant
+//    bits).  With two warpgroups per CTA one tile's softmax overlaps the
+//    other tile's MMAs.  At the end they read O, divide by the row sum and
+//    store the row.
+// The heaviest pairs of tiles (latest query tokens, most keys) start first.
 // Every wait is a bounded mbarrier wait; on expiry the CTA records
 // PA_ERR_TIMEOUT and winds down (tensor memory is always released).
 #include <cuda.h>
@@ -44,9 +50,11 @@
 namespace pa {
 namespace {
 
-constexpr int kRows = 128;    // query rows per CTA (TMEM lanes)
+constexpr int kRows = 128;    // query rows per tile (TMEM lanes)
+constexpr int kTiles = 2;     // query tiles per CTA
 constexpr int kKeys = 64;     // keys per tile
-constexpr int kThreads = 192;  // producer, MMA, 4 softmax warps
+constexpr int kThreads = 64 + kTiles * 128;  // producer, MMA, one softmax warpgroup per query tile
+static_assert(kTiles == 2, "the softmax warpgroups select their tile's values between two");
 constexpr int kStages = 4;     // K/V ring depth
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.f;  // lazy-rescale threshold of the running max (log2 units)
@@ -91,6 +99,16 @@ __device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t da, uint64_t db, 
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
         "l"(da), "l"(db), "r"(idesc), "r"(accumulate));
+}
+
+// the same with A (the M x K operand) read from tensor memory: row r of A is
+// lane r, two bf16 per 32-bit column along K
+__device__ __forceinline__ void umma_tmem_a(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(db), "r"(idesc), "r"(accumulate));
 }
 
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -141,6 +159,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+        "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+        "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -153,32 +182,36 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, in
 }
 
 // ---- the kernel ------------------------------------------------------------
+// Two query tiles per CTA (tiles 2x and 2x + 1 of one (sequence, kv head)),
+// each with its own softmax warpgroup, S double buffer and O accumulator in
+// tensor memory; the K/V tiles they both need are loaded once.  While one
+// warpgroup works on its scores the tensor core runs the other tile's MMAs.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmq,
                       const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
     constexpr int SLABS = D / 64;
-    constexpr int Q_BYTES = SLABS * kRows * 128;     // 128 rows x D
-    constexpr int KV_SLAB = kKeys * 128;             // 64 rows x 64 elements
-    constexpr int KV_BYTES = SLABS * KV_SLAB;        // one of K or V for one tile
-    constexpr int P_BYTES = kRows * 128;             // 128 rows x 64 keys (bf16)
-    constexpr int S_COLS = kKeys;                    // TMEM columns of one S buffer
-    constexpr uint32_t O_COL = 2 * S_COLS;           // O after the two S buffers
-    constexpr uint32_t TMEM_COLS = 2 * S_COLS + D <= 256 ? 256 : 512;
+    constexpr int Q_BYTES = SLABS * kRows * 128;  // 128 rows x D
+    constexpr int KV_SLAB = kKeys * 128;          // 64 rows x 64 elements
+    constexpr int KV_BYTES = SLABS * KV_SLAB;     // one of K or V for one tile
+    constexpr int S_COLS = kKeys;                 // TMEM columns of one S buffer
+    constexpr uint32_t O_COL = 2 * S_COLS;        // O after the tile's two S buffers
+    constexpr uint32_t TILE_COLS = 256;           // TMEM columns per query tile
+    static_assert(O_COL + D <= TILE_COLS, "tensor-memory layout");
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-    uint8_t* sQ = smem;
-    uint8_t* sK = sQ + Q_BYTES;                  // [kStages][KV_BYTES]
+    uint8_t* sQ = smem;                          // [kTiles][Q_BYTES]
+    uint8_t* sK = sQ + kTiles * Q_BYTES;         // [kStages][KV_BYTES]
     uint8_t* sV = sK + kStages * KV_BYTES;       // [kStages][KV_BYTES]
-    uint8_t* sPh = sV + kStages * KV_BYTES;      // P high part, [2][P_BYTES]
-    uint8_t* sPl = sPh + 2 * P_BYTES;      // P residual,  [2][P_BYTES]
 
-    __shared__ uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[2], s_free[2], p_full[2], pv_done[2];
+    __shared__ uint64_t q_full, kv_full[kStages], kv_empty[kStages];
+    __shared__ uint64_t s_full[kTiles][2], p_full[kTiles][2], pv_done[kTiles][2];
     __shared__ uint32_t tmem_base;
     __shared__ int s_abort;
 
-    const int qtile = blockIdx.x;
+    // heaviest pairs (latest query tokens, most keys) first
+    const int pair = gridDim.x - 1 - blockIdx.x;
     const int kvh = blockIdx.y;
     const int b = blockIdx.z;
     const int warp = threadIdx.x >> 5;
@@ -189,16 +222,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q0 = p.query_start[b];
     const int n = p.query_start[b + 1] - q0;
     const int L = p.context_lens[b];
-    const int t0 = qtile * TQ;
-    if (t0 >= n) return;  // uniform over the CTA
+    if (pair * kTiles * TQ >= n) return;  // uniform over the CTA
     if (n > L || (int64_t)L > (int64_t)p.max_blocks_per_seq * p.block_size) {
-        if (threadIdx.x == 0 && qtile == 0 && kvh == 0) record_error(p.err, PA_ERR_BAD_BLOCK_ID);
+        if (threadIdx.x == 0 && pair == 0 && kvh == 0) record_error(p.err, PA_ERR_BAD_BLOCK_ID);
         return;
     }
-    const int nq = min(TQ, n - t0);
-    const int pos_first = L - n + t0;        // position of the tile's first query token
-    const int n_kv = pos_first + nq;         // keys the tile needs: 0 .. pos_first + nq - 1
-    const int nt = (n_kv + kKeys - 1) / kKeys;
+    // per tile: first query token, tokens, position of the first one, key tiles
+    int t0[kTiles], nq[kTiles], pos_first[kTiles], nt[kTiles];
+    int n_kv = 0, nt_cta = 0;
+#pragma unroll
+    for (int t = 0; t < kTiles; ++t) {
+        t0[t] = (pair * kTiles + t) * TQ;
+        nq[t] = max(0, min(TQ, n - t0[t]));
+        pos_first[t] = L - n + t0[t];
+        nt[t] = nq[t] > 0 ? (pos_first[t] + nq[t] + kKeys - 1) / kKeys : 0;
+        if (nq[t] > 0) n_kv = pos_first[t] + nq[t];
+        nt_cta = max(nt_cta, nt[t]);
+    }
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -210,17 +250,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&kv_full[s], 1);
             mbar_init(&kv_empty[s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&s_full[s], 1);
-            mbar_init(&s_free[s], 4);
-            mbar_init(&p_full[s], 128);
-            mbar_init(&pv_done[s], 1);
-        }
+        for (int t = 0; t < kTiles; ++t)
+            for (int s = 0; s < 2; ++s) {
+                mbar_init(&s_full[t][s], 1);
+                mbar_init(&p_full[t][s], 128);
+                mbar_init(&pv_done[t][s], 1);
+            }
         fence_barrier_init();
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&tmem_base)),
-                     "r"(TMEM_COLS));
+                     "r"(kTiles * TILE_COLS));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     tc_fence_before();
@@ -233,13 +273,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int bs = p.block_size;
         const int boxes = kKeys / bs;  // pool boxes per tile and slab
         if (lane == 0) {
-            mbar_arrive_expect_tx(&q_full, (uint32_t)Q_BYTES);
+            uint32_t qbytes = 0;
 #pragma unroll
-            for (int sl = 0; sl < SLABS; ++sl)
-                tma_load_3d(sQ + sl * kRows * 128, &tmq, sl * 64, kvh * G, q0 + t0, &q_full);
+            for (int t = 0; t < kTiles; ++t) qbytes += nq[t] > 0 ? (uint32_t)Q_BYTES : 0u;
+            mbar_arrive_expect_tx(&q_full, qbytes);
+#pragma unroll
+            for (int t = 0; t < kTiles; ++t) {
+                if (nq[t] == 0) continue;
+#pragma unroll
+                for (int sl = 0; sl < SLABS; ++sl)
+                    tma_load_3d(sQ + t * Q_BYTES + sl * kRows * 128, &tmq, sl * 64, kvh * G, q0 + t0[t], &q_full);
+            }
         }
         const int32_t* table = p.block_tables + (int64_t)b * p.max_blocks_per_seq;
-        for (int j = 0; j < nt; ++j) {
+        const uint64_t policy = l2_policy_evict_first();
+        for (int j = 0; j < nt_cta; ++j) {
             const int s = j % kStages;
             if (j >= kStages) {
                 int ok = 1;
@@ -266,7 +314,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive_expect_tx(&kv_full[s], total);
             __syncwarp();
             if (bytes) {
-                const uint64_t policy = l2_policy_evict_first();
 #pragma unroll
                 for (int sl = 0; sl < SLABS; ++sl) {
                     tma_load_2d(sK + s * KV_BYTES + sl * KV_SLAB + lane * bs * 128, &tmk, sl * 64, y, &kv_full[s],
@@ -278,84 +325,104 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
+        // Step j issues S_j = Q_t . K_j^T for both tiles, then O_t += P_{j-1} . V_{j-1}
+        // once each warpgroup has written P_{j-1}.  tcgen05.mma ops from one
+        // thread run in issue order, so S_j may overwrite the buffer that
+        // held P_{j-2}: its P.V was issued one step earlier.
         if (lane == 0) {
             constexpr uint32_t IDESC_S = umma_idesc(kRows, kKeys, false);
             constexpr uint32_t IDESC_O = umma_idesc(kRows, D, true);
-            const uint32_t q_base = smem_addr(sQ);
             bool ok = mbar_wait(&q_full, 0, p.err);
-            auto issue_s = [&](int j) -> bool {
-                const int s = j & 1;  // S buffer
-                const int ks = j % kStages;
-                if (!mbar_wait(&kv_full[ks], (j / kStages) & 1, p.err)) return false;
-                if (j >= 2 && !mbar_wait(&s_free[s], ((j >> 1) - 1) & 1, p.err)) return false;
-                tc_fence_after();
-                const uint32_t k_base = smem_addr(sK + ks * KV_BYTES);
+            for (int j = 0; ok && j <= nt_cta; ++j) {
+                if (j < nt_cta) {
+                    const int ks = j % kStages;
+                    if (!(ok = mbar_wait(&kv_full[ks], (j / kStages) & 1, p.err))) break;
+                    tc_fence_after();
+                    const uint32_t k_base = smem_addr(sK + ks * KV_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk & 3) * 32;
-                    const uint64_t da = umma_desc(q_base + (kk >> 2) * (kRows * 128) + off, 16, 1024);
-                    const uint64_t db = umma_desc(k_base + (kk >> 2) * KV_SLAB + off, 16, 1024);
-                    umma(tmem + s * S_COLS, da, db, IDESC_S, kk > 0 ? 1u : 0u);
-                }
-                umma_commit(&s_full[s]);
-                return true;
-            };
-            if (ok) ok = issue_s(0);
-            for (int j = 0; ok && j < nt; ++j) {
-                if (j + 1 < nt && !(ok = issue_s(j + 1))) break;
-                if (!(ok = mbar_wait(&p_full[j & 1], (j >> 1) & 1, p.err))) break;
-                tc_fence_after();
-                const uint32_t v_base = smem_addr(sV + (j % kStages) * KV_BYTES);
+                    for (int t = 0; t < kTiles; ++t) {
+                        if (j >= nt[t]) continue;
+                        const uint32_t q_base = smem_addr(sQ + t * Q_BYTES);
+                        const uint32_t d_s = tmem + t * TILE_COLS + (j & 1) * S_COLS;
 #pragma unroll
-                for (int kk = 0; kk < kKeys / 16; ++kk) {
-                    const uint64_t db = umma_desc(v_base + kk * 2048, KV_SLAB, 1024);
-                    const uint64_t dh = umma_desc(smem_addr(sPh + (j & 1) * P_BYTES) + kk * 32, 16, 1024);
-                    const uint64_t dl = umma_desc(smem_addr(sPl + (j & 1) * P_BYTES) + kk * 32, 16, 1024);
-                    umma(tmem + O_COL, dh, db, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
-                    umma(tmem + O_COL, dl, db, IDESC_O, 1u);
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t off = (kk & 3) * 32;
+                            const uint64_t da = umma_desc(q_base + (kk >> 2) * (kRows * 128) + off, 16, 1024);
+                            const uint64_t db = umma_desc(k_base + (kk >> 2) * KV_SLAB + off, 16, 1024);
+                            umma(d_s, da, db, IDESC_S, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&s_full[t][j & 1]);
+                    }
                 }
-                umma_commit(&pv_done[j & 1]);
-                umma_commit(&kv_empty[j % kStages]);
+                if (j >= 1) {
+                    const int jp = j - 1;
+                    const uint32_t v_base = smem_addr(sV + (jp % kStages) * KV_BYTES);
+#pragma unroll
+                    for (int t = 0; t < kTiles; ++t) {
+                        if (jp >= nt[t]) continue;
+                        if (!(ok = mbar_wait(&p_full[t][jp & 1], (jp >> 1) & 1, p.err))) break;
+                        tc_fence_after();
+                        const uint32_t p_col = tmem + t * TILE_COLS + (jp & 1) * S_COLS;
+#pragma unroll
+                        for (int kk = 0; kk < kKeys / 16; ++kk) {
+                            const uint64_t db = umma_desc(v_base + kk * 2048, KV_SLAB, 1024);
+                            umma_tmem_a(tmem + t * TILE_COLS + O_COL, p_col + kk * 8, db, IDESC_O,
+                                        (jp > 0 || kk > 0) ? 1u : 0u);
+                            umma_tmem_a(tmem + t * TILE_COLS + O_COL, p_col + S_COLS / 2 + kk * 8, db, IDESC_O, 1u);
+                        }
+                        umma_commit(&pv_done[t][jp & 1]);
+                    }
+                    if (!ok) break;
+                    umma_commit(&kv_empty[jp % kStages]);
+                }
             }
             if (!ok) s_abort = 1;
         }
     } else {
         // ---------------- softmax / epilogue: one query row per thread ----------------
-        const int quarter = warp & 3;                 // TMEM lane quarter this warp may access
-        const int row = quarter * 32 + lane;          // query row of the tile = TMEM lane
-        const int tq = row / G;                       // query token within the tile
-        const bool valid = tq < nq;
-        const int limit = valid ? pos_first + tq : -1;  // last key this row may see
-        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-        float m = -INFINITY, l = 0.f;
+        const int t = (warp - 2) >> 2;               // query tile of this warpgroup
+        const int quarter = warp & 3;                // TMEM lane quarter this warp may access
+        const int row = quarter * 32 + lane;         // query row of the tile = TMEM lane
+        const int tq = row / G;                      // query token within the tile
+        const int my_t0 = t ? t0[1] : t0[0];
+        const bool valid = tq < (t ? nq[1] : nq[0]);
+        const int limit = valid ? (t ? pos_first[1] : pos_first[0]) + tq : -1;  // last key this row may see
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + t * TILE_COLS;
+        const int ntt = t ? nt[1] : nt[0];
+        float m = -INFINITY, l = 0.f;  // running max (log2 units, scaled) and sum
         bool ok = true;
-        for (int j = 0; j < nt; ++j) {
+        for (int j = 0; j < ntt; ++j) {
             const int s = j & 1;
-            if (!(ok = mbar_wait(&s_full[s], (j >> 1) & 1, p.err))) break;
+            if (!(ok = mbar_wait(&s_full[t][s], (j >> 1) & 1, p.err))) break;
             tc_fence_after();
             float sv[kKeys];
             tmem_ld32(lane_base + s * S_COLS, sv);
             tmem_ld32(lane_base + s * S_COLS + 32, sv + 32);
             tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_free[s]);
             const int kbase = j * kKeys;
-            float mx = -INFINITY;
-            if (__all_sync(0xffffffffu, kbase + kKeys - 1 <= limit)) {
-                // every key of the tile is visible to every row of this warp
+            // With a positive scale (the usual case) the row max is taken on
+            // the raw scores and the scale folds into the exponent's FMA;
+            // otherwise the scores are scaled first.  Masked keys are -inf
+            // either way.
+            const bool fold = p.scale_log2 > 0.f;
+            if (!fold) {
 #pragma unroll
-                for (int c = 0; c < kKeys; ++c) {
-                    sv[c] *= p.scale_log2;
-                    mx = fmaxf(mx, sv[c]);
-                }
-            } else {
-#pragma unroll
-                for (int c = 0; c < kKeys; ++c) {
-                    sv[c] = kbase + c <= limit ? sv[c] * p.scale_log2 : -INFINITY;
-                    mx = fmaxf(mx, sv[c]);
-                }
+                for (int c = 0; c < kKeys; ++c) sv[c] *= p.scale_log2;
             }
+            if (!__all_sync(0xffffffffu, kbase + kKeys - 1 <= limit)) {
+#pragma unroll
+                for (int c = 0; c < kKeys; ++c)
+                    if (kbase + c > limit) sv[c] = -INFINITY;
+            }
+            // row max in eight independent chains
+            float mx8[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) mx8[c] = sv[c];
+#pragma unroll
+            for (int c = 8; c < kKeys; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
+            float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            if (fold) mx *= p.scale_log2;
             // Lazy rescale: the weights are exp2(s - m) against a reference max
             // m that only moves when the row's max exceeds it by more than
             // kRescaleLog2 (weights stay <= 2^kRescaleLog2, far inside fp32 and
@@ -367,21 +434,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 alpha = m == -INFINITY ? 0.f : exp2f(m - mx);
                 m = mx;
             }
-            float sum = 0.f;
+            float sum8[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) sum8[c] = 0.f;
             if (m != -INFINITY) {
+                const float neg_m = -m;
+                const float mul = fold ? p.scale_log2 : 1.f;
 #pragma unroll
                 for (int c = 0; c < kKeys; ++c) {
-                    sv[c] = ex2_approx(sv[c] - m);
-                    sum += sv[c];
+                    sv[c] = ex2_approx(fmaf(sv[c], mul, neg_m));
+                    sum8[c & 7] += sv[c];
                 }
             } else {
 #pragma unroll
                 for (int c = 0; c < kKeys; ++c) sv[c] = 0.f;
             }
-            l = l * alpha + sum;
+            l = l * alpha + (((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7])));
             if (j > 0 && __any_sync(0xffffffffu, grow)) {
                 // O holds P.V of tiles < j: wait for the last of them, then rescale
-                if (!(ok = mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, p.err))) break;
+                if (!(ok = mbar_wait(&pv_done[t][(j - 1) & 1], ((j - 1) >> 1) & 1, p.err))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int c0 = 0; c0 < D; c0 += 32) {
@@ -392,53 +463,46 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < 32; ++i) ov[i] *= alpha;
                     tmem_st32(lane_base + O_COL + c0, ov);
                 }
-                tmem_wait_st();
             }
-            // the P buffer of tile j was read by P.V of tile j - 2
-            if (j >= 2) {
-                if (!(ok = mbar_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1, p.err))) break;
-            }
-            uint8_t* ph = sPh + (j & 1) * P_BYTES;
-            uint8_t* pl = sPl + (j & 1) * P_BYTES;
-            // P row: 64 keys = one 128-byte row per part, 8 chunks of 8 keys
+            // P_j over S_j's columns: bf16 high parts of the 64 weights in the
+            // first 32 columns (two per column, lower key in the low half),
+            // bf16 residuals in the last 32
+            uint32_t hi[kKeys / 2], lo[kKeys / 2];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint32_t hi[4], lo[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float a = sv[8 * c + 2 * e], bb = sv[8 * c + 2 * e + 1];
-                    hi[e] = pack_bf16x2(a, bb);
-                    lo[e] = pack_bf16x2(a - bf16_lo_to_f32(hi[e]), bb - bf16_hi_to_f32(hi[e]));
-                }
-                const int pc = (c ^ (row & 7)) << 4;
-                *reinterpret_cast<uint4*>(ph + row * 128 + pc) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4*>(pl + row * 128 + pc) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            for (int c = 0; c < kKeys / 2; ++c) {
+                const float a = sv[2 * c], bb = sv[2 * c + 1];
+                hi[c] = pack_bf16x2(a, bb);
+                lo[c] = pack_bf16x2(a - bf16_lo_to_f32(hi[c]), bb - bf16_hi_to_f32(hi[c]));
             }
+            tmem_st32u(lane_base + s * S_COLS, hi);
+            tmem_st32u(lane_base + s * S_COLS + S_COLS / 2, lo);
             // keys past the sequence end carry weight 0, but 0 * NaN is NaN in
-            // the MMA: zero those V rows of the last tile
-            if (j == nt - 1 && n_kv < nt * kKeys) {
+            // the MMA: zero those V rows of the CTA's last tile (both
+            // warpgroups that use it do, each before it signals its P)
+            if (j == nt_cta - 1 && n_kv < nt_cta * kKeys) {
                 uint8_t* vs = sV + (j % kStages) * KV_BYTES;
                 const int first = n_kv - j * kKeys;
                 const int nch = (kKeys - first) * SLABS * 8;
-                for (int c = threadIdx.x - 64; c < nch; c += 128) {
+                for (int c = row; c < nch; c += 128) {
                     const int r = first + c / (SLABS * 8);
                     const int rem = c % (SLABS * 8);
                     *reinterpret_cast<uint4*>(vs + (rem >> 3) * KV_SLAB + r * 128 + (rem & 7) * 16) =
                         make_uint4(0u, 0u, 0u, 0u);
                 }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             }
-            // every softmax thread signals its own P row (and V zeroing) to the
-            // MMA thread; no named barrier, so a timed-out warp cannot strand
-            // the others
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tmem_wait_st();
+            // every softmax thread signals its own P row to the MMA thread; no
+            // named barrier, so a timed-out warp cannot strand the others
             tc_fence_before();
-            mbar_arrive(&p_full[j & 1]);
+            mbar_arrive(&p_full[t][s]);
         }
         // epilogue: O / l for this row
-        if (ok && (ok = mbar_wait(&pv_done[(nt - 1) & 1], ((nt - 1) >> 1) & 1, p.err))) {
+        if (ok && ntt > 0 && (ok = mbar_wait(&pv_done[t][(ntt - 1) & 1], ((ntt - 1) >> 1) & 1, p.err))) {
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            const int64_t orow = ((int64_t)(q0 + t0 + tq) * p.num_q_heads + (int64_t)kvh * G + (row % G)) * D;
+            const int64_t orow =
+                ((int64_t)(q0 + my_t0 + tq) * p.num_q_heads + (int64_t)kvh * G + (row % G)) * D;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
                 float ov[32];
@@ -446,15 +510,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_wait_ld();
                 if (valid) {
                     if (p.out_bf16) {
-                        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + orow + c0;
+                        uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + orow + c0);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __float2bfloat16_rn(ov[i] * inv);
+                        for (int i = 0; i < 32; i += 8)
+                            o[i / 8] = make_uint4(pack_bf16x2(ov[i] * inv, ov[i + 1] * inv),
+                                                  pack_bf16x2(ov[i + 2] * inv, ov[i + 3] * inv),
+                                                  pack_bf16x2(ov[i + 4] * inv, ov[i + 5] * inv),
+                                                  pack_bf16x2(ov[i + 6] * inv, ov[i + 7] * inv));
                     } else {
-                        float* o = static_cast<float*>(p.out) + orow + c0;
+                        float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow + c0);
 #pragma unroll
                         for (int i = 0; i < 32; i += 4)
-                            *reinterpret_cast<float4*>(o + i) =
-                                make_float4(ov[i] * inv, ov[i + 1] * inv, ov[i + 2] * inv, ov[i + 3] * inv);
+                            o[i / 4] = make_float4(ov[i] * inv, ov[i + 1] * inv, ov[i + 2] * inv, ov[i + 3] * inv);
                     }
                 }
             }
@@ -465,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTiles * TILE_COLS));
     }
 }
 
@@ -499,7 +566,10 @@ int encode(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
 template <int D>
 size_t prefill_smem_bytes() {
     constexpr int SLABS = D / 64;
-    return 1024 + SLABS * kRows * 128 + 2 * kStages * SLABS * kKeys * 128 + 4 * kRows * 128;
+    // at least 120 KB so that one CTA, holding all 512 TMEM columns, is
+    // alone on its SM (the head_dim 64 tiles alone would let two fit)
+    const size_t need = 1024 + kTiles * SLABS * kRows * 128 + 2 * kStages * SLABS * kKeys * 128;
+    return need < 120 * 1024 ? 120 * 1024 : need;
 }
 
 template <int D>
@@ -580,7 +650,8 @@ extern "C" int pa_paged_attention_prefill(const void* q, const void* k_pool, con
     p.block_size = block_size;
     p.out_bf16 = out_dtype == PA_BF16;
     p.scale_log2 = scale * kLog2e;
-    dim3 grid((unsigned)((max_query_len + TQ - 1) / TQ), (unsigned)num_kv_heads, (unsigned)batch);
+    const int q_tiles = (max_query_len + TQ - 1) / TQ;
+    dim3 grid((unsigned)((q_tiles + kTiles - 1) / kTiles), (unsigned)num_kv_heads, (unsigned)batch);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return head_dim == 128 ? launch_prefill<128>(p, tq, tk, tv, grid, st) : launch_prefill<64>(p, tq, tk, tv, grid, st);
 }

@@ -91,6 +91,55 @@ def test_reshape_and_cache_flags_slot_outside_pool(pa):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("bs", [8, 16, 32])
+def test_fused_decode_write_matches_two_step_oracle(pa, dtype, D, bs):
+    """pa_reshape_and_cache_decode = decode slot mapping + cache write, bit for bit,
+    with a length-0 sequence in the batch (no write, slot -1)."""
+    g = torch.Generator().manual_seed(3 * D + bs)
+    B, MBS, Hkv = 45, 7, 4
+    NB = B * MBS + 5
+    bt = torch.randperm(NB, generator=g)[: B * MBS].reshape(B, MBS).to(torch.int32)
+    lens = torch.randint(1, MBS * bs + 1, (B,), generator=g, dtype=torch.int32)
+    lens[3] = 0
+    lens[4] = MBS * bs  # last slot of the last block
+    k_pool = torch.randn(NB, Hkv, bs, D, generator=g).to(DT[dtype])
+    v_pool = torch.randn(NB, Hkv, bs, D, generator=g).to(DT[dtype])
+    key = torch.randn(B, Hkv, D, generator=g).to(DT[dtype])
+    val = torch.randn(B, Hkv, D, generator=g).to(DT[dtype])
+    want_slots = oracle.slot_mapping(np_of(bt), np.arange(B, dtype=np.int32), np_of(lens) - 1, bs)
+    want_slots[3] = -1
+    kp, vp = np_of(k_pool).copy(), np_of(v_pool).copy()
+    oracle.reshape_and_cache(np_of(key), np_of(val), kp, vp, want_slots)
+    gk, gv = k_pool.cuda(), v_pool.cuda()
+    got = torch.full((B,), 7, dtype=torch.int64, device="cuda")
+    pa.pa_reshape_and_cache_decode(key.cuda(), val.cuda(), gk, gv, bt.cuda(), lens.cuda(), got)
+    assert np.array_equal(np_of(got), want_slots)
+    assert np_of(gk).tobytes() == kp.tobytes()
+    assert np_of(gv).tobytes() == vp.tobytes()
+    # without the slot output the pools come out the same
+    gk2, gv2 = k_pool.cuda(), v_pool.cuda()
+    pa.pa_reshape_and_cache_decode(key.cuda(), val.cuda(), gk2, gv2, bt.cuda(), lens.cuda())
+    assert torch.equal(gk2, gk) and torch.equal(gv2, gv)
+    assert pa.pa_read_error_flag() == 0
+
+
+def test_fused_decode_write_flags_bad_entries(pa):
+    k_pool = torch.zeros(2, 1, 8, 64, device="cuda")
+    v_pool = torch.zeros_like(k_pool)
+    key = torch.ones(4, 1, 64, device="cuda")
+    bt = torch.tensor([[1, -1], [1, 0], [5, 0], [0, 1]], dtype=torch.int32, device="cuda")
+    # seq 0: unmapped block; seq 1: slot 0*8+0; seq 2: block 5 outside a 2-block pool; seq 3: length 0
+    lens = torch.tensor([9, 9, 3, 0], dtype=torch.int32, device="cuda")
+    got = torch.empty(4, dtype=torch.int64, device="cuda")
+    pa.pa_reshape_and_cache_decode(key, 2 * key, k_pool, v_pool, bt, lens, got)
+    assert got.tolist() == [-1, 0, 5 * 8 + 2, -1]
+    assert pa.pa_read_error_flag() == 5
+    assert k_pool[0, 0, 0].eq(1).all() and k_pool.sum().item() == 64
+    assert v_pool[0, 0, 0].eq(2).all() and v_pool.sum().item() == 128
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("bs", [8, 16, 32])
 def test_copy_blocks_bit_exact(pa, dtype, bs):
     g = torch.Generator().manual_seed(bs)

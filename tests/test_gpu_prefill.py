@@ -75,6 +75,18 @@ def test_prefill_single_token_equals_decode(pa):
     assert_matches_oracle(dec, ref, True, "decode vs prefill oracle")
 
 
+@pytest.mark.parametrize("scale", [-0.0883883461356163, 0.0])
+def test_prefill_nonpositive_scale(pa, scale):
+    """A negative or zero scale takes the kernel's scale-first path (a positive
+    one folds the scale into the exponent); scale 0 is the plain average of
+    the visible V rows."""
+    case = custom_case([90, 300], 8, 2, 128, 16, torch.bfloat16, seed=11)
+    case.scale = float(np.float32(scale))
+    out, ref = _run(pa, case, [90, 170])
+    assert_matches_oracle(out, ref, True, f"prefill scale {scale}")
+    assert pa.pa_read_error_flag() == 0
+
+
 def test_prefill_never_reads_past_the_sequence(pa):
     lengths = [40, 129, 17]
     case = custom_case(lengths, 8, 2, 128, 16, torch.bfloat16, seed=7, extra_blocks=6)
