@@ -25,7 +25,9 @@ value  = K/V bytes attention reads (tokens < length, K and V) / step time,
          data-path collective).
 e2e    = the same metric through the public API with the step's inputs in
          pinned host memory: H2D of q, new K/V, block tables and lengths, the
-         step, and D2H of the output, all inside the timed events.
+         step (direct calls), and D2H of the output, all inside the timed
+         events; a device spin before each step lets the host enqueue it
+         ahead, so host issue latency stays out.
 roofline = the decode call alone (pass 1 + merge) against the measured HBM
          copy bandwidth.
 
@@ -53,6 +55,7 @@ if ROOT not in sys.path:
 METRIC = "Paged decode attn: achieved HBM GB/s vs peak; decode tokens/s per batch"
 FALLBACK_HBM_GBS = 6650.0
 FLUSH_BYTES = 256 << 20
+SPIN_CYCLES = 2_000_000  # ~1 ms at 1.9 GHz
 
 DESCRIPTIONS = {
     "tiny": "tiny: batch 4, lengths 1,7,16,33 (+1 appended), 4/4 heads, head_dim 64, block_size 16, fp32",
@@ -451,6 +454,10 @@ def run_ours(args):
     e2e_ev = []
     for i in range(args.warmup + args.steps):
         flush_l2()
+        # a 1 ms spin on the device before the start event: the host enqueues
+        # the whole step (copies, API calls, read-back) while it runs, so the
+        # events time the step's device work, not Python's issue rate
+        torch.cuda._sleep(SPIN_CYCLES)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for dst, src in ((d_q, h_q), (d_kn, h_kn), (d_vn, h_vn), (d_bt, h_bt), (d_lens, h_lens)):
@@ -503,7 +510,9 @@ def run_ours(args):
         "paging_overhead": {"paged_ms_median": paged_med, "contiguous_ms_median": contig_med,
                             "overhead": paged_med / contig_med - 1.0, "contiguous_ms_mean_max_ranks": ms_contig},
         "e2e": {"value": world * kv_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
+                "timing": "device time from before the H2D copies to after the D2H read-back, direct API calls "
+                          "(no graph); a device spin ahead of each step keeps host issue latency out"},
         "gpu_launches": (cache_launches + decode_launches) * args.steps,
         "gpu_launches_decode_roofline_loop": decode_launches * args.steps,
         "timing": ("K replays of the step's CUDA graph (value), then K replays of the decode call's graph "

@@ -107,7 +107,9 @@ def test_fused_decode_write_matches_two_step_oracle(pa, dtype, D, bs):
     v_pool = torch.randn(NB, Hkv, bs, D, generator=g).to(DT[dtype])
     key = torch.randn(B, Hkv, D, generator=g).to(DT[dtype])
     val = torch.randn(B, Hkv, D, generator=g).to(DT[dtype])
-    want_slots = oracle.slot_mapping(np_of(bt), np.arange(B, dtype=np.int32), np_of(lens) - 1, bs)
+    pos = np_of(lens) - 1
+    pos[3] = 0  # the empty sequence writes nothing: its slot is -1 below
+    want_slots = oracle.slot_mapping(np_of(bt), np.arange(B, dtype=np.int32), pos, bs)
     want_slots[3] = -1
     kp, vp = np_of(k_pool).copy(), np_of(v_pool).copy()
     oracle.reshape_and_cache(np_of(key), np_of(val), kp, vp, want_slots)
