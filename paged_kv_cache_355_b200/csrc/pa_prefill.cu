@@ -14,14 +14,15 @@
 //    and streams K/V tiles of 64 tokens through a 4-stage ring (tiled TMA
 //    boxes of block_size rows from the pool, 128-byte swizzle), each tile
 //    used by both query tiles;
-//  * warp 1 allocates all 512 tensor-memory columns and issues the MMAs from
-//    one thread, per query tile t:
+//  * warp 1 allocates all 512 tensor-memory columns; warps 1 and 2 each issue
+//    one query tile's MMAs from one thread, so neither tile's chain waits on
+//    the other's softmax:
 //        S_tj = Q_t . K_j^T       (M = 128 rows, N = 64 keys, K = D)
 //        O_t += P_tj . V_j        (M = 128 rows, N = D, K = 64 keys)
 //    S is double-buffered in tensor memory, so S_t,j+1 runs while the
 //    softmax works on S_tj, and P_tj is written back over S_tj's columns and
 //    read by the P.V MMA straight from tensor memory;
-//  * warps 2..5 and 6..9 are the two tiles' softmax warpgroups (one query
+//  * warps 3..6 and 7..10 are the two tiles' softmax warpgroups (one query
 //    row per thread: TMEM lane = row).  Each loads S_tj, applies the causal
 //    mask and scale, keeps its row's running max and sum in registers,
 //    rescales O in tensor memory only when the max has grown by more than
@@ -53,7 +54,7 @@ namespace {
 constexpr int kRows = 128;    // query rows per tile (TMEM lanes)
 constexpr int kTiles = 2;     // query tiles per CTA
 constexpr int kKeys = 64;     // keys per tile
-constexpr int kThreads = 64 + kTiles * 128;  // producer, MMA, one softmax warpgroup per query tile
+constexpr int kThreads = 96 + kTiles * 128;  // producer, two MMA issuers, one softmax warpgroup per query tile
 static_assert(kTiles == 2, "the softmax warpgroups select their tile's values between two");
 constexpr int kStages = 4;     // K/V ring depth
 constexpr float kLog2e = 1.4426950408889634f;
@@ -248,12 +249,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&q_full, 1);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
+            mbar_init(&kv_empty[s], kTiles);
         }
         for (int t = 0; t < kTiles; ++t)
             for (int s = 0; s < 2; ++s) {
                 mbar_init(&s_full[t][s], 1);
-                mbar_init(&p_full[t][s], 128);
+                mbar_init(&p_full[t][s], 4);
                 mbar_init(&pv_done[t][s], 1);
             }
         fence_barrier_init();
@@ -323,64 +324,64 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-    } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
-        // Step j issues S_j = Q_t . K_j^T for both tiles, then O_t += P_{j-1} . V_{j-1}
-        // once each warpgroup has written P_{j-1}.  tcgen05.mma ops from one
-        // thread run in issue order, so S_j may overwrite the buffer that
-        // held P_{j-2}: its P.V was issued one step earlier.
+    } else if (warp <= kTiles) {
+        // ---------------- MMA issuers: warp 1 + t for query tile t ----------------
+        // Each issuer runs its tile's chain on its own: S_j = Q_t . K_j^T, then
+        // O_t += P_{j-1} . V_{j-1} once the softmax has written P_{j-1}.  Its
+        // tcgen05.mma ops run in issue order, so S_j may overwrite the buffer
+        // that held P_{j-2}.  A K/V stage is released when both issuers have
+        // arrived; a tile that needs fewer key tiles arrives for the rest once
+        // they are loaded (so the arrival lands in the right phase).
+        const int t = warp - 1;
         if (lane == 0) {
             constexpr uint32_t IDESC_S = umma_idesc(kRows, kKeys, false);
             constexpr uint32_t IDESC_O = umma_idesc(kRows, D, true);
-            bool ok = mbar_wait(&q_full, 0, p.err);
-            for (int j = 0; ok && j <= nt_cta; ++j) {
-                if (j < nt_cta) {
+            const int ntt = t ? nt[1] : nt[0];
+            const uint32_t q_base = smem_addr(sQ + t * Q_BYTES);
+            bool ok = ntt == 0 || mbar_wait(&q_full, 0, p.err);
+            for (int j = 0; ok && j <= ntt; ++j) {
+                if (j < ntt) {
                     const int ks = j % kStages;
                     if (!(ok = mbar_wait(&kv_full[ks], (j / kStages) & 1, p.err))) break;
                     tc_fence_after();
                     const uint32_t k_base = smem_addr(sK + ks * KV_BYTES);
+                    const uint32_t d_s = tmem + t * TILE_COLS + (j & 1) * S_COLS;
 #pragma unroll
-                    for (int t = 0; t < kTiles; ++t) {
-                        if (j >= nt[t]) continue;
-                        const uint32_t q_base = smem_addr(sQ + t * Q_BYTES);
-                        const uint32_t d_s = tmem + t * TILE_COLS + (j & 1) * S_COLS;
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t off = (kk & 3) * 32;
-                            const uint64_t da = umma_desc(q_base + (kk >> 2) * (kRows * 128) + off, 16, 1024);
-                            const uint64_t db = umma_desc(k_base + (kk >> 2) * KV_SLAB + off, 16, 1024);
-                            umma(d_s, da, db, IDESC_S, kk > 0 ? 1u : 0u);
-                        }
-                        umma_commit(&s_full[t][j & 1]);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk & 3) * 32;
+                        const uint64_t da = umma_desc(q_base + (kk >> 2) * (kRows * 128) + off, 16, 1024);
+                        const uint64_t db = umma_desc(k_base + (kk >> 2) * KV_SLAB + off, 16, 1024);
+                        umma(d_s, da, db, IDESC_S, kk > 0 ? 1u : 0u);
                     }
+                    umma_commit(&s_full[t][j & 1]);
                 }
                 if (j >= 1) {
                     const int jp = j - 1;
+                    if (!(ok = mbar_wait(&p_full[t][jp & 1], (jp >> 1) & 1, p.err))) break;
+                    tc_fence_after();
                     const uint32_t v_base = smem_addr(sV + (jp % kStages) * KV_BYTES);
+                    const uint32_t p_col = tmem + t * TILE_COLS + (jp & 1) * S_COLS;
 #pragma unroll
-                    for (int t = 0; t < kTiles; ++t) {
-                        if (jp >= nt[t]) continue;
-                        if (!(ok = mbar_wait(&p_full[t][jp & 1], (jp >> 1) & 1, p.err))) break;
-                        tc_fence_after();
-                        const uint32_t p_col = tmem + t * TILE_COLS + (jp & 1) * S_COLS;
-#pragma unroll
-                        for (int kk = 0; kk < kKeys / 16; ++kk) {
-                            const uint64_t db = umma_desc(v_base + kk * 2048, KV_SLAB, 1024);
-                            umma_tmem_a(tmem + t * TILE_COLS + O_COL, p_col + kk * 8, db, IDESC_O,
-                                        (jp > 0 || kk > 0) ? 1u : 0u);
-                            umma_tmem_a(tmem + t * TILE_COLS + O_COL, p_col + S_COLS / 2 + kk * 8, db, IDESC_O, 1u);
-                        }
-                        umma_commit(&pv_done[t][jp & 1]);
+                    for (int kk = 0; kk < kKeys / 16; ++kk) {
+                        const uint64_t db = umma_desc(v_base + kk * 2048, KV_SLAB, 1024);
+                        umma_tmem_a(tmem + t * TILE_COLS + O_COL, p_col + kk * 8, db, IDESC_O,
+                                    (jp > 0 || kk > 0) ? 1u : 0u);
+                        umma_tmem_a(tmem + t * TILE_COLS + O_COL, p_col + S_COLS / 2 + kk * 8, db, IDESC_O, 1u);
                     }
-                    if (!ok) break;
+                    umma_commit(&pv_done[t][jp & 1]);
                     umma_commit(&kv_empty[jp % kStages]);
                 }
+            }
+            for (int j = ntt; ok && j < nt_cta; ++j) {
+                const int ks = j % kStages;
+                if (!(ok = mbar_wait(&kv_full[ks], (j / kStages) & 1, p.err))) break;
+                mbar_arrive(&kv_empty[ks]);
             }
             if (!ok) s_abort = 1;
         }
     } else {
         // ---------------- softmax / epilogue: one query row per thread ----------------
-        const int t = (warp - 2) >> 2;               // query tile of this warpgroup
+        const int t = (warp - 1 - kTiles) >> 2;      // query tile of this warpgroup
         const int quarter = warp & 3;                // TMEM lane quarter this warp may access
         const int row = quarter * 32 + lane;         // query row of the tile = TMEM lane
         const int tq = row / G;                      // query token within the tile
@@ -492,10 +493,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             }
             tmem_wait_st();
-            // every softmax thread signals its own P row to the MMA thread; no
-            // named barrier, so a timed-out warp cannot strand the others
+            // each warp signals its 32 P rows (and its share of the V zeroing)
+            // to the MMA thread once all its lanes are done
             tc_fence_before();
-            mbar_arrive(&p_full[t][s]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[t][s]);
         }
         // epilogue: O / l for this row
         if (ok && ntt > 0 && (ok = mbar_wait(&pv_done[t][(ntt - 1) & 1], ((ntt - 1) >> 1) & 1, p.err))) {
