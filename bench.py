@@ -102,16 +102,27 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def code_sha256(path: str) -> str:
+    """sha256 of a source file's code: // comments and blank lines removed,
+    so that a comment edit does not void a measurement of the same kernel."""
+    lines = []
+    for line in open(path, encoding="utf-8"):
+        code = line.split("//", 1)[0].rstrip()
+        if code:
+            lines.append(code)
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()
+
+
 def dram_traffic(workload: str):
     """Per-launch DRAM bytes of the decode kernel from the committed ncu
-    summary, if it was taken on the current kernel source; else None."""
+    summary, if it was taken on the current kernel code; else None."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
     src = os.path.join(ROOT, "paged_kv_cache_355_b200", "csrc", "pa_decode.cu")
     try:
         rec = json.load(open(path))
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        sha = code_sha256(src)
         entry = rec.get(workload)
-        if entry and entry.get("kernel_source_sha256") == sha:
+        if entry and entry.get("kernel_code_sha256") == sha:
             return int(entry["dram_bytes_per_launch"])
     except Exception:
         pass

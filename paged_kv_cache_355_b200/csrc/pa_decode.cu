@@ -12,28 +12,39 @@
 //    with a log-sum-exp rescale.  Split boundaries depend only on logical
 //    token positions, so the result is independent of where the blocks sit
 //    in the pool and bit-identical from run to run (no atomics).
-//  * Warp 0 is the producer: its lane 0 reads the CTA's slice of the block
-//    table (staged once into shared memory) and streams K and V tiles with
-//    bulk copies (cp.async.bulk, the TMA engine) into a ring of `stages`
-//    shared-memory stages, each holding 32 tokens of K and 32 of V.  A stage
-//    gathers 32 / block_size physical blocks into one contiguous 32-token
-//    tile, so the math never depends on block_size.  Full/empty mbarriers
-//    hand stages to the consumers and back.
+//  * Sequences are taken longest first: every CTA's prologue ranks the
+//    batch's lengths with a counting sort (64 length buckets) and maps its
+//    blockIdx.z to the sequence of that rank, so the grid's tail holds the
+//    short sequences.
+//  * Warp 0 is the producer: the CTA's slice of the block table is staged
+//    once into shared memory, and lane i of warp 0 copies tile i of each
+//    32-token stage (one block, or block_size contiguous tokens) with the
+//    TMA engine into a ring of `stages` shared-memory stages (K and V of 32
+//    tokens each), so the copies of one stage are issued in parallel.  bf16
+//    tiles use tiled copies (cp.async.bulk.tensor, 128-byte swizzle), fp32
+//    tiles linear ones (cp.async.bulk).  A stage gathers 32 / block_size
+//    physical blocks into one contiguous 32-token tile, so the math never
+//    depends on block_size.  Full/empty mbarriers hand stages to the
+//    consumers and back; every wait is bounded.
 //  * Warps 1..2 are consumers.  Stage j goes to consumer warp j % 2, which
 //    keeps its own fp32 online-softmax state (running max m, running sum l,
 //    output accumulator o) for all G = Hq / Hkv query heads of the kv head:
 //    every K and V element loaded from shared memory is used by all G heads.
-//    Inside a warp, a group of TPT lanes owns one token row (16 bytes per
-//    lane), so K/V shared-memory reads are conflict-free row segments; the
-//    q.k partial sums are reduced across the TPT lanes with shuffles, and the
-//    32 / TPT groups of a warp are independent softmax states.
-//  * At the end the groups and the warps are merged (shuffles, then shared
-//    memory), and the CTA writes either the final row (one split) or its
-//    normalised partial row plus (m, l) for the merge kernel.
-//  * Scores are kept in the log2 domain: q is pre-multiplied by
-//    scale * log2(e) and exp2f is used throughout.
+//    bf16 runs the contractions on the tensor cores (decode_pass1_mma_kernel,
+//    described there); fp32 on the CUDA cores (decode_pass1_kernel): a group
+//    of TPT lanes owns one token row (16 bytes per lane), so shared-memory
+//    reads are conflict-free row segments, and the q.k partial sums are
+//    reduced across the TPT lanes with shuffles.
+//  * At the end the warps' states are merged (shuffles, then shared memory),
+//    and the CTA writes either the final row (one split) or its normalised
+//    partial row plus (m, l) for the merge kernel.
+//  * Scores are kept in the log2 domain (scale * log2(e) folded in) and
+//    exponentials are exp2.
 //  * Tokens past the sequence end are masked to -inf and their V rows are
 //    never multiplied (stale shared memory may hold anything, NaN included).
+//  * Pass 1 and the merge are launched with programmatic stream
+//    serialisation and wait (griddepcontrol.wait) before touching global
+//    memory, so they can be scheduled while the previous kernel drains.
 //
 // The contiguous-cache variant is the same kernel: only the producer's source
 // address differs (one bulk copy per 32-token stage instead of one per block).
