@@ -333,7 +333,7 @@ def run_reference(args):
 def run_ours(args):
     world, rank, local = dist_setup(args.gpus)
     import paged_kv_cache_355_b200 as pa
-    from paged_kv_cache_355_b200.workloads import SEEDS, make_case
+    from paged_kv_cache_355_b200.workloads import SEEDS, WORKLOADS, make_case
 
     dev = torch.device("cuda", local)
     case = make_case(args.workload, device=dev, seed=SEEDS[args.workload] + 101 * rank, batch=args.batch)
@@ -517,7 +517,8 @@ def run_ours(args):
     peak, peak_kind = measured_hbm_peak()
     achieved = kv_bytes / (ms_dec * 1e-3) / 1e9
     value = world * kv_bytes / (ms_step * 1e-3) / 1e9
-    traffic = dram_traffic(args.workload)
+    # the committed ncu record covers the workloads at their own batch only
+    traffic = dram_traffic(args.workload) if args.batch in (None, WORKLOADS[args.workload].batch) else None
     clk = clocks.summary()
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
