@@ -437,6 +437,34 @@ def run_ours(args):
     ms_dec = max_over_ranks(sum(dec_ms) / len(dec_ms), world)
     assert pa.pa_read_error_flag() == 0, "device error during the timed steps"
 
+    # ---- the step's cache kernels alone (slot mapping, cache write, copy-on-write
+    # copies), captured and timed the same way; their algorithmic bytes: each new
+    # token's K and V rows read and written, each copied block's K and V read and
+    # written, and the slots
+    elt = case.k_pool.element_size()
+    n_new = case.new_seq_ids.numel()
+    cache_bytes = (n_new * Hkv * D * elt * 2 * 2 + pairs.shape[0] * Hkv * bs * D * elt * 2 * 2
+                   + n_new * 8 * (1 if plain_decode else 2))
+    run_cache_only = cache_part
+    if graphs is not None:
+        g_cache = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_cache):
+            cache_part()
+        run_cache_only = g_cache.replay
+    cache_ev = []
+    for i in range(args.warmup + min(args.steps, 200)):
+        flush_l2()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run_cache_only()
+        e1.record(stream)
+        if i >= args.warmup:
+            cache_ev.append((e0, e1))
+    torch.cuda.synchronize()
+    ms_cache = max_over_ranks(sum(a.elapsed_time(b_) for a, b_ in cache_ev) / len(cache_ev), world)
+    if graphs is not None:
+        del g_cache
+
     # ---- contiguous-cache variant of the same kernel on the same lengths (paging overhead),
     # timed the same way (graph replay)
     L_pad = -(-max_len // 32) * 32
@@ -541,6 +569,12 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "kernel": "pa_paged_attention_decode (pass 1 + split merge)",
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)"},
+        "cache_part": {"kernels": (["pa_copy_blocks"] if pairs.numel() else [])
+                       + (["pa_reshape_and_cache_decode"] if plain_decode
+                          else ["pa_slot_mapping", "pa_reshape_and_cache"]),
+                       "ms": ms_cache, "bytes": cache_bytes, "gbs": cache_bytes / (ms_cache * 1e-3) / 1e9,
+                       "frac": cache_bytes / (ms_cache * 1e-3) / 1e9 / peak,
+                       "note": "timed alone as one graph; small writes are launch-latency bound"},
         "paging_overhead": {"paged_ms_median": paged_med, "contiguous_ms_median": contig_med,
                             "overhead": paged_med / contig_med - 1.0, "contiguous_ms_mean_max_ranks": ms_contig},
         "e2e": {"value": world * kv_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,

@@ -45,7 +45,7 @@ def test_decode_bench_line_has_the_contract_fields(bench, capsys, workload, batc
     d = _line(capsys)
     for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
                 "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks",
-                "cpu_baseline", "paging_overhead", "tokens_per_s"):
+                "cpu_baseline", "paging_overhead", "tokens_per_s", "cache_part"):
         assert key in d, key
     assert d["value"] > 0 and d["ms_per_step"] > 0 and d["n_gpus"] == 1 and d["steps"] == 3
     assert d["unit"] == "GB/s" and d["higher_is_better"] is True and d["scaling"] == "weak"
@@ -58,6 +58,7 @@ def test_decode_bench_line_has_the_contract_fields(bench, capsys, workload, batc
     e = d["e2e"]
     assert e["value"] > 0 and e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
     assert d["gpu_launches"] >= 2 * d["steps"]
+    assert d["cache_part"]["ms"] > 0 and d["cache_part"]["bytes"] > 0
     assert {"sm_mhz", "sm_max_mhz", "reasons"} <= set(d["clocks"])
     if workload == "cow":
         assert d["unique_kv"]["bytes_per_step"] < d["config"]["kv_bytes_per_step"]
