@@ -838,62 +838,108 @@ __global__ void __launch_bounds__(kDecodeThreads)
 }
 
 // Second pass: out = sum_s w_s o_s / sum_s w_s with w_s = l_s * 2^(m_s - max m),
-// for sequences that were cut into more than one split.  One warp per
-// (sequence, query head) row, eight rows per CTA: lane s loads split s's
-// (m, l), the max and the sum are warp shuffles, and lane i accumulates
-// output elements [i * D / 32, (i + 1) * D / 32) over the splits in order
-// (deterministic, no shared memory, no block barrier).
+// for sequences that were cut into more than one split.  Four warps share a
+// (sequence, query head) row, two rows per CTA: warp k of a row takes splits
+// k, k + 4, ..., eight at a time, issuing all their (m, l) and partial-row
+// loads before it needs any of them (lane i holds output elements
+// [i * D / 32, (i + 1) * D / 32)), and keeps its own running max, weight sum
+// and accumulator; the four warps' states are then combined through shared
+// memory by the row's first warp.  The order of every sum is fixed, so the
+// result is deterministic.
 constexpr int kMergeWarps = 8;
+constexpr int kMergeWarpsPerRow = 4;
+constexpr int kMergeChunk = 8;  // splits per warp in flight
 
 template <int D>
 __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(const DecodeParams p, int64_t rows) {
     constexpr int VPL = D / 32;  // output elements per lane
+    constexpr int STRIDE = kMergeWarpsPerRow * kMergeChunk;
+    __shared__ float s_acc[kMergeWarps][D];
+    __shared__ float s_m[kMergeWarps], s_w[kMergeWarps];
     const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int wk = warp % kMergeWarpsPerRow;
     griddep_wait();  // the partial rows come from pass 1
-    const int64_t row = (int64_t)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);  // b * Hq + h
-    if (row >= rows) return;
-    const int b = (int)(row / p.num_q_heads);
-    const int L = clamp_len(p, b, false);
-    const int ns = L > 0 ? (L + p.partition - 1) / p.partition : 1;
-    if (ns <= 1) return;
-    const float* ml = p.part_ml + row * p.max_splits * 2;
-    const float* po = p.part_o + row * p.max_splits * D + lane * VPL;
-
-    float M = -INFINITY;
-    for (int s = lane; s < ns; s += 32) M = fmaxf(M, ml[2 * s]);
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-
-    float acc[VPL];
+    const int64_t row = (int64_t)blockIdx.x * (kMergeWarps / kMergeWarpsPerRow) + warp / kMergeWarpsPerRow;
+    int ns = 0;
+    if (row < rows) {
+        const int L = clamp_len(p, (int)(row / p.num_q_heads), false);
+        ns = L > 0 ? (L + p.partition - 1) / p.partition : 1;
+    }
+    float m = -INFINITY, W = 0.f, acc[VPL];
 #pragma unroll
     for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
-    float W = 0.f;
-    for (int s0 = 0; s0 < ns; s0 += 32) {
-        const int s = s0 + lane;
-        const float w = s < ns ? ml[2 * s + 1] * exp2f(ml[2 * s] - M) : 0.f;
-        W += w;
-        const int n = min(32, ns - s0);
-#pragma unroll 8
-        for (int k = 0; k < n; ++k) {
-            const float wk = __shfl_sync(0xffffffffu, w, k);
-            const float* src = po + (int64_t)(s0 + k) * D;
-            if constexpr (VPL == 4) {
-                const float4 v = *reinterpret_cast<const float4*>(src);
-                acc[0] = fmaf(wk, v.x, acc[0]);
-                acc[1] = fmaf(wk, v.y, acc[1]);
-                acc[2] = fmaf(wk, v.z, acc[2]);
-                acc[3] = fmaf(wk, v.w, acc[3]);
-            } else {
-                const float2 v = *reinterpret_cast<const float2*>(src);
-                acc[0] = fmaf(wk, v.x, acc[0]);
-                acc[1] = fmaf(wk, v.y, acc[1]);
+    if (ns > 1) {
+        const float* ml = p.part_ml + row * p.max_splits * 2;
+        const float* po = p.part_o + row * p.max_splits * D + lane * VPL;
+        for (int s0 = wk; s0 < ns; s0 += STRIDE) {
+            float mv[kMergeChunk], lv[kMergeChunk], ov[kMergeChunk][VPL];
+#pragma unroll
+            for (int k = 0; k < kMergeChunk; ++k) {
+                const int sp = s0 + k * kMergeWarpsPerRow;
+                if (sp < ns) {
+                    mv[k] = ml[2 * sp];
+                    lv[k] = ml[2 * sp + 1];
+                    const float* src = po + (int64_t)sp * D;
+                    if constexpr (VPL == 4) {
+                        const float4 v = *reinterpret_cast<const float4*>(src);
+                        ov[k][0] = v.x;
+                        ov[k][1] = v.y;
+                        ov[k][2] = v.z;
+                        ov[k][3] = v.w;
+                    } else {
+                        const float2 v = *reinterpret_cast<const float2*>(src);
+                        ov[k][0] = v.x;
+                        ov[k][1] = v.y;
+                    }
+                } else {
+                    mv[k] = -INFINITY;
+                    lv[k] = 0.f;
+#pragma unroll
+                    for (int i = 0; i < VPL; ++i) ov[k][i] = 0.f;
+                }
             }
+            float cm = m;
+#pragma unroll
+            for (int k = 0; k < kMergeChunk; ++k) cm = fmaxf(cm, mv[k]);
+            const float alpha = m == -INFINITY ? 0.f : exp2f(m - cm);
+            W *= alpha;
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) acc[i] *= alpha;
+#pragma unroll
+            for (int k = 0; k < kMergeChunk; ++k) {
+                const float w = mv[k] == -INFINITY ? 0.f : lv[k] * exp2f(mv[k] - cm);
+                W += w;
+#pragma unroll
+                for (int i = 0; i < VPL; ++i) acc[i] = fmaf(w, ov[k][i], acc[i]);
+            }
+            m = cm;
         }
     }
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
+    for (int i = 0; i < VPL; ++i) s_acc[warp][lane * VPL + i] = acc[i];
+    if (lane == 0) {
+        s_m[warp] = m;
+        s_w[warp] = W;
+    }
+    __syncthreads();
+    if (wk != 0 || ns <= 1) return;
+    float M = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) store_out(p, row * D + lane * VPL + i, W > 0.f ? acc[i] / W : 0.f);
+    for (int k = 0; k < kMergeWarpsPerRow; ++k) M = fmaxf(M, s_m[warp + k]);
+    float scale[kMergeWarpsPerRow], Wt = 0.f;
+#pragma unroll
+    for (int k = 0; k < kMergeWarpsPerRow; ++k) {
+        scale[k] = s_m[warp + k] == -INFINITY ? 0.f : exp2f(s_m[warp + k] - M);
+        Wt += s_w[warp + k] * scale[k];
+    }
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+        float v = 0.f;
+#pragma unroll
+        for (int k = 0; k < kMergeWarpsPerRow; ++k) v = fmaf(scale[k], s_acc[warp + k][lane * VPL + i], v);
+        store_out(p, row * D + lane * VPL + i, Wt > 0.f ? v / Wt : 0.f);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -1079,7 +1125,8 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
     if (rc) return rc;
     if (plan.max_splits > 1) {
         const int64_t rows = (int64_t)batch * p.num_q_heads;
-        const unsigned blocks = (unsigned)((rows + kMergeWarps - 1) / kMergeWarps);
+        constexpr int rows_per_cta = kMergeWarps / kMergeWarpsPerRow;
+        const unsigned blocks = (unsigned)((rows + rows_per_cta - 1) / rows_per_cta);
         rc = head_dim == 128 ? launch_pdl(decode_merge_kernel<128>, dim3(blocks), dim3(32 * kMergeWarps), 0, st, p, rows)
                              : launch_pdl(decode_merge_kernel<64>, dim3(blocks), dim3(32 * kMergeWarps), 0, st, p, rows);
     }
