@@ -300,6 +300,9 @@ def run_reference(args):
 
     import oracle
 
+    if args.op == "prefill":
+        run_reference_prefill(args, world)
+        return
     case = make_case(args.workload, device="cpu")
     w = case.workload
     # each step: the oracle over a bounded sample of the workload's sequences
@@ -325,6 +328,45 @@ def run_reference(args):
                              "sample": sample},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def run_reference_prefill(args, world):
+    """Reference arm of --op prefill: the oracle's causal multi-query attention
+    on the host cores; each step is the first 64 queries of the workload's
+    first sequence (all heads)."""
+    import numpy as np
+
+    import oracle
+    from paged_kv_cache_355_b200.workloads import custom_case
+
+    B, Hq, Hkv, D, bs, L, n = PREFILL_SHAPE
+    case = custom_case([L] * B, Hq, Hkv, D, bs, torch.bfloat16, seed=2001, device="cpu")
+    g = torch.Generator().manual_seed(2002)
+    q = torch.randn(n, Hq, D, generator=g).to(torch.bfloat16)
+    u16 = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    m = 64  # the sample: the first m of the n new queries, so context L - n + m
+    kp, vp, qm = u16(case.k_pool), u16(case.v_pool), u16(q[:m])
+    bt, lens = case.block_tables[:1].numpy(), np.array([L - n + m], dtype=np.int32)
+    qs = np.array([0, m], dtype=np.int32)
+    flops = 4.0 * D * Hq * (m * (L - n) + m * (m + 1) // 2)
+    for _ in range(args.warmup):
+        oracle.paged_prefill(qm, kp, vp, bt, lens, qs, case.scale, bs)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.paged_prefill(qm, kp, vp, bt, lens, qs, case.scale, bs)
+        times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    value = flops / sec / 1e12
+    sample = f"the first {m} of {n} new queries of 1 of {B} sequences, all {Hq} heads, fp64 oracle"
+    print(json.dumps({
+        "impl": "reference", "metric": PREFILL_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "dtype": "f64", "data": "synthetic", "config": {"workload": PREFILL_WORKLOAD},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+        flush=True)
 
 
 # ---------------------------------------------------------------------------
@@ -592,6 +634,8 @@ def run_ours(args):
     print(json.dumps(line), flush=True)
 
 
+PREFILL_SHAPE = (8, 32, 8, 128, 16, 4096, 2048)  # batch, Hq, Hkv, head_dim, block_size, context, new tokens
+PREFILL_METRIC = "Paged prefill attn (causal, multi-query): achieved TFLOP/s vs bf16 peak"
 PREFILL_WORKLOAD = ("chunked prefill: batch 8, 32 q / 8 kv heads, head_dim 128, block_size 16, bf16, "
                     "context 4096 of which the last 2048 tokens are the new chunk, blocks scattered")
 
@@ -604,7 +648,7 @@ def run_prefill(args):
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    B, Hq, Hkv, D, bs, L, n = 8, 32, 8, 128, 16, 4096, 2048
+    B, Hq, Hkv, D, bs, L, n = PREFILL_SHAPE
     case = custom_case([L] * B, Hq, Hkv, D, bs, torch.bfloat16, seed=2001, device=dev)
     qs = torch.arange(0, (B + 1) * n, n, dtype=torch.int32, device=dev)
     g = torch.Generator(device=dev).manual_seed(2002)
@@ -614,6 +658,7 @@ def run_prefill(args):
     pairs = sum(n * (L - n) + n * (n + 1) // 2 for _ in range(B))  # visible (query, key) pairs per head
     flops = 4.0 * D * Hq * pairs
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    clean = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     run = lambda: pa.pa_paged_attention_prefill(q, case.k_pool, case.v_pool, bt, lens, qs, n, case.scale, out)
     for _ in range(args.warmup):
         run()
@@ -621,7 +666,8 @@ def run_prefill(args):
     torch.cuda.synchronize()
     with ClockSampler(0) as clocks:
         for _ in range(args.steps):
-            flush.zero_()
+            flush.zero_()  # L2 flush outside the events: write, then read another buffer
+            clean.sum()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
             run()
@@ -634,8 +680,9 @@ def run_prefill(args):
         os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
     peak = float(peaks.get("bf16_tflops", 1590.0))
     tflops = flops / (ms * 1e-3) / 1e12
+    cpu = None if args.no_cpu_baseline else time_oracle_prefill(case, q, n, L, bs)
     print(json.dumps({
-        "metric": "Paged prefill attn (causal, multi-query): achieved TFLOP/s vs bf16 peak", "value": tflops,
+        "metric": PREFILL_METRIC, "value": tflops,
         "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "dtype": "bf16", "data": "synthetic", "config": {"workload": PREFILL_WORKLOAD},
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
@@ -644,7 +691,33 @@ def run_prefill(args):
                      else "fallback"},
         "note": "useful FLOPs only; the kernel multiplies P by V twice (bf16 high part and residual), "
                 "so the tensor pipe executes 1.5x these FLOPs",
-        "clocks": clocks.summary()}), flush=True)
+        "clocks": clocks.summary(), "cpu_baseline": cpu}), flush=True)
+
+
+def time_oracle_prefill(case, q, n, L, bs, min_seconds=10.0, max_reps=100):
+    """The oracle's causal multi-query attention for the first sequence of the
+    prefill workload (all its n queries and heads), on the host cores,
+    repeated until about min_seconds of CPU work have run."""
+    import numpy as np
+
+    import oracle
+
+    u16 = lambda t: t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    kp, vp, q0 = u16(case.k_pool), u16(case.v_pool), u16(q[:n])
+    bt, lens = case.block_tables[:1].numpy(), case.lengths[:1].numpy()
+    qs = np.array([0, n], dtype=np.int32)
+    Hq, D = q.shape[1], q.shape[2]
+    flops = 4.0 * D * Hq * (n * (L - n) + n * (n + 1) // 2)
+    reps, t_total = 0, 0.0
+    while reps < max_reps and (reps == 0 or t_total < min_seconds):
+        t0 = time.perf_counter()
+        oracle.paged_prefill(q0, kp, vp, bt, lens, qs, case.scale, bs)
+        t_total += time.perf_counter() - t0
+        reps += 1
+    sec = t_total / reps
+    return {"value": flops / sec / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"1 of 8 sequences of the same workload (its {n} new queries, all {Hq} heads), "
+                      f"{reps} repetition(s), {sec:.2f} s each, {t_total:.1f} s in all", "seconds_per_step": sec}
 
 
 def main():

@@ -72,3 +72,4 @@ def test_prefill_bench_line(bench, capsys):
     assert d["unit"] == "TFLOP/s" and d["value"] > 0
     r = d["roofline"]
     assert r["bound"] == "tensor" and abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-9
+    assert d["cpu_baseline"] is None  # skipped with --no-cpu-baseline
