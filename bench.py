@@ -24,8 +24,9 @@ value  = K/V bytes attention reads (tokens < length, K and V) / step time,
          summed over ranks (each rank runs its own batch: weak scaling, no
          data-path collective).
 e2e    = the same metric through the public API with the step's inputs in
-         pinned host memory: H2D of q, new K/V, block tables and lengths, the
-         step (direct calls), and D2H of the output, all inside the timed
+         pinned host memory: one H2D copy of q, new K/V, block tables and
+         lengths packed together, the step (direct calls on views of the
+         device copy), and D2H of the output, all inside the timed
          events; a device spin before each step lets the host enqueue it
          ahead, so host issue latency stays out.
 roofline = the decode call alone (pass 1 + merge) against the measured HBM
@@ -541,13 +542,30 @@ def run_ours(args):
         del g_contig
 
     # ---- end to end through the public API with host buffers
-    pin = lambda t: t.detach().to("cpu").pin_memory()
-    h_q, h_kn, h_vn = pin(case.q), pin(case.k_new), pin(case.v_new)
-    h_bt, h_lens = pin(case.block_tables), pin(case.lengths)
+    # The step's inputs (q, new K/V, block tables, lengths) sit in one pinned
+    # host buffer and cross to the device in one copy; the API gets tensor
+    # views of the device copy.
+    srcs = [case.q, case.k_new, case.v_new, case.block_tables, case.lengths]
+    if not plain_decode:  # the new tokens' sequences and positions, and the copy-on-write pairs
+        srcs += [case.new_seq_ids, case.new_positions, case.cow_pairs]
+    offs, total = [], 0
+    for t in srcs:
+        offs.append(total)
+        total += -(-t.numel() * t.element_size() // 256) * 256
+    h_pack = torch.empty(total, dtype=torch.uint8).pin_memory()
+    d_pack = torch.empty(total, dtype=torch.uint8, device=dev)
+
+    def view(buf, i):
+        t = srcs[i]
+        n = t.numel() * t.element_size()
+        return buf[offs[i]: offs[i] + n].view(t.dtype).view(t.shape)
+
+    for i, t in enumerate(srcs):
+        view(h_pack, i).copy_(t.detach().cpu())
+    d_q, d_kn, d_vn, d_bt, d_lens = (view(d_pack, i) for i in range(5))
+    d_sid, d_pos, d_pairs = (view(d_pack, i) for i in range(5, 8)) if not plain_decode else (None, None, None)
     h_out = torch.empty(B, Hq, D, dtype=torch.float32).pin_memory()
-    d_q, d_kn, d_vn = torch.empty_like(case.q), torch.empty_like(case.k_new), torch.empty_like(case.v_new)
-    d_bt, d_lens = torch.empty_like(bt), torch.empty_like(lens)
-    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_kn, h_vn, h_bt, h_lens))
+    h2d = total
     d2h = h_out.numel() * h_out.element_size()
     e2e_ev = []
     for i in range(args.warmup + args.steps):
@@ -558,15 +576,14 @@ def run_ours(args):
         torch.cuda._sleep(SPIN_CYCLES)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for dst, src in ((d_q, h_q), (d_kn, h_kn), (d_vn, h_vn), (d_bt, h_bt), (d_lens, h_lens)):
-            dst.copy_(src, non_blocking=True)
+        d_pack.copy_(h_pack, non_blocking=True)
         if plain_decode:
             pa.decode_step(d_q, d_kn, d_vn, case.k_pool, case.v_pool, d_bt, d_lens, max_len, case.scale, out, slots,
                            workspace=ws, partition_size=part)
         else:
-            if pairs.numel():
-                pa.pa_copy_blocks(case.k_pool, case.v_pool, pairs)
-            pa.pa_slot_mapping(d_bt, sid, pos, bs, slots)
+            if d_pairs.numel():
+                pa.pa_copy_blocks(case.k_pool, case.v_pool, d_pairs)
+            pa.pa_slot_mapping(d_bt, d_sid, d_pos, bs, slots)
             pa.pa_reshape_and_cache(d_kn, d_vn, case.k_pool, case.v_pool, slots)
             pa.pa_paged_attention_decode(d_q, case.k_pool, case.v_pool, d_bt, d_lens, max_len, case.scale, out,
                                          partition_size=part, workspace=ws)

@@ -87,6 +87,27 @@ def test_prefill_nonpositive_scale(pa, scale):
     assert pa.pa_read_error_flag() == 0
 
 
+def test_prefill_empty_chunks_and_empty_sequence(pa):
+    """Sequences with no new tokens (one of them empty) take no query rows and
+    leave their neighbours' rows exact; max_query_len above the longest chunk
+    only adds CTAs that exit at once."""
+    case = custom_case([0, 50, 300, 7, 129], 16, 4, 64, 16, torch.bfloat16, seed=12)
+    Hq, D = 16, 64
+    news = [0, 0, 130, 7, 0]
+    qs = np.concatenate([[0], np.cumsum(news)]).astype(np.int32)
+    T = int(qs[-1])
+    g = torch.Generator().manual_seed(13)
+    q = torch.randn(T, Hq, D, generator=g).to(torch.bfloat16)
+    out = torch.full((T, Hq, D), float("nan"), dtype=torch.float32, device="cuda")
+    pa.pa_paged_attention_prefill(q.cuda(), case.k_pool.cuda(), case.v_pool.cuda(), case.block_tables.cuda(),
+                                  case.lengths.cuda(), torch.from_numpy(qs).cuda(), 512, case.scale, out)
+    torch.cuda.synchronize()
+    ref = oracle.paged_prefill(np_of(q), np_of(case.k_pool), np_of(case.v_pool), np_of(case.block_tables),
+                               np_of(case.lengths), qs, case.scale, 16)
+    assert_matches_oracle(out, ref, True, "empty chunks")
+    assert pa.pa_read_error_flag() == 0
+
+
 def test_prefill_never_reads_past_the_sequence(pa):
     lengths = [40, 129, 17]
     case = custom_case(lengths, 8, 2, 128, 16, torch.bfloat16, seed=7, extra_blocks=6)
