@@ -84,9 +84,10 @@ def parse():
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", default="decode", choices=["decode", "prefill"],
+    ap.add_argument("--op", default="decode", choices=["decode", "prefill", "blocks"],
                     help="decode: the decode step (default); prefill: causal multi-query paged attention "
-                         "on a chunked-prefill workload, in TFLOP/s")
+                         "on a chunked-prefill workload, in TFLOP/s; blocks: copy_blocks inside the device "
+                         "pool and swap_blocks to and from a pinned host pool, in GB/s")
     return ap.parse_args()
 
 
@@ -737,6 +738,88 @@ def time_oracle_prefill(case, q, n, L, bs, min_seconds=10.0, max_reps=100):
                       f"{reps} repetition(s), {sec:.2f} s each, {t_total:.1f} s in all", "seconds_per_step": sec}
 
 
+def run_blocks(args):
+    """Whole-block copies for 2048 scattered blocks (256 MiB of K+V at 8 kv
+    heads, bs 16, head_dim 128, bf16): pa_copy_blocks inside the device pool
+    (copy-on-write) against the measured HBM copy bandwidth, and
+    pa_swap_blocks between the device pool and a pinned host pool, each way,
+    against a plain contiguous copy of the same bytes over the same host link
+    (torch copy_, one DMA transfer) measured in the same run."""
+    import paged_kv_cache_355_b200 as pa
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    NB, Hkv, bs, D = 2048, 8, 16, 128
+    g = torch.Generator(device=dev).manual_seed(3001)
+    k = torch.randn(NB, Hkv, bs, D, generator=g, device=dev).to(torch.bfloat16)
+    v = torch.randn(NB, Hkv, bs, D, generator=g, device=dev).to(torch.bfloat16)
+    hk = torch.empty(NB, Hkv, bs, D, dtype=torch.bfloat16).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    perm = torch.randperm(NB, generator=torch.Generator().manual_seed(3002))
+    m = torch.stack([torch.arange(NB), perm], 1).to(torch.int64).to(dev)
+    nbytes = 2 * k.numel() * k.element_size()
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        evs = []
+        for _ in range(args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            evs.append((e0, e1))
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b_) for a, b_ in evs) / len(evs)
+
+    # copy-on-write inside a 4096-block device pool: blocks 0..2047 to 2048..4095, scattered
+    pool_k = torch.empty(2 * NB, Hkv, bs, D, dtype=torch.bfloat16, device=dev).normal_()
+    pool_v = torch.empty_like(pool_k).normal_()
+    cp = torch.stack([perm, NB + torch.randperm(NB, generator=torch.Generator().manual_seed(3003))], 1)
+    cp = cp.to(torch.int64).to(dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    clean = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    with ClockSampler(0) as clocks:
+        evs = []
+        for i in range(args.warmup + args.steps):
+            flush.zero_()
+            clean.sum()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            pa.pa_copy_blocks(pool_k, pool_v, cp)
+            e1.record()
+            if i >= args.warmup:
+                evs.append((e0, e1))
+        torch.cuda.synchronize()
+        ms_copy = sum(a.elapsed_time(b_) for a, b_ in evs) / len(evs)
+        ms_out = timed(lambda: pa.pa_swap_blocks(k, v, hk, hv, m))
+        ms_in = timed(lambda: pa.pa_swap_blocks(hk, hv, k, v, m))
+        ms_d2h = timed(lambda: (hk.copy_(k, non_blocking=True), hv.copy_(v, non_blocking=True)))
+        ms_h2d = timed(lambda: (k.copy_(hk, non_blocking=True), v.copy_(hv, non_blocking=True)))
+    assert pa.pa_read_error_flag() == 0
+    gbs = lambda ms: nbytes / (ms * 1e-3) / 1e9
+    out, inn, d2h, h2d = gbs(ms_out), gbs(ms_in), gbs(ms_d2h), gbs(ms_h2d)
+    copy_gbs = 2 * nbytes / (ms_copy * 1e-3) / 1e9  # read and written
+    peak, peak_kind = measured_hbm_peak()
+    print(json.dumps({
+        "metric": "pa_copy_blocks GB/s vs HBM peak; pa_swap_blocks host-link GB/s vs a plain copy",
+        "value": copy_gbs, "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "2048 scattered blocks, 8 kv heads, block_size 16, head_dim 128, bf16 "
+                               f"({nbytes} bytes of K and V per direction)",
+                   "l2": "flushed before each copy_blocks launch (256 MiB written, 256 MiB read)"},
+        "roofline": {"bound": "hbm", "achieved": copy_gbs, "peak": peak, "unit": "GB/s", "frac": copy_gbs / peak,
+                     "traffic": None, "kernel": "pa_copy_blocks (read + written bytes)",
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)"},
+        "copy_blocks": {"ms": ms_copy, "gbs": copy_gbs},
+        "swap_out": {"ms": ms_out, "gbs": out, "frac_of_plain_copy": out / d2h},
+        "swap_in": {"ms": ms_in, "gbs": inn, "frac_of_plain_copy": inn / h2d},
+        "host_link": {"d2h_gbs": d2h, "h2d_gbs": h2d,
+                      "source": "torch copy_ of the same bytes, contiguous, measured in this run"},
+        "clocks": clocks.summary()}), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -744,6 +827,9 @@ def main():
         return
     if args.op == "prefill":
         run_prefill(args)
+        return
+    if args.op == "blocks":
+        run_blocks(args)
         return
     run_ours(args)
     if int(os.environ.get("WORLD_SIZE", "1")) > 1:

@@ -73,3 +73,11 @@ def test_prefill_bench_line(bench, capsys):
     r = d["roofline"]
     assert r["bound"] == "tensor" and abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-9
     assert d["cpu_baseline"] is None  # skipped with --no-cpu-baseline
+
+
+def test_blocks_bench_line(bench, capsys):
+    bench.run_blocks(_args(op="blocks", steps=2, warmup=1))
+    d = _line(capsys)
+    assert d["unit"] == "GB/s" and d["value"] > 0 and d["roofline"]["bound"] == "hbm"
+    assert d["swap_out"]["gbs"] > 0 and d["swap_in"]["gbs"] > 0
+    assert d["host_link"]["d2h_gbs"] > 0 and d["host_link"]["h2d_gbs"] > 0
