@@ -108,6 +108,26 @@ def test_prefill_empty_chunks_and_empty_sequence(pa):
     assert pa.pa_read_error_flag() == 0
 
 
+@pytest.mark.parametrize("seed", range(6))
+def test_prefill_random_shapes(pa, seed):
+    """Seeded random head_dim, block size, group size, batch, lengths and
+    chunk sizes (zero-length chunks included), four cases per seed."""
+    rng = np.random.default_rng(100 + seed)
+    for it in range(4):
+        D = int(rng.choice([64, 128]))
+        bs = int(rng.choice([8, 16, 32]))
+        G = int(rng.choice([1, 2, 4, 8, 16]))
+        Hkv = int(rng.integers(1, 3))
+        lengths = [int(x) for x in rng.integers(1, 700, int(rng.integers(1, 5)))]
+        news = [int(rng.integers(0, L + 1)) for L in lengths]
+        if sum(news) == 0:
+            news[0] = lengths[0]
+        case = custom_case(lengths, Hkv * G, Hkv, D, bs, torch.bfloat16, seed=1000 * seed + it)
+        out, ref = _run(pa, case, news)
+        assert_matches_oracle(out, ref, True, f"random prefill seed {seed}.{it} D{D} bs{bs} G{G} {lengths} {news}")
+    assert pa.pa_read_error_flag() == 0
+
+
 def test_prefill_never_reads_past_the_sequence(pa):
     lengths = [40, 129, 17]
     case = custom_case(lengths, 8, 2, 128, 16, torch.bfloat16, seed=7, extra_blocks=6)
