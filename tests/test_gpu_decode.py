@@ -110,6 +110,18 @@ def test_single_sequence_edge_lengths(pa, dtype):
     assert pa.pa_read_error_flag() == 0
 
 
+def test_large_batch_takes_index_order(pa):
+    """Above 2048 sequences the kernel skips the longest-first ranking and
+    takes sequences in index order; results are the same attention."""
+    rng = np.random.default_rng(21)
+    lengths = [int(x) for x in rng.integers(0, 90, 2100)]
+    case = custom_case(lengths, 4, 2, 64, 16, torch.bfloat16, seed=21)
+    for part in (0, 32):
+        out = run_gpu(pa, case, part)
+        assert_matches_oracle(out, run_oracle(case), True, f"batch 2100 P={part}")
+    assert pa.pa_read_error_flag() == 0
+
+
 def test_single_token_returns_value_bit_exactly(pa):
     case = custom_case([1, 1, 1], 8, 4, 128, 16, torch.float32, seed=11)
     out = run_gpu(pa, case)
