@@ -19,7 +19,12 @@
  *  * `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Every call only enqueues work on it and returns; a returned
  *    PA_OK means the arguments passed host-side validation and the launches
- *    were accepted, not that the kernels have finished.
+ *    were accepted, not that the kernels have finished.  The decode kernels
+ *    and pa_reshape_and_cache_decode are launched with programmatic stream
+ *    serialisation: they may be scheduled while the previous kernel on the
+ *    stream drains, but touch no global memory before it has completed, so
+ *    stream order holds exactly as for ordinary launches.  Calls may be
+ *    captured into CUDA graphs.
  *  * Element types: PA_F32 (IEEE fp32) or PA_BF16 (bfloat16).  Query, key
  *    and value share one element type; all arithmetic accumulates in fp32.
  *  * KV pool layout (the pages fix none; [P1] "The kernel side" only says
