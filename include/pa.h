@@ -85,6 +85,17 @@ const char* pa_version(void);
 int pa_read_error_flag(void* stream);
 
 /*
+ * pa_selftest_wait_timeout -- exercise the bounded-wait path without a
+ * fault (no counterpart in the pages; it exists so that tests can show a wait
+ * that runs out is reported and leaves the context usable).  Launches one
+ * CTA that waits on a shared-memory mbarrier nothing ever arrives on; after
+ * limit_us microseconds (1 .. 2,000,000) the wait gives up, records
+ * PA_ERR_TIMEOUT in the device error word and the kernel returns normally.
+ * Read the result with pa_read_error_flag.
+ */
+int pa_selftest_wait_timeout(uint32_t limit_us, void* stream);
+
+/*
  * pa_slot_mapping -- slot of each new token ([P3] "Detail": logical block
  * pos / block_size of the sequence maps to the physical block its table
  * names; the token sits at offset pos % block_size inside it).

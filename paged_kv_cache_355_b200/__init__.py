@@ -16,7 +16,7 @@ _BINDING_NAMES = (
     "pa_paged_attention_decode", "pa_paged_attention_decode_contiguous", "pa_paged_attention_partition_size",
     "pa_paged_attention_workspace_size", "pa_read_error_flag", "pa_reshape_and_cache", "pa_slot_mapping",
     "pa_status_string", "pa_version", "pa_paged_attention_decode_static_scratch", "STATIC_SCRATCH_BYTES",
-    "pa_paged_attention_prefill", "pa_reshape_and_cache_decode",
+    "pa_paged_attention_prefill", "pa_reshape_and_cache_decode", "pa_selftest_wait_timeout",
 )
 __all__ = list(_BINDING_NAMES) + ["decode_step"]
 

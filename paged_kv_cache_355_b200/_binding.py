@@ -33,6 +33,7 @@ _SIGS = {
     "pa_status_string": ([_I], ctypes.c_char_p),
     "pa_version": ([], ctypes.c_char_p),
     "pa_read_error_flag": ([_P], _I),
+    "pa_selftest_wait_timeout": ([ctypes.c_uint32, _P], _I),
     "pa_slot_mapping": ([_P, _I, _I, _P, _P, _I64, _I, _P, _P], _I),
     "pa_decode_slot_mapping": ([_P, _I, _P, _I, _I, _P, _P], _I),
     "pa_reshape_and_cache": ([_P, _P, _P, _P, _P, _I64, _I, _I, _I, _I64, _I, _P], _I),
@@ -116,6 +117,10 @@ def pa_version() -> str:
 def pa_read_error_flag(stream=None) -> int:
     """Synchronise the stream and return (then clear) the device error word."""
     return int(_lib.pa_read_error_flag(_stream(stream)))
+
+
+def pa_selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    _check("pa_selftest_wait_timeout", _lib.pa_selftest_wait_timeout(limit_us, _stream(stream)))
 
 
 def pa_slot_mapping(block_tables, seq_ids, positions, block_size: int, slot_mapping, stream=None) -> None:

@@ -5,6 +5,7 @@
 #include <mutex>
 
 #include "pa.h"
+#include "pa_device.cuh"
 #include "pa_internal.h"
 
 namespace pa {
@@ -50,7 +51,29 @@ int num_sms() {
     return g_num_sms[dev];
 }
 
+namespace {
+// One CTA waits on an mbarrier that nothing ever arrives on: the bounded wait
+// runs out after limit_ns, records PA_ERR_TIMEOUT and the kernel returns.
+__global__ void wait_selftest_kernel(int* err, uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait_for(&bar, 0, err, limit_ns);
+}
+}  // namespace
+
 }  // namespace pa
+
+extern "C" int pa_selftest_wait_timeout(uint32_t limit_us, void* stream) {
+    if (limit_us == 0 || limit_us > 2000000u) return PA_ERR_INVALID_ARG;
+    int* err = pa::error_word_ptr();
+    if (!err) return PA_ERR_CUDA;
+    pa::wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(err, (uint64_t)limit_us * 1000u);
+    return pa::launch_status();
+}
 
 extern "C" const char* pa_status_string(int status) {
     switch (status) {

@@ -73,16 +73,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Bounded: after
-// kWaitLimitNs (or 2^30 polls) it records PA_ERR_TIMEOUT and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
+// limit_ns (or 2^30 polls) it records PA_ERR_TIMEOUT and returns false.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, int* err, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1; it < (1u << 30); ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) break;
+        if ((it & 63u) == 0 && global_timer_ns() - t0 > limit_ns) break;
     }
     record_error(err, PA_ERR_TIMEOUT);
     return false;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
+    return mbar_wait_for(bar, parity, err, kWaitLimitNs);
 }
 
 // Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from

@@ -122,3 +122,8 @@ def test_cache_kernels_reject_bad_arguments(lib):
     assert lib.pa_slot_mapping(P(0), 4, 2, P(16), P(16), I64(3), 16, P(16), None) == INVALID
     assert lib.pa_slot_mapping(P(16), 4, 2, P(16), P(16), I64(3), 0, P(16), None) == INVALID
     assert lib.pa_decode_slot_mapping(P(16), 4, P(0), 2, 16, P(16), None) == INVALID
+
+
+def test_selftest_rejects_bad_limits(lib):
+    assert lib.pa_selftest_wait_timeout(0, None) == INVALID
+    assert lib.pa_selftest_wait_timeout(2_000_001, None) == INVALID
