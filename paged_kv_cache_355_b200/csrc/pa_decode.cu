@@ -838,19 +838,19 @@ __global__ void __launch_bounds__(kDecodeThreads)
 }
 
 // Second pass: out = sum_s w_s o_s / sum_s w_s with w_s = l_s * 2^(m_s - max m),
-// for sequences that were cut into more than one split.  Four warps share a
-// (sequence, query head) row, two rows per CTA: warp k of a row takes splits
-// k, k + 4, ..., eight at a time, issuing all their (m, l) and partial-row
+// for sequences that were cut into more than one split.  W warps share a
+// (sequence, query head) row: W = 4 with two rows per CTA, or W = 8 with one
+// row per CTA when rows are few and splits many.  Warp k of a row takes
+// splits k, k + W, ..., eight at a time, issuing all their (m, l) and partial-row
 // loads before it needs any of them (lane i holds output elements
 // [i * D / 32, (i + 1) * D / 32)), and keeps its own running max, weight sum
-// and accumulator; the four warps' states are then combined through shared
+// and accumulator; the W warps' states are then combined through shared
 // memory by the row's first warp.  The order of every sum is fixed, so the
 // result is deterministic.
 constexpr int kMergeWarps = 8;
-constexpr int kMergeWarpsPerRow = 4;
 constexpr int kMergeChunk = 8;  // splits per warp in flight
 
-template <int D>
+template <int D, int kMergeWarpsPerRow>
 __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(const DecodeParams p, int64_t rows) {
     constexpr int VPL = D / 32;  // output elements per lane
     constexpr int STRIDE = kMergeWarpsPerRow * kMergeChunk;
@@ -1125,10 +1125,18 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
     if (rc) return rc;
     if (plan.max_splits > 1) {
         const int64_t rows = (int64_t)batch * p.num_q_heads;
-        constexpr int rows_per_cta = kMergeWarps / kMergeWarpsPerRow;
+        // four warps per row, or all eight of a CTA when rows carry many splits
+        // and there are too few rows to fill the GPU with four-warp groups
+        const bool wide = plan.max_splits > 32 && rows < (int64_t)num_sms() * 2;
+        const int rows_per_cta = wide ? 1 : kMergeWarps / 4;
         const unsigned blocks = (unsigned)((rows + rows_per_cta - 1) / rows_per_cta);
-        rc = head_dim == 128 ? launch_pdl(decode_merge_kernel<128>, dim3(blocks), dim3(32 * kMergeWarps), 0, st, p, rows)
-                             : launch_pdl(decode_merge_kernel<64>, dim3(blocks), dim3(32 * kMergeWarps), 0, st, p, rows);
+        const dim3 mg(blocks), mb(32 * kMergeWarps);
+        if (head_dim == 128)
+            rc = wide ? launch_pdl(decode_merge_kernel<128, 8>, mg, mb, 0, st, p, rows)
+                      : launch_pdl(decode_merge_kernel<128, 4>, mg, mb, 0, st, p, rows);
+        else
+            rc = wide ? launch_pdl(decode_merge_kernel<64, 8>, mg, mb, 0, st, p, rows)
+                      : launch_pdl(decode_merge_kernel<64, 4>, mg, mb, 0, st, p, rows);
     }
     return rc;
 }
