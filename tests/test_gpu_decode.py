@@ -122,6 +122,16 @@ def test_large_batch_takes_index_order(pa):
     assert pa.pa_read_error_flag() == 0
 
 
+@pytest.mark.parametrize("part", [0, 512])
+def test_many_splits_few_rows(pa, part):
+    """Few long rows cut into many splits: the merge gives each row a whole
+    CTA (eight warps)."""
+    case = custom_case([30001, 17000, 1], 8, 2, 128, 16, torch.bfloat16, seed=22)
+    out = run_gpu(pa, case, part)
+    assert_matches_oracle(out, run_oracle(case), True, f"many splits P={part}")
+    assert pa.pa_read_error_flag() == 0
+
+
 def test_single_token_returns_value_bit_exactly(pa):
     case = custom_case([1, 1, 1], 8, 4, 128, 16, torch.float32, seed=11)
     out = run_gpu(pa, case)
