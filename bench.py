@@ -3,12 +3,12 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 A step is one decode step of one attention layer over one batch: the new
-token's slot and its K/V write (pa_reshape_and_cache_decode, one launch; the
-workloads that append several tokens per sequence use pa_slot_mapping and
-pa_reshape_and_cache), copy-on-write copies when the workload has them
-(pa_copy_blocks), and paged decode attention over every sequence
-(pa_paged_attention_decode, pass 1 plus the split-KV merge when a sequence is
-split).  Inputs are seeded synthetic tensors shaped like the named workload,
+token's slot and its K/V write, and paged decode attention over every
+sequence, in one call (pa_paged_attention_decode_append: for bf16 one pass-1
+launch that also writes the new token, plus the split-KV merge when a
+sequence is split).  The workloads that append several tokens per sequence
+run pa_slot_mapping and pa_reshape_and_cache, copy-on-write copies when the
+workload has them (pa_copy_blocks), and pa_paged_attention_decode.  Inputs are seeded synthetic tensors shaped like the named workload,
 resident in HBM before timing.
 
 Timing: W untimed warm-up steps, then the step is captured into a CUDA graph
@@ -415,8 +415,14 @@ def run_ours(args):
                                      partition_size=part, workspace=ws)
 
     def step():
-        cache_part()
-        decode_part()
+        if plain_decode and w.dtype == torch.bfloat16:
+            # the new token's slot and cache write folded into the attention launch
+            pa.pa_paged_attention_decode_append(case.q, case.k_new, case.v_new, case.k_pool, case.v_pool, bt, lens,
+                                                max_len, case.scale, out, partition_size=part, workspace=ws,
+                                                slot_mapping=slots)
+        else:
+            cache_part()
+            decode_part()
 
     def flush_l2():
         # write a buffer twice the L2, then read another one, so that the
@@ -428,6 +434,7 @@ def run_ours(args):
     max_splits = -(-max(max_len, 1) // part)
     cache_launches = (1 if pairs.numel() else 0) + (1 if plain_decode else 2)
     decode_launches = 1 + (1 if max_splits > 1 else 0)
+    step_launches = decode_launches + (0 if plain_decode and w.dtype == torch.bfloat16 else cache_launches)
 
     # ---- device-resident timed region
     # The step is captured once into a CUDA graph and replayed, as a serving
@@ -634,14 +641,16 @@ def run_ours(args):
                           else ["pa_slot_mapping", "pa_reshape_and_cache"]),
                        "ms": ms_cache, "bytes": cache_bytes, "gbs": cache_bytes / (ms_cache * 1e-3) / 1e9,
                        "frac": cache_bytes / (ms_cache * 1e-3) / 1e9 / peak,
-                       "note": "timed alone as one graph; small writes are launch-latency bound"},
+                       "note": "timed alone as one graph; small writes are launch-latency bound"
+                               + ("; the bf16 decode step itself does this write inside its attention launch"
+                                  if plain_decode and w.dtype == torch.bfloat16 else "")},
         "paging_overhead": {"paged_ms_median": paged_med, "contiguous_ms_median": contig_med,
                             "overhead": paged_med / contig_med - 1.0, "contiguous_ms_mean_max_ranks": ms_contig},
         "e2e": {"value": world * kv_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
                 "timing": "device time from before the H2D copies to after the D2H read-back, direct API calls "
                           "(no graph); a device spin ahead of each step keeps host issue latency out"},
-        "gpu_launches": (cache_launches + decode_launches) * args.steps,
+        "gpu_launches": step_launches * args.steps,
         "gpu_launches_decode_roofline_loop": decode_launches * args.steps,
         "timing": ("K replays of the step's CUDA graph (value), then K replays of the decode call's graph "
                    "(roofline), each bracketed by events" if graphs is not None else "direct calls"),

@@ -251,6 +251,30 @@ int pa_paged_attention_decode(const void* q, const void* k_pool, const void* v_p
                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * pa_paged_attention_decode_append -- one whole decode step: the new token's
+ * slot and cache write (exactly pa_reshape_and_cache_decode: token b is
+ * position context_lens[b] - 1 of sequence b) followed by
+ * pa_paged_attention_decode over lengths that include it ([P3] "Key
+ * Technical Innovations" item 2 for the write, [P1] "The kernel side" for the
+ * attention).  Arguments are those of the two calls: key, value
+ * [batch][num_kv_heads][head_dim] (kv_dtype); slot_mapping int64 [batch]
+ * output or NULL.  The pools are updated in place, bit for bit as the
+ * two-call sequence leaves them, and the output matches it within rounding.
+ * For bf16 it is one launch (plus the merge when sequences are split): the
+ * CTA that reads a sequence's last block writes the new K and V rows into
+ * the pool slot and into the tile it has staged, so no separate write kernel
+ * runs.  fp32 runs the two calls.  Errors as for the two calls.
+ */
+int pa_paged_attention_decode_append(const void* q, const void* key, const void* value,
+                                     void* k_pool, void* v_pool, const int32_t* block_tables,
+                                     int max_blocks_per_seq, const int32_t* context_lens,
+                                     int max_context_len, float scale, int block_size, void* out,
+                                     int out_dtype, int batch, int num_q_heads, int num_kv_heads,
+                                     int head_dim, int64_t num_blocks, int kv_dtype,
+                                     int partition_size, void* workspace, size_t workspace_bytes,
+                                     int64_t* slot_mapping, void* stream);
+
+/*
  * pa_paged_attention_prefill -- causal attention for several new query
  * tokens per sequence over the paged cache (chunked prefill, or speculative
  * tokens): the multi-query form of pa_paged_attention_decode, reading K and V

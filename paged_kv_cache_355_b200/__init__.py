@@ -17,6 +17,7 @@ _BINDING_NAMES = (
     "pa_paged_attention_workspace_size", "pa_read_error_flag", "pa_reshape_and_cache", "pa_slot_mapping",
     "pa_status_string", "pa_version", "pa_paged_attention_decode_static_scratch", "STATIC_SCRATCH_BYTES",
     "pa_paged_attention_prefill", "pa_reshape_and_cache_decode", "pa_selftest_wait_timeout",
+    "pa_paged_attention_decode_append",
 )
 __all__ = list(_BINDING_NAMES) + ["decode_step"]
 
@@ -36,9 +37,9 @@ def decode_step(q, k_new, v_new, k_pool, v_pool, block_tables, context_lens, max
     """One decode step of one attention layer, entirely in libpa's kernels:
 
     1. copy_blocks for pending copy-on-write pairs (if any),
-    2. the new token's slot from the block table and the write of its K and V
-       there, in one launch (pa_reshape_and_cache_decode),
-    3. paged decode attention over every sequence (pa_paged_attention_decode).
+    2. the new token's slot from the block table, the write of its K and V
+       there, and paged decode attention over every sequence
+       (pa_paged_attention_decode_append: one launch for bf16).
 
     `context_lens` counts the new token; `slots` is an int64 [B] output buffer
     (or None) that receives each token's slot.
@@ -47,6 +48,6 @@ def decode_step(q, k_new, v_new, k_pool, v_pool, block_tables, context_lens, max
 
     if cow_pairs is not None and cow_pairs.numel():
         b.pa_copy_blocks(k_pool, v_pool, cow_pairs, stream=stream)
-    b.pa_reshape_and_cache_decode(k_new, v_new, k_pool, v_pool, block_tables, context_lens, slots, stream=stream)
-    b.pa_paged_attention_decode(q, k_pool, v_pool, block_tables, context_lens, max_context_len, scale, out,
-                                partition_size=partition_size, workspace=workspace, stream=stream)
+    b.pa_paged_attention_decode_append(q, k_new, v_new, k_pool, v_pool, block_tables, context_lens, max_context_len,
+                                       scale, out, partition_size=partition_size, workspace=workspace,
+                                       slot_mapping=slots, stream=stream)

@@ -44,6 +44,8 @@ _SIGS = {
     "pa_paged_attention_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
     "pa_paged_attention_decode": ([_P, _P, _P, _P, _I, _P, _I, _F, _I, _P, _I, _I, _I, _I, _I, _I64, _I, _I, _P,
                                    _SZ, _P], _I),
+    "pa_paged_attention_decode_append": ([_P, _P, _P, _P, _P, _P, _I, _P, _I, _F, _I, _P, _I, _I, _I, _I, _I, _I64, _I,
+                                          _I, _P, _SZ, _P, _P], _I),
     "pa_paged_attention_decode_contiguous": ([_P, _P, _P, _I64, _P, _I, _F, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P,
                                               _SZ, _P], _I),
     "pa_paged_attention_prefill": ([_P, _P, _P, _P, _I, _P, _P, _I, _F, _I, _P, _I, _I, _I, _I, _I, _I64, _I64, _I,
@@ -255,6 +257,32 @@ def pa_paged_attention_decode(q, k_pool, v_pool, block_tables, context_lens, max
         _dev(q, "q"), k_pool.data_ptr(), v_pool.data_ptr(), _dev(block_tables, "block_tables", torch.int32), MBS,
         _dev(context_lens, "context_lens", torch.int32), int(max_context_len), float(scale), bs, _dev(out, "out"),
         _kv_dtype(out), B, Hq, Hkv, D, NB, dt, partition_size, ws, ws_bytes, _stream(stream)))
+
+
+def pa_paged_attention_decode_append(q, key, value, k_pool, v_pool, block_tables, context_lens, max_context_len: int,
+                                     scale: float, out, partition_size: int = 0, workspace=None, slot_mapping=None,
+                                     stream=None) -> None:
+    """One decode step: write each sequence's new token (position
+    context_lens[b] - 1) into the pool, then attend over the lengths that
+    include it."""
+    B, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_pool.shape
+    if D2 != D or v_pool.shape != k_pool.shape or tuple(out.shape) != (B, Hq, D):
+        raise ValueError("q / pool / out shapes disagree")
+    if tuple(key.shape) != (B, Hkv, D) or value.shape != key.shape:
+        raise ValueError("key / value must be [batch, num_kv_heads, head_dim]")
+    MBS = block_tables.shape[1]
+    dt = _kv_dtype(q)
+    for t, n in ((key, "key"), (value, "value"), (k_pool, "k_pool"), (v_pool, "v_pool")):
+        _dev(t, n, q.dtype)
+    need = pa_paged_attention_workspace_size(B, Hq, Hkv, D, max_context_len, bs, partition_size)
+    ws, ws_bytes = _workspace(workspace, need, q.device, stream)
+    slots = _dev(slot_mapping, "slot_mapping", torch.int64) if slot_mapping is not None else None
+    _check("pa_paged_attention_decode_append", _lib.pa_paged_attention_decode_append(
+        _dev(q, "q"), key.data_ptr(), value.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
+        _dev(block_tables, "block_tables", torch.int32), MBS, _dev(context_lens, "context_lens", torch.int32),
+        int(max_context_len), float(scale), bs, _dev(out, "out"), _kv_dtype(out), B, Hq, Hkv, D, NB, dt,
+        partition_size, ws, ws_bytes, slots, _stream(stream)))
 
 
 def pa_paged_attention_decode_contiguous(q, k_c, v_c, context_lens, max_context_len: int, scale: float, out,

@@ -103,6 +103,15 @@ struct DecodeParams {
     int batch;
     int longest_first;  // blockIdx.z is a rank in decreasing-length order
     float scale_log2;
+    // decode step with the new token's cache write folded in (bf16 only):
+    // token b is position context_lens[b] - 1 of sequence b; its K and V rows
+    // k_new / v_new [batch][Hkv][D] go to the pool slot and into the staged
+    // tile of the CTA that owns that position; slots (optional) receives the
+    // slot of each token
+    const void* k_new;
+    const void* v_new;
+    int64_t* slots;
+    int append;
 };
 
 template <typename T>
@@ -551,6 +560,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
     const int G = p.num_q_heads / p.num_kv_heads;
 
     const int L = clamp_len(p, b, threadIdx.x == 0 && split == 0 && kvh == 0);
+    if (p.append && L == 0 && split == 0 && kvh == 0 && threadIdx.x == 0 && p.slots) p.slots[b] = -1;
     const int tok_begin = split * p.partition;
     if (split > 0 && tok_begin >= L) return;
     const int ntok = max(0, min(L, tok_begin + p.partition) - tok_begin);
@@ -664,6 +674,17 @@ __global__ void __launch_bounds__(kDecodeThreads)
         }
         const int q4 = lane >> 3;  // which of the four ldmatrix matrices this lane addresses
         const int r8 = lane & 7;   // which row of it
+        // a folded-in cache write: the warp that takes the last stage of the
+        // sequence's last split loads the new K and V rows now, so their
+        // latency is hidden behind the stream (lane c holds 16-byte chunk c)
+        const bool appends = p.append && nstage > 0 && split == num_splits_b - 1 &&
+                             (nstage - 1) % kConsumerWarps == cw;
+        uint4 new_k = make_uint4(0u, 0u, 0u, 0u), new_v = new_k;
+        if (appends && lane < D / 8) {
+            const int64_t src = ((int64_t)b * p.num_kv_heads + kvh) * (D / 8) + lane;
+            new_k = static_cast<const uint4*>(p.k_new)[src];
+            new_v = static_cast<const uint4*>(p.v_new)[src];
+        }
         for (int j = cw; j < nstage; j += kConsumerWarps) {
             const int slot = j % p.stages;
             if (!mbar_wait(&full[slot], (j / p.stages) & 1, p.err)) {
@@ -685,6 +706,29 @@ __global__ void __launch_bounds__(kDecodeThreads)
                     *reinterpret_cast<uint4*>(vstage + (rem >> 3) * SLAB_BYTES + row * 128 + (rem & 7) * 16) =
                         make_uint4(0u, 0u, 0u, 0u);
                 }
+                __syncwarp();
+            }
+            if (appends && j == nstage - 1) {
+                // the appended token is the stage's last valid row: its K and V
+                // rows (loaded at the start) go into the staged tile, whatever
+                // the copy brought from the slot, and into the pool slot itself
+                const int r = valid - 1;
+                const int pos = L - 1;
+                const int32_t phys = tbl[(pos - tok_begin) / p.block_size];
+                const bool in_pool = phys >= 0 && phys < p.num_blocks;
+                const int64_t dst = (((int64_t)phys * p.num_kv_heads + kvh) * p.block_size + pos % p.block_size) * (D / 8);
+                if (lane < D / 8) {
+                    const int c = lane;
+                    const int off = (c >> 3) * SLAB_BYTES + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+                    *reinterpret_cast<uint4*>(kstage + off) = new_k;
+                    *reinterpret_cast<uint4*>(vstage + off) = new_v;
+                    if (in_pool) {
+                        static_cast<uint4*>(const_cast<void*>(p.k))[dst + c] = new_k;
+                        static_cast<uint4*>(const_cast<void*>(p.v))[dst + c] = new_v;
+                    }
+                }
+                if (lane == 0 && kvh == 0 && p.slots)
+                    p.slots[b] = phys >= 0 ? (int64_t)phys * p.block_size + pos % p.block_size : -1;
                 __syncwarp();
             }
             // S^T = K . Q^T : two 16-token M tiles
@@ -1213,6 +1257,59 @@ extern "C" int pa_paged_attention_decode(const void* q, const void* k_pool, cons
     p.out_bf16 = out_dtype == PA_BF16;
     p.contiguous = 0;
     p.scale_log2 = scale * kLog2e;
+    return run_decode(p, head_dim, kv_dtype, batch, workspace, workspace_bytes, max_context_len, partition_size,
+                      static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int pa_paged_attention_decode_append(const void* q, const void* key, const void* value, void* k_pool,
+                                                void* v_pool, const int32_t* block_tables, int max_blocks_per_seq,
+                                                const int32_t* context_lens, int max_context_len, float scale,
+                                                int block_size, void* out, int out_dtype, int batch, int num_q_heads,
+                                                int num_kv_heads, int head_dim, int64_t num_blocks, int kv_dtype,
+                                                int partition_size, void* workspace, size_t workspace_bytes,
+                                                int64_t* slot_mapping, void* stream) {
+    int rc = check_shapes(batch, num_q_heads, num_kv_heads, head_dim, block_size, kv_dtype, out_dtype,
+                          max_context_len);
+    if (rc) return rc;
+    if (max_blocks_per_seq < 0 || num_blocks < 0) return PA_ERR_INVALID_ARG;
+    if ((int64_t)max_context_len > (int64_t)max_blocks_per_seq * block_size) return PA_ERR_INVALID_ARG;
+    if (batch == 0) return PA_OK;
+    if (!q || !key || !value || !k_pool || !v_pool || !block_tables || !context_lens || !out)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(key) || !aligned16(value) || !aligned16(k_pool) || !aligned16(v_pool))
+        return PA_ERR_INVALID_ARG;
+    if (kv_dtype != PA_BF16) {
+        // fp32: the write and the attention as two launches
+        rc = pa_reshape_and_cache_decode(key, value, k_pool, v_pool, block_tables, max_blocks_per_seq, context_lens,
+                                         batch, num_kv_heads, head_dim, block_size, num_blocks, kv_dtype,
+                                         slot_mapping, stream);
+        if (rc) return rc;
+        return pa_paged_attention_decode(q, k_pool, v_pool, block_tables, max_blocks_per_seq, context_lens,
+                                         max_context_len, scale, block_size, out, out_dtype, batch, num_q_heads,
+                                         num_kv_heads, head_dim, num_blocks, kv_dtype, partition_size, workspace,
+                                         workspace_bytes, stream);
+    }
+    DecodeParams p = {};
+    p.q = q;
+    p.k = k_pool;
+    p.v = v_pool;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.out = out;
+    p.num_blocks = num_blocks;
+    p.L_pad = 0;
+    p.max_len = max_context_len;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.block_size = block_size;
+    p.out_bf16 = out_dtype == PA_BF16;
+    p.contiguous = 0;
+    p.scale_log2 = scale * kLog2e;
+    p.k_new = key;
+    p.v_new = value;
+    p.slots = slot_mapping;
+    p.append = 1;
     return run_decode(p, head_dim, kv_dtype, batch, workspace, workspace_bytes, max_context_len, partition_size,
                       static_cast<cudaStream_t>(stream));
 }

@@ -132,6 +132,49 @@ def test_many_splits_few_rows(pa, part):
     assert pa.pa_read_error_flag() == 0
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("D,bs,G", [(128, 16, 1), (128, 8, 4), (64, 32, 8), (128, 16, 16), (64, 16, 2)])
+@pytest.mark.parametrize("partition", [0, 32])
+def test_decode_append_equals_write_then_decode(pa, dtype, D, bs, G, partition):
+    """pa_paged_attention_decode_append = pa_reshape_and_cache_decode then
+    pa_paged_attention_decode: pools and slots bit for bit, attention at the
+    bar.  The appended slots start as NaN, so a tile staged before the write
+    landed would poison the result."""
+    if dtype == "f32" and G == 16:
+        pytest.skip("group size 16 is bf16 only")
+    Hkv = 2
+    lengths = [1, 17, 0, 64, 65, 200, 33]
+    case = custom_case(lengths, Hkv * G, Hkv, D, bs, DT[dtype], seed=D + bs + G)
+    B = len(lengths)
+    g = torch.Generator().manual_seed(7 * G + bs)
+    key = torch.randn(B, Hkv, D, generator=g).to(DT[dtype])
+    val = torch.randn(B, Hkv, D, generator=g).to(DT[dtype])
+    kp, vp = case.k_pool.clone(), case.v_pool.clone()
+    for b, L in enumerate(lengths):
+        if L > 0:
+            blk = int(case.block_tables[b, (L - 1) // bs])
+            kp[blk, :, (L - 1) % bs] = float("nan")
+            vp[blk, :, (L - 1) % bs] = float("nan")
+    live = np.array([b for b, L in enumerate(lengths) if L > 0], dtype=np.int32)
+    want_slots = np.full(B, -1, dtype=np.int64)
+    want_slots[live] = oracle.slot_mapping(np_of(case.block_tables), live,
+                                           np.array([lengths[b] - 1 for b in live], dtype=np.int32), bs)
+    hk, hv = np_of(kp).copy(), np_of(vp).copy()
+    oracle.reshape_and_cache(np_of(key), np_of(val), hk, hv, want_slots)
+    want = oracle.paged_decode(np_of(case.q), hk, hv, np_of(case.block_tables), np_of(case.lengths), case.scale, bs)
+    gk, gv = kp.cuda(), vp.cuda()
+    out = torch.full(tuple(case.q.shape), float("nan"), dtype=torch.float32, device="cuda")
+    slots = torch.full((B,), 7, dtype=torch.int64, device="cuda")
+    pa.pa_paged_attention_decode_append(case.q.cuda(), key.cuda(), val.cuda(), gk, gv, case.block_tables.cuda(),
+                                        case.lengths.cuda(), case.max_len, case.scale, out,
+                                        partition_size=partition, slot_mapping=slots)
+    torch.cuda.synchronize()
+    assert np.array_equal(np_of(slots), want_slots)
+    assert np_of(gk).tobytes() == hk.tobytes() and np_of(gv).tobytes() == hv.tobytes()
+    assert_matches_oracle(out, want, dtype == "bf16", f"append {dtype} D{D} bs{bs} G{G} P{partition}")
+    assert pa.pa_read_error_flag() == 0
+
+
 def test_single_token_returns_value_bit_exactly(pa):
     case = custom_case([1, 1, 1], 8, 4, 128, 16, torch.float32, seed=11)
     out = run_gpu(pa, case)
