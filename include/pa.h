@@ -263,7 +263,10 @@ int pa_paged_attention_decode(const void* q, const void* k_pool, const void* v_p
  * For bf16 it is one launch (plus the merge when sequences are split): the
  * CTA that reads a sequence's last block writes the new K and V rows into
  * the pool slot and into the tile it has staged, so no separate write kernel
- * runs.  fp32 runs the two calls.  Errors as for the two calls.
+ * runs.  fp32 runs the two calls.  Errors as for the two calls.  As for
+ * pa_reshape_and_cache, the written slots must be distinct and the block
+ * holding each one must belong to its sequence alone (no other sequence of
+ * the batch reads it), which copy-on-write before the step guarantees.
  */
 int pa_paged_attention_decode_append(const void* q, const void* key, const void* value,
                                      void* k_pool, void* v_pool, const int32_t* block_tables,
