@@ -28,9 +28,17 @@ e2e    = the same metric through the public API with the step's inputs in
          lengths packed together, the step (direct calls on views of the
          device copy), and D2H of the output, all inside the timed
          events; a device spin before each step lets the host enqueue it
-         ahead, so host issue latency stays out.
-roofline = the decode call alone (pass 1 + merge) against the measured HBM
-         copy bandwidth.
+         ahead, so host issue latency stays out.  host_wall_ms_per_step
+         times the same calls by the host clock with no spin (issue to a
+         synchronize after the read-back).
+roofline = the decode call alone (pass 1 + merge; at least 100 timed replays,
+         mean, median, p10 and p90 reported) against the measured HBM copy
+         bandwidth, and against the read ceiling that pa_hbm_read_probe (a
+         plain bulk read stream of 2 GiB) reaches in the same run.
+other_workloads = (default run only) the decode calls of the GQA,
+         long-context and shared-prefix workloads, timed the same way, with
+         their paging overheads; the shared-prefix workload also by the
+         distinct (unique) K/V bytes it reads.
 
 --impl reference times the CPU oracle (fp64, OpenMP) on the host cores on a
 bounded sample of the same workload.
@@ -84,6 +92,9 @@ def parse():
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip the GQA, long-context and shared-prefix decode calls that the default "
+                         "Llama-7B-shaped run also times")
     ap.add_argument("--op", default="decode", choices=["decode", "prefill", "blocks"],
                     help="decode: the decode step (default); prefill: causal multi-query paged attention "
                          "on a chunked-prefill workload, in TFLOP/s; blocks: copy_blocks inside the device "
@@ -374,6 +385,130 @@ def run_reference_prefill(args, world):
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
+ROOFLINE_MIN_ITERS = 100  # timed replays of the decode call alone (at least)
+PROBE_BYTES = 2 << 30     # read-ceiling probe buffer: 2 GiB, 16x the L2
+OTHER_WORKLOADS = ("gqa", "long16", "cow")
+
+
+def time_stats(ms):
+    """mean, median, p10 and p90 (nearest rank) of a list of times in ms."""
+    s = sorted(ms)
+    at = lambda f: s[min(len(s) - 1, max(0, int(round(f * (len(s) - 1)))))]
+    return {"mean": sum(s) / len(s), "median": statistics.median(s), "p10": at(0.1), "p90": at(0.9), "n": len(s)}
+
+
+def timed_replays(run, n, flush_l2, stream, warmup=0):
+    """CUDA-event times (ms) of n calls of run(), each preceded by an L2
+    flush outside the events."""
+    evs = []
+    for i in range(warmup + n):
+        flush_l2()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run()
+        e1.record(stream)
+        if i >= warmup:
+            evs.append((e0, e1))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b_) for a, b_ in evs]
+
+
+def capture(fn):
+    """fn captured into a CUDA graph (returns the graph and its replay), or
+    (None, fn) when capture is unavailable."""
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        torch.cuda.synchronize()
+        return g, g.replay
+    except Exception as exc:
+        print(f"bench: CUDA graph capture failed ({exc}); timing direct calls", file=sys.stderr)
+        return None, fn
+
+
+def make_decode_call(pa, case, bt, lens, out, part, ws, groups=None):
+    """The decode-attention call the step makes for a case: the shared-prefix
+    form when the case's sequences share prompt blocks, else the plain one."""
+    if groups is not None:
+        gs, gl, max_prefix, max_group = groups
+        return lambda: pa.pa_paged_attention_decode_shared_prefix(
+            case.q, case.k_pool, case.v_pool, bt, lens, case.max_len, case.scale, out, gs, gl, max_prefix,
+            max_group, partition_size=part, workspace=ws)
+    return lambda: pa.pa_paged_attention_decode(case.q, case.k_pool, case.v_pool, bt, lens, case.max_len, case.scale,
+                                                out, partition_size=part, workspace=ws)
+
+
+def prefix_groups(pa, case, dev):
+    """(group_starts, group_prefix_len, max_prefix_len, max_group_size) of a
+    case whose consecutive sequences share leading blocks, as device tensors;
+    None when no two sequences share a block."""
+    from paged_kv_cache_355_b200.workloads import shared_prefix_groups
+
+    groups = shared_prefix_groups(case)
+    if groups is None:
+        return None
+    starts, plen = groups
+    return (torch.tensor(starts, dtype=torch.int32, device=dev), torch.tensor(plen, dtype=torch.int32, device=dev),
+            max(plen), max(b - a for a, b in zip(starts[:-1], starts[1:])))
+
+
+def workspace_for(pa, case, part, groups):
+    w = case.workload
+    B, Hq, Hkv, D, bs = w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size
+    if groups is not None:
+        return pa.pa_paged_attention_shared_prefix_workspace_size(B, Hq, Hkv, D, case.max_len, bs,
+                                                                  groups[1].numel(), groups[3], groups[2], part)
+    return pa.pa_paged_attention_workspace_size(B, Hq, Hkv, D, case.max_len, bs, part)
+
+
+def measure_other_workload(pa, name, dev, flush_l2, stream, iters, peak):
+    """The decode-attention call of another named workload, timed like the
+    headline's roofline loop (graph replays, L2 flushed between them), with
+    its paging overhead against the contiguous-cache kernel."""
+    from paged_kv_cache_355_b200.workloads import make_case
+
+    case = make_case(name, device=dev)
+    w = case.workload
+    B, Hq, Hkv, D, bs = w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size
+    bt, lens = case.block_tables.to(dev), case.lengths.to(dev)
+    part = pa.pa_paged_attention_partition_size(B, Hq, Hkv, D, case.max_len, bs)
+    groups = prefix_groups(pa, case, dev)
+    ws = torch.empty(max(workspace_for(pa, case, part, groups), 16), dtype=torch.uint8, device=dev)
+    out = torch.empty(B, Hq, D, dtype=torch.float32, device=dev)
+    call = make_decode_call(pa, case, bt, lens, out, part, ws, groups)
+    call()
+    g, run = capture(call)
+    ms = timed_replays(run, iters, flush_l2, stream, warmup=3)
+    del g
+    kv = case.kv_bytes()
+    st = time_stats(ms)
+    res = {"workload": DESCRIPTIONS[name], "decode_call": "pa_paged_attention_decode_shared_prefix"
+           if groups is not None else "pa_paged_attention_decode", "partition_tokens": part,
+           "kv_bytes": kv, "decode_ms": st, "gbs": kv / (st["median"] * 1e-3) / 1e9}
+    res["frac"] = res["gbs"] / peak
+    ub = unique_kv_bytes(case)
+    if ub != kv:
+        res["unique_kv"] = {"bytes": ub, "gbs": ub / (st["median"] * 1e-3) / 1e9,
+                            "frac": ub / (st["median"] * 1e-3) / 1e9 / peak}
+    # the same kernel on a contiguous cache with the same lengths
+    L_pad = -(-case.max_len // 32) * 32
+    k_c = torch.empty(B, Hkv, L_pad, D, dtype=w.dtype, device=dev).normal_()
+    v_c = torch.empty_like(k_c).normal_()
+    out_c = torch.empty_like(out)
+    ws_c = torch.empty(max(pa.pa_paged_attention_workspace_size(B, Hq, Hkv, D, case.max_len, bs, part), 16),
+                       dtype=torch.uint8, device=dev)
+    contig = lambda: pa.pa_paged_attention_decode_contiguous(case.q, k_c, v_c, lens, case.max_len, case.scale, out_c,
+                                                             block_size=bs, partition_size=part, workspace=ws_c)
+    contig()
+    g, run = capture(contig)
+    ms_c = timed_replays(run, iters, flush_l2, stream, warmup=3)
+    del g
+    res["paging_overhead"] = st["median"] / statistics.median(ms_c) - 1.0
+    assert pa.pa_read_error_flag() == 0, f"device error during the {name} measurement"
+    del case, k_c, v_c, out_c, ws, ws_c
+    torch.cuda.empty_cache()
+    return res
 def run_ours(args):
     world, rank, local = dist_setup(args.gpus)
     import paged_kv_cache_355_b200 as pa
@@ -394,11 +529,13 @@ def run_ours(args):
     sid, pos = case.new_seq_ids.to(dev), case.new_positions.to(dev)
     pairs = case.cow_pairs.to(dev)
     part = args.partition or pa.pa_paged_attention_partition_size(B, Hq, Hkv, D, max_len, bs)
-    ws_bytes = pa.pa_paged_attention_workspace_size(B, Hq, Hkv, D, max_len, bs, part)
+    groups = prefix_groups(pa, case, dev)
+    ws_bytes = workspace_for(pa, case, part, groups)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     clean = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     plain_decode = pairs.numel() == 0 and case.new_seq_ids.numel() == B
+    peak, peak_kind = measured_hbm_peak()
 
     def cache_part():
         if pairs.numel():
@@ -410,9 +547,7 @@ def run_ours(args):
             pa.pa_slot_mapping(bt, sid, pos, bs, slots)
             pa.pa_reshape_and_cache(case.k_new, case.v_new, case.k_pool, case.v_pool, slots)
 
-    def decode_part():
-        pa.pa_paged_attention_decode(case.q, case.k_pool, case.v_pool, bt, lens, max_len, case.scale, out,
-                                     partition_size=part, workspace=ws)
+    decode_part = make_decode_call(pa, case, bt, lens, out, part, ws, groups)
 
     def step():
         if plain_decode and w.dtype == torch.bfloat16:
@@ -433,7 +568,7 @@ def run_ours(args):
 
     max_splits = -(-max(max_len, 1) // part)
     cache_launches = (1 if pairs.numel() else 0) + (1 if plain_decode else 2)
-    decode_launches = 1 + (1 if max_splits > 1 else 0)
+    decode_launches = (3 if groups is not None else 1 + (1 if max_splits > 1 else 0))
     step_launches = decode_launches + (0 if plain_decode and w.dtype == torch.bfloat16 else cache_launches)
 
     # ---- device-resident timed region
@@ -441,28 +576,24 @@ def run_ours(args):
     # engine runs its decode step: Python's launch overhead stays out of the
     # device timeline and the kernels' programmatic launches overlap each
     # kernel's start with the previous one's drain.  The decode call alone is
-    # captured into a second graph and timed the same way, for the roofline.
+    # captured into a second graph and timed the same way (at least 100
+    # replays), for the roofline; then the read-ceiling probe.
     for _ in range(args.warmup):
         flush_l2()
         step()
     torch.cuda.synchronize()
-    graphs = None
-    try:
-        g_step, g_decode = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_step):
-            step()
-        with torch.cuda.graph(g_decode):
-            decode_part()
-        torch.cuda.synchronize()
-        graphs = (g_step, g_decode)
-        run_step, run_decode = g_step.replay, g_decode.replay
-        for _ in range(2):
-            run_step()
-            run_decode()
-    except Exception as exc:  # capture unavailable: time the direct calls
-        print(f"bench: CUDA graph capture failed ({exc}); timing direct calls", file=sys.stderr)
-        run_step, run_decode = step, decode_part
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    g_step, run_step = capture(step)
+    g_decode, run_decode = capture(decode_part)
+    graphs = g_step is not None and g_decode is not None
+    for _ in range(2):
+        run_step()
+        run_decode()
+    n_dec = max(args.steps, ROOFLINE_MIN_ITERS)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    ev_dec = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_dec)]
+    probe_buf = torch.zeros(PROBE_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        pa.pa_hbm_read_probe(probe_buf)
     torch.cuda.synchronize()
     barrier(world)
     with ClockSampler(torch.cuda.current_device()) as clocks:
@@ -474,19 +605,22 @@ def run_ours(args):
             ev[i][0].record(stream)
             run_step()
             ev[i][1].record(stream)
-        for i in range(args.steps):
+        for i in range(n_dec):
             flush_l2()
-            ev[i][2].record(stream)
+            ev_dec[i][0].record(stream)
             run_decode()
-            ev[i][3].record(stream)
+            ev_dec[i][1].record(stream)
         torch.cuda.synchronize()
         barrier(world)
         t_wall = time.perf_counter() - t_wall
+        probe_ms = timed_replays(lambda: pa.pa_hbm_read_probe(probe_buf), 20, flush_l2, stream)
     step_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    dec_ms = [e[2].elapsed_time(e[3]) for e in ev]
+    dec_ms = [e[0].elapsed_time(e[1]) for e in ev_dec]
     ms_step = max_over_ranks(sum(step_ms) / len(step_ms), world)
     ms_dec = max_over_ranks(sum(dec_ms) / len(dec_ms), world)
     assert pa.pa_read_error_flag() == 0, "device error during the timed steps"
+    del probe_buf
+    read_ceiling = PROBE_BYTES / (statistics.median(probe_ms) * 1e-3) / 1e9
 
     # ---- the step's cache kernels alone (slot mapping, cache write, copy-on-write
     # copies), captured and timed the same way; their algorithmic bytes: each new
@@ -496,25 +630,10 @@ def run_ours(args):
     n_new = case.new_seq_ids.numel()
     cache_bytes = (n_new * Hkv * D * elt * 2 * 2 + pairs.shape[0] * Hkv * bs * D * elt * 2 * 2
                    + n_new * 8 * (1 if plain_decode else 2))
-    run_cache_only = cache_part
-    if graphs is not None:
-        g_cache = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_cache):
-            cache_part()
-        run_cache_only = g_cache.replay
-    cache_ev = []
-    for i in range(args.warmup + min(args.steps, 200)):
-        flush_l2()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        run_cache_only()
-        e1.record(stream)
-        if i >= args.warmup:
-            cache_ev.append((e0, e1))
-    torch.cuda.synchronize()
-    ms_cache = max_over_ranks(sum(a.elapsed_time(b_) for a, b_ in cache_ev) / len(cache_ev), world)
-    if graphs is not None:
-        del g_cache
+    g_cache, run_cache_only = capture(cache_part)
+    cache_ms = timed_replays(run_cache_only, min(args.steps, 200), flush_l2, stream, warmup=args.warmup)
+    ms_cache = max_over_ranks(sum(cache_ms) / len(cache_ms), world)
+    del g_cache
 
     # ---- contiguous-cache variant of the same kernel on the same lengths (paging overhead),
     # timed the same way (graph replay)
@@ -522,32 +641,18 @@ def run_ours(args):
     k_c = torch.empty(B, Hkv, L_pad, D, dtype=w.dtype, device=dev).normal_()
     v_c = torch.empty_like(k_c).normal_()
     out_c = torch.empty_like(out)
+    ws_c = torch.empty(max(pa.pa_paged_attention_workspace_size(B, Hq, Hkv, D, max_len, bs, part), 16),
+                       dtype=torch.uint8, device=dev)
     contig = lambda: pa.pa_paged_attention_decode_contiguous(case.q, k_c, v_c, lens, max_len, case.scale, out_c,
-                                                             block_size=bs, partition_size=part, workspace=ws)
+                                                             block_size=bs, partition_size=part, workspace=ws_c)
     contig()
     torch.cuda.synchronize()
-    run_contig = contig
-    if graphs is not None:
-        g_contig = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_contig):
-            contig()
-        run_contig = g_contig.replay
-    contig_ms = []
-    for i in range(args.warmup + min(args.steps, 200)):
-        flush_l2()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        run_contig()
-        e1.record(stream)
-        if i >= args.warmup:
-            contig_ms.append((e0, e1))
-    torch.cuda.synchronize()
-    ms_contig = max_over_ranks(sum(a.elapsed_time(b_) for a, b_ in contig_ms) / len(contig_ms), world)
+    g_contig, run_contig = capture(contig)
+    contig_ms = timed_replays(run_contig, min(n_dec, 200), flush_l2, stream, warmup=args.warmup)
+    ms_contig = max_over_ranks(sum(contig_ms) / len(contig_ms), world)
     paged_med = statistics.median(dec_ms)
-    contig_med = statistics.median(a.elapsed_time(b_) for a, b_ in contig_ms)
-    del k_c, v_c, run_contig
-    if graphs is not None:
-        del g_contig
+    contig_med = statistics.median(contig_ms)
+    del k_c, v_c, run_contig, g_contig
 
     # ---- end to end through the public API with host buffers
     # The step's inputs (q, new K/V, block tables, lengths) sit in one pinned
@@ -575,15 +680,8 @@ def run_ours(args):
     h_out = torch.empty(B, Hq, D, dtype=torch.float32).pin_memory()
     h2d = total
     d2h = h_out.numel() * h_out.element_size()
-    e2e_ev = []
-    for i in range(args.warmup + args.steps):
-        flush_l2()
-        # a 1 ms spin on the device before the start event: the host enqueues
-        # the whole step (copies, API calls, read-back) while it runs, so the
-        # events time the step's device work, not Python's issue rate
-        torch.cuda._sleep(SPIN_CYCLES)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
+
+    def e2e_step():
         d_pack.copy_(h_pack, non_blocking=True)
         if plain_decode:
             pa.decode_step(d_q, d_kn, d_vn, case.k_pool, case.v_pool, d_bt, d_lens, max_len, case.scale, out, slots,
@@ -593,14 +691,55 @@ def run_ours(args):
                 pa.pa_copy_blocks(case.k_pool, case.v_pool, d_pairs)
             pa.pa_slot_mapping(d_bt, d_sid, d_pos, bs, slots)
             pa.pa_reshape_and_cache(d_kn, d_vn, case.k_pool, case.v_pool, slots)
-            pa.pa_paged_attention_decode(d_q, case.k_pool, case.v_pool, d_bt, d_lens, max_len, case.scale, out,
-                                         partition_size=part, workspace=ws)
+            if groups is not None:
+                pa.pa_paged_attention_decode_shared_prefix(d_q, case.k_pool, case.v_pool, d_bt, d_lens, max_len,
+                                                           case.scale, out, groups[0], groups[1], groups[2],
+                                                           groups[3], partition_size=part, workspace=ws)
+            else:
+                pa.pa_paged_attention_decode(d_q, case.k_pool, case.v_pool, d_bt, d_lens, max_len, case.scale, out,
+                                             partition_size=part, workspace=ws)
         h_out.copy_(out, non_blocking=True)
+
+    e2e_ev = []
+    for i in range(args.warmup + args.steps):
+        flush_l2()
+        # a 1 ms spin on the device before the start event: the host enqueues
+        # the whole step (copies, API calls, read-back) while it runs, so the
+        # events time the step's device work, not Python's issue rate
+        torch.cuda._sleep(SPIN_CYCLES)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        e2e_step()
         e1.record(stream)
         if i >= args.warmup:
             e2e_ev.append((e0, e1))
     torch.cuda.synchronize()
-    ms_e2e = max_over_ranks(sum(a.elapsed_time(b_) for a, b_ in e2e_ev) / len(e2e_ev), world)
+    e2e_ms = [a.elapsed_time(b_) for a, b_ in e2e_ev]
+    ms_e2e = max_over_ranks(sum(e2e_ms) / len(e2e_ms), world)
+    # the same step as a caller without graphs or a device spin sees it: host
+    # wall time from the first copy's issue to the read-back's completion
+    host_ms = []
+    for i in range(args.warmup + args.steps):
+        flush_l2()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        e2e_step()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            host_ms.append((time.perf_counter() - t0) * 1e3)
+    ms_host = max_over_ranks(sum(host_ms) / len(host_ms), world)
+    assert pa.pa_read_error_flag() == 0, "device error during the end-to-end steps"
+
+    # ---- the other decode workloads, each timed like the roofline loop above
+    # (one GPU, default headline run only)
+    others = None
+    if world == 1 and not args.no_other_workloads and args.batch is None and args.workload == "llama7b":
+        torch.cuda.empty_cache()
+        others = {}
+        with ClockSampler(torch.cuda.current_device()) as oclocks:
+            for name in OTHER_WORKLOADS:
+                others[name] = measure_other_workload(pa, name, dev, flush_l2, stream, ROOFLINE_MIN_ITERS, peak)
+        others["clocks"] = oclocks.summary()
 
     # ---- CPU oracle on this machine's host cores (rank 0, one GPU only)
     cpu = None
@@ -609,12 +748,12 @@ def run_ours(args):
 
     if rank != 0:
         return
-    peak, peak_kind = measured_hbm_peak()
     achieved = kv_bytes / (ms_dec * 1e-3) / 1e9
     value = world * kv_bytes / (ms_step * 1e-3) / 1e9
     # the committed ncu record covers the workloads at their own batch only
     traffic = dram_traffic(args.workload) if args.batch in (None, WORKLOADS[args.workload].batch) else None
     clk = clocks.summary()
+    st_step, st_dec = time_stats(step_ms), time_stats(dec_ms)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -627,15 +766,23 @@ def run_ours(args):
                          "step also exceeds the 126 MB L2",
                    "parallelism": f"{world} independent replicas (sequences sharded, no collective)"},
         "tokens_per_s": world * B / (ms_step * 1e-3),
+        "step_ms": st_step,
+        "decode_attention_ms": st_dec,
+        "decode_gbs_median": kv_bytes / (st_dec["median"] * 1e-3) / 1e9,
         "unique_kv": ({"bytes_per_step": unique_bytes,
                        "step_gbs": world * unique_bytes / (ms_step * 1e-3) / 1e9,
                        "decode_gbs": unique_bytes / (ms_dec * 1e-3) / 1e9,
                        "note": "distinct pool slots read; shared prompt blocks counted once"}
                       if unique_bytes != kv_bytes else None),
-        "decode_attention_ms": ms_dec,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": traffic, "kernel": "pa_paged_attention_decode (pass 1 + split merge)",
-                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)"},
+                     "traffic": traffic,
+                     "kernel": ("pa_paged_attention_decode_shared_prefix (prefix pass + suffix pass + merge)"
+                                if groups is not None else "pa_paged_attention_decode (pass 1 + split merge)"),
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)",
+                     "read_ceiling_gbs": read_ceiling, "frac_of_read_ceiling": achieved / read_ceiling,
+                     "read_ceiling_source": f"pa_hbm_read_probe: a {PROBE_BYTES >> 30} GiB buffer streamed through "
+                                            "shared memory by bulk TMA copies, median of 20 launches, this run",
+                     "timed_iterations": n_dec},
         "cache_part": {"kernels": (["pa_copy_blocks"] if pairs.numel() else [])
                        + (["pa_reshape_and_cache_decode"] if plain_decode
                           else ["pa_slot_mapping", "pa_reshape_and_cache"]),
@@ -647,13 +794,18 @@ def run_ours(args):
         "paging_overhead": {"paged_ms_median": paged_med, "contiguous_ms_median": contig_med,
                             "overhead": paged_med / contig_med - 1.0, "contiguous_ms_mean_max_ranks": ms_contig},
         "e2e": {"value": world * kv_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
+                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e, "ms_stats": time_stats(e2e_ms),
+                "host_wall_ms_per_step": ms_host, "host_wall_ms_stats": time_stats(host_ms),
+                "host_wall_gbs": world * kv_bytes / (ms_host * 1e-3) / 1e9,
                 "timing": "device time from before the H2D copies to after the D2H read-back, direct API calls "
-                          "(no graph); a device spin ahead of each step keeps host issue latency out"},
+                          "(no graph); a device spin ahead of each step keeps host issue latency out. "
+                          "host_wall: the same calls timed by the host clock from the first issue to a "
+                          "synchronize after the read-back, with no spin (what a caller without graphs waits)"},
+        "other_workloads": others,
         "gpu_launches": step_launches * args.steps,
-        "gpu_launches_decode_roofline_loop": decode_launches * args.steps,
-        "timing": ("K replays of the step's CUDA graph (value), then K replays of the decode call's graph "
-                   "(roofline), each bracketed by events" if graphs is not None else "direct calls"),
+        "gpu_launches_decode_roofline_loop": decode_launches * n_dec,
+        "timing": ("K replays of the step's CUDA graph (value), then max(K, 100) replays of the decode call's "
+                   "graph (roofline), each bracketed by events" if graphs else "direct calls"),
         "clocks": clk,
         "wall_s_timed_region": t_wall,
         "cpu_baseline": cpu,

@@ -80,7 +80,10 @@ const char* pa_version(void);
  * pa_read_error_flag -- synchronise `stream`, then return the first
  * device-side error recorded by any kernel of this library on the current
  * device since the previous call (PA_OK if none), and clear it.  Returns
- * PA_ERR_CUDA if the synchronisation itself fails.
+ * PA_ERR_CUDA if the synchronisation itself fails.  The error word's device
+ * address is looked up once per device and cached, which assumes the
+ * device's primary context lives until the process exits (no
+ * cudaDeviceReset between calls into the library).
  */
 int pa_read_error_flag(void* stream);
 
@@ -94,6 +97,18 @@ int pa_read_error_flag(void* stream);
  * Read the result with pa_read_error_flag.
  */
 int pa_selftest_wait_timeout(uint32_t limit_us, void* stream);
+
+/*
+ * pa_hbm_read_probe -- read `bytes` of device memory at `buffer` as one
+ * stream and discard them: the HBM read ceiling against which paged decode
+ * attention, itself a read stream of K/V bytes, is judged.  No counterpart in
+ * the pages: a measurement aid.  Each CTA (3 per SM) moves a grid-strided
+ * series of 16 KB chunks of the buffer into a 4-stage shared-memory ring with
+ * bulk TMA copies and never looks at them; nothing is written to global
+ * memory.  buffer: device pointer, 16-byte aligned; bytes: a multiple of 16
+ * (0 does nothing); else PA_ERR_INVALID_ARG.  Waits are bounded as everywhere.
+ */
+int pa_hbm_read_probe(const void* buffer, size_t bytes, void* stream);
 
 /*
  * pa_slot_mapping -- slot of each new token ([P3] "Detail": logical block
@@ -278,6 +293,67 @@ int pa_paged_attention_decode_append(const void* q, const void* key, const void*
                                      int64_t* slot_mapping, void* stream);
 
 /*
+ * pa_paged_attention_shared_prefix_workspace_size -- bytes of scratch that
+ * pa_paged_attention_decode_shared_prefix needs for these sizes (always > 0:
+ * the prefix pass's partial results and each sequence's prefix length).
+ * num_groups >= 1, max_group_size >= 1, 0 <= max_prefix_len <=
+ * max_context_len; partition_size as for pa_paged_attention_decode.
+ */
+int pa_paged_attention_shared_prefix_workspace_size(int batch, int num_q_heads, int num_kv_heads,
+                                                    int head_dim, int max_context_len,
+                                                    int block_size, int num_groups,
+                                                    int max_group_size, int max_prefix_len,
+                                                    int partition_size, size_t* workspace_bytes);
+
+/*
+ * pa_paged_attention_decode_shared_prefix -- pa_paged_attention_decode for a
+ * batch whose sequences come in groups that share a prompt: parallel samples
+ * hold one copy of the prompt's blocks, shared by reference count
+ * ([P1] "Key takeaways": samples share a prompt without copying it;
+ * [P2] "Key terms in this lesson", Reference count and Copy-on-write).  The
+ * result is the same attention as pa_paged_attention_decode over the same
+ * tables and lengths (within rounding: the softmax is split at different
+ * points), but each shared block is read from memory once per group instead
+ * of once per member: a prefix pass attends the group's shared tokens for
+ * all its members' query heads at once (tensor cores, queries stacked on the
+ * MMA's M side), pass 1 attends each member's own tokens after the prefix,
+ * and the merge pass combines the two.
+ *   group_starts       int32 [num_groups + 1], device: group g is sequences
+ *                      group_starts[g] .. group_starts[g + 1] - 1, with
+ *                      group_starts[0] = 0, non-decreasing,
+ *                      group_starts[num_groups] = batch (the groups cover the
+ *                      batch; a sequence that shares nothing is a group of
+ *                      one with prefix 0)
+ *   group_prefix_lens  int32 [num_groups], device: tokens 0 .. P_g - 1 of
+ *                      every member of group g are the same physical slots:
+ *                      P_g is a multiple of block_size, the first P_g /
+ *                      block_size entries of every member's table are equal,
+ *                      and P_g <= context_lens[b] for every member
+ *   max_group_size     host-side upper bound of the group sizes
+ *   max_prefix_len     host-side upper bound of the P_g (<= max_context_len)
+ *   workspace          pa_paged_attention_shared_prefix_workspace_size bytes
+ * Other arguments as for pa_paged_attention_decode.  bf16 only (kv_dtype
+ * PA_BF16, else PA_ERR_UNSUPPORTED).  A group whose description breaks these
+ * rules (a prefix that is not whole blocks, longer than a member or than
+ * max_prefix_len, a group larger than max_group_size, starts out of order)
+ * records PA_ERR_BAD_BLOCK_ID and is attended without sharing (prefix 0);
+ * groups that do not cover the batch record it too, and the uncovered
+ * sequences' outputs are unspecified.  Equal table entries are the caller's
+ * precondition and are not checked.
+ */
+int pa_paged_attention_decode_shared_prefix(const void* q, const void* k_pool, const void* v_pool,
+                                            const int32_t* block_tables, int max_blocks_per_seq,
+                                            const int32_t* context_lens, int max_context_len,
+                                            float scale, int block_size, void* out, int out_dtype,
+                                            int batch, int num_q_heads, int num_kv_heads,
+                                            int head_dim, int64_t num_blocks, int kv_dtype,
+                                            const int32_t* group_starts,
+                                            const int32_t* group_prefix_lens, int num_groups,
+                                            int max_group_size, int max_prefix_len,
+                                            int partition_size, void* workspace,
+                                            size_t workspace_bytes, void* stream);
+
+/*
  * pa_paged_attention_prefill -- causal attention for several new query
  * tokens per sequence over the paged cache (chunked prefill, or speculative
  * tokens): the multi-query form of pa_paged_attention_decode, reading K and V
@@ -403,7 +479,12 @@ int pa_bm_free_list(const pa_block_manager* bm, int64_t* out, int64_t cap, int64
  *    launching; a larger partition_size needs less scratch.
  *  * Set-up: the first call on each device looks up the array's device
  *    address (cudaGetSymbolAddress, with that device current) and caches it;
- *    make that first call before any stream capture on the device.
+ *    make that first call before any stream capture on the device.  The
+ *    cached address assumes the device's primary CUDA context lives as long
+ *    as the process: after cudaDeviceReset (or any teardown of that context)
+ *    the library must not be called again in the same process, since the
+ *    cached address (and the library's cached error-word address, see
+ *    pa_read_error_flag) would point into the destroyed context.
  *  * Sharing: every call uses the same array, which keeps the previous call's
  *    contents (nothing in it needs to start at zero).  Calls that overlap on
  *    the GPU, for example on two streams, race on it; calls ordered on one

@@ -17,7 +17,8 @@ _BINDING_NAMES = (
     "pa_paged_attention_workspace_size", "pa_read_error_flag", "pa_reshape_and_cache", "pa_slot_mapping",
     "pa_status_string", "pa_version", "pa_paged_attention_decode_static_scratch", "STATIC_SCRATCH_BYTES",
     "pa_paged_attention_prefill", "pa_reshape_and_cache_decode", "pa_selftest_wait_timeout",
-    "pa_paged_attention_decode_append",
+    "pa_paged_attention_decode_append", "pa_hbm_read_probe", "pa_paged_attention_decode_shared_prefix",
+    "pa_paged_attention_shared_prefix_workspace_size",
 )
 __all__ = list(_BINDING_NAMES) + ["decode_step"]
 

@@ -34,6 +34,7 @@ _SIGS = {
     "pa_version": ([], ctypes.c_char_p),
     "pa_read_error_flag": ([_P], _I),
     "pa_selftest_wait_timeout": ([ctypes.c_uint32, _P], _I),
+    "pa_hbm_read_probe": ([_P, _SZ, _P], _I),
     "pa_slot_mapping": ([_P, _I, _I, _P, _P, _I64, _I, _P, _P], _I),
     "pa_decode_slot_mapping": ([_P, _I, _P, _I, _I, _P, _P], _I),
     "pa_reshape_and_cache": ([_P, _P, _P, _P, _P, _I64, _I, _I, _I, _I64, _I, _P], _I),
@@ -46,6 +47,10 @@ _SIGS = {
                                    _SZ, _P], _I),
     "pa_paged_attention_decode_append": ([_P, _P, _P, _P, _P, _P, _I, _P, _I, _F, _I, _P, _I, _I, _I, _I, _I, _I64, _I,
                                           _I, _P, _SZ, _P, _P], _I),
+    "pa_paged_attention_shared_prefix_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, _I, _I, _I,
+                                                        ctypes.POINTER(_SZ)], _I),
+    "pa_paged_attention_decode_shared_prefix": ([_P, _P, _P, _P, _I, _P, _I, _F, _I, _P, _I, _I, _I, _I, _I, _I64,
+                                                 _I, _P, _P, _I, _I, _I, _I, _P, _SZ, _P], _I),
     "pa_paged_attention_decode_contiguous": ([_P, _P, _P, _I64, _P, _I, _F, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P,
                                               _SZ, _P], _I),
     "pa_paged_attention_prefill": ([_P, _P, _P, _P, _I, _P, _P, _I, _F, _I, _P, _I, _I, _I, _I, _I, _I64, _I64, _I,
@@ -123,6 +128,13 @@ def pa_read_error_flag(stream=None) -> int:
 
 def pa_selftest_wait_timeout(limit_us: int, stream=None) -> None:
     _check("pa_selftest_wait_timeout", _lib.pa_selftest_wait_timeout(limit_us, _stream(stream)))
+
+
+def pa_hbm_read_probe(buffer, stream=None) -> None:
+    """Stream every byte of a CUDA tensor through shared memory and discard
+    it (the device's HBM read ceiling; nothing is written)."""
+    nbytes = buffer.numel() * buffer.element_size()
+    _check("pa_hbm_read_probe", _lib.pa_hbm_read_probe(_dev(buffer, "buffer"), nbytes, _stream(stream)))
 
 
 def pa_slot_mapping(block_tables, seq_ids, positions, block_size: int, slot_mapping, stream=None) -> None:
@@ -283,6 +295,45 @@ def pa_paged_attention_decode_append(q, key, value, k_pool, v_pool, block_tables
         _dev(block_tables, "block_tables", torch.int32), MBS, _dev(context_lens, "context_lens", torch.int32),
         int(max_context_len), float(scale), bs, _dev(out, "out"), _kv_dtype(out), B, Hq, Hkv, D, NB, dt,
         partition_size, ws, ws_bytes, slots, _stream(stream)))
+
+
+def pa_paged_attention_shared_prefix_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                                                    block_size, num_groups, max_group_size, max_prefix_len,
+                                                    partition_size=0) -> int:
+    n = ctypes.c_size_t(0)
+    _check("pa_paged_attention_shared_prefix_workspace_size", _lib.pa_paged_attention_shared_prefix_workspace_size(
+        batch, num_q_heads, num_kv_heads, head_dim, int(max_context_len), block_size, num_groups, max_group_size,
+        int(max_prefix_len), partition_size, ctypes.byref(n)))
+    return n.value
+
+
+def pa_paged_attention_decode_shared_prefix(q, k_pool, v_pool, block_tables, context_lens, max_context_len: int,
+                                            scale: float, out, group_starts, group_prefix_lens, max_prefix_len: int,
+                                            max_group_size: int, partition_size: int = 0, workspace=None,
+                                            stream=None) -> None:
+    """Decode attention for groups of consecutive sequences that share their
+    first group_prefix_lens[g] tokens (whole blocks, equal table entries):
+    sequences group_starts[g] .. group_starts[g + 1] - 1 form group g
+    (int32 device tensors of num_groups + 1 and num_groups entries)."""
+    B, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_pool.shape
+    if D2 != D or v_pool.shape != k_pool.shape or tuple(out.shape) != (B, Hq, D):
+        raise ValueError("q / pool / out shapes disagree")
+    G = group_prefix_lens.numel()
+    if group_starts.numel() != G + 1:
+        raise ValueError("group_starts needs num_groups + 1 entries")
+    dt = _kv_dtype(q)
+    _dev(k_pool, "k_pool", q.dtype)
+    _dev(v_pool, "v_pool", q.dtype)
+    need = pa_paged_attention_shared_prefix_workspace_size(B, Hq, Hkv, D, max_context_len, bs, G, max_group_size,
+                                                           max_prefix_len, partition_size)
+    ws, ws_bytes = _workspace(workspace, need, q.device, stream)
+    _check("pa_paged_attention_decode_shared_prefix", _lib.pa_paged_attention_decode_shared_prefix(
+        _dev(q, "q"), k_pool.data_ptr(), v_pool.data_ptr(), _dev(block_tables, "block_tables", torch.int32),
+        block_tables.shape[1], _dev(context_lens, "context_lens", torch.int32), int(max_context_len), float(scale), bs,
+        _dev(out, "out"), _kv_dtype(out), B, Hq, Hkv, D, NB, dt, _dev(group_starts, "group_starts", torch.int32),
+        _dev(group_prefix_lens, "group_prefix_lens", torch.int32), G, int(max_group_size), int(max_prefix_len),
+        partition_size, ws, ws_bytes, _stream(stream)))
 
 
 def pa_paged_attention_decode_contiguous(q, k_c, v_c, context_lens, max_context_len: int, scale: float, out,

@@ -27,6 +27,8 @@ int current_device() {
 }
 }  // namespace
 
+// Cached per device: valid while the device's primary context lives (the
+// library is not used across a cudaDeviceReset).
 int* error_word_ptr() {
     const int dev = current_device();
     if (dev < 0) return nullptr;

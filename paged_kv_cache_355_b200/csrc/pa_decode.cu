@@ -112,6 +112,21 @@ struct DecodeParams {
     const void* v_new;
     int64_t* slots;
     int append;
+    // shared-prefix decode: sequences [group_starts[g], group_starts[g + 1])
+    // share their first group_prefix[g] tokens (whole blocks, the same
+    // physical ids in every member's table).  The prefix pass attends each
+    // group's shared tokens once for all its members' queries and stores each
+    // member's prefix length in seq_prefix; pass 1 then covers only tokens
+    // [seq_prefix[b], L) of sequence b.  Partial-result slot s of a row holds
+    // prefix split s for s < ceil(prefix / prefix_partition), then the
+    // suffix splits.  seq_prefix == nullptr: no sharing.
+    const int32_t* group_starts;
+    const int32_t* group_prefix;
+    int32_t* seq_prefix;
+    int num_groups;
+    int max_group;
+    int max_prefix;
+    int prefix_partition;
 };
 
 template <typename T>
@@ -151,6 +166,28 @@ __device__ __forceinline__ int clamp_len(const DecodeParams& p, int b, bool repo
         L = L < 0 ? 0 : (int)p.max_len;
     }
     return L;
+}
+
+// Leading tokens of sequence b that the prefix pass covered (0 without
+// shared prefixes), clamped to [0, min(L, max_prefix)] and to whole blocks, so
+// that a value left unwritten under a violated precondition can never send
+// pass 1 or the merge outside the table or the partial-result slots.
+__device__ __forceinline__ int seq_prefix_len(const DecodeParams& p, int b, int L) {
+    if (!p.seq_prefix) return 0;
+    int v = p.seq_prefix[b];
+    const int hi = L < p.max_prefix ? L : p.max_prefix;
+    v = v < 0 ? 0 : (v > hi ? hi : v);
+    return v - v % p.block_size;
+}
+
+// Partial-result slots of sequence b (prefix splits, then suffix splits; at
+// least one suffix split, empty when the prefix covers the whole sequence),
+// and the number of prefix splits before the suffix's first slot.
+__device__ __forceinline__ int row_splits(const DecodeParams& p, int L, int pre, int* prefix_splits) {
+    const int sp = pre > 0 ? (pre + p.prefix_partition - 1) / p.prefix_partition : 0;
+    const int nsuf = L > pre ? (L - pre + p.partition - 1) / p.partition : 1;
+    *prefix_splits = sp;
+    return sp + nsuf;
 }
 
 __device__ __forceinline__ void store_out(const DecodeParams& p, int64_t idx, float v) {
@@ -222,6 +259,7 @@ __device__ __forceinline__ int schedule_sequence(const DecodeParams& p, uint8_t*
     for (int b = tid; b < p.batch; b += blockDim.x) {
         int L = p.context_lens[b];
         L = L < 0 ? 0 : ((int64_t)L > p.max_len ? (int)p.max_len : L);
+        L -= seq_prefix_len(p, b, L);  // the tokens this pass reads
         int k = (int)(((int64_t)L * 64) / (p.max_len + 1));
         k = 63 - (k > 63 ? 63 : k);  // longer sequences get lower keys
         key[b] = (uint8_t)k;
@@ -560,12 +598,21 @@ __global__ void __launch_bounds__(kDecodeThreads)
     const int G = p.num_q_heads / p.num_kv_heads;
 
     const int L = clamp_len(p, b, threadIdx.x == 0 && split == 0 && kvh == 0);
-    if (p.append && L == 0 && split == 0 && kvh == 0 && threadIdx.x == 0 && p.slots) p.slots[b] = -1;
-    const int tok_begin = split * p.partition;
+    // A length beyond max_context_len is clamped for the attention (and
+    // flagged), but the folded write still goes to the slot of the length as
+    // given, where pa_reshape_and_cache_decode puts it: split 0 writes it
+    // directly, outside the (clamped) range any CTA of this launch reads.
+    const bool overflow = p.append && p.context_lens[b] > p.max_len;
+    if (p.append && !overflow && L == 0 && split == 0 && kvh == 0 && threadIdx.x == 0 && p.slots) p.slots[b] = -1;
+    // with shared prefixes this pass covers the tokens after the sequence's
+    // prefix, and its splits' partial results follow the prefix splits' slots
+    const int pre = seq_prefix_len(p, b, L);
+    const int tok_begin = pre + split * p.partition;
     if (split > 0 && tok_begin >= L) return;
     const int ntok = max(0, min(L, tok_begin + p.partition) - tok_begin);
     const int nstage = (ntok + kStageTokens - 1) / kStageTokens;
-    const int num_splits_b = L > 0 ? (L + p.partition - 1) / p.partition : 1;
+    int prefix_splits;
+    const int num_splits_b = row_splits(p, L, pre, &prefix_splits);
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -582,6 +629,22 @@ __global__ void __launch_bounds__(kDecodeThreads)
         for (int i = threadIdx.x; i < nblk; i += blockDim.x) tbl[i] = row[i];
     }
     __syncthreads();
+
+    if (overflow && split == 0 && warp == 1) {
+        const int pos = p.context_lens[b] - 1;
+        int32_t phys = -1;
+        if (pos / p.block_size < p.max_blocks_per_seq)
+            phys = p.block_tables[(int64_t)b * p.max_blocks_per_seq + pos / p.block_size];
+        if (phys >= 0 && phys < p.num_blocks && lane < D / 8) {
+            const int64_t src = ((int64_t)b * p.num_kv_heads + kvh) * (D / 8) + lane;
+            const int64_t dst =
+                (((int64_t)phys * p.num_kv_heads + kvh) * p.block_size + pos % p.block_size) * (D / 8) + lane;
+            static_cast<uint4*>(const_cast<void*>(p.k))[dst] = static_cast<const uint4*>(p.k_new)[src];
+            static_cast<uint4*>(const_cast<void*>(p.v))[dst] = static_cast<const uint4*>(p.v_new)[src];
+        }
+        if (lane == 0 && kvh == 0 && p.slots)
+            p.slots[b] = phys >= 0 ? (int64_t)phys * p.block_size + pos % p.block_size : -1;
+    }
 
     const int g = lane >> 2;  // fragment row group
     const int t = lane & 3;   // fragment column pair
@@ -677,7 +740,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
         // a folded-in cache write: the warp that takes the last stage of the
         // sequence's last split loads the new K and V rows now, so their
         // latency is hidden behind the stream (lane c holds 16-byte chunk c)
-        const bool appends = p.append && nstage > 0 && split == num_splits_b - 1 &&
+        const bool appends = p.append && !overflow && nstage > 0 && split == num_splits_b - prefix_splits - 1 &&
                              (nstage - 1) % kConsumerWarps == cw;
         uint4 new_k = make_uint4(0u, 0u, 0u, 0u), new_v = new_k;
         if (appends && lane < D / 8) {
@@ -706,6 +769,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
                     *reinterpret_cast<uint4*>(vstage + (rem >> 3) * SLAB_BYTES + row * 128 + (rem & 7) * 16) =
                         make_uint4(0u, 0u, 0u, 0u);
                 }
+                fence_proxy_async_smem();  // the slot is refilled by TMA later
                 __syncwarp();
             }
             if (appends && j == nstage - 1) {
@@ -729,6 +793,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
                 }
                 if (lane == 0 && kvh == 0 && p.slots)
                     p.slots[b] = phys >= 0 ? (int64_t)phys * p.block_size + pos % p.block_size : -1;
+                fence_proxy_async_smem();
                 __syncwarp();
             }
             // S^T = K . Q^T : two 16-token M tiles
@@ -878,7 +943,331 @@ __global__ void __launch_bounds__(kDecodeThreads)
         }
     }
     __syncthreads();
-    merge_warps_and_store(p, sm_o, sm_m, sm_l, G, D, b, kvh, split, num_splits_b);
+    merge_warps_and_store(p, sm_o, sm_m, sm_l, G, D, b, kvh, prefix_splits + split, num_splits_b);
+}
+
+// ---------------------------------------------------------------------------
+// Shared-prefix pass (bf16, tensor cores).
+//
+// Parallel samples of one prompt share the prompt's blocks by reference count
+// ("PagedAttention and KV memory management", "Key takeaways"; "Paged
+// Attention: OS-Inspired Memory Management for KV Caches", "Key terms in this
+// lesson", Reference count).  Per-sequence attention reads those blocks once
+// per sample.  This pass reads them once per group instead: a CTA owns
+// (prefix split, kv head x row chunk, group), streams the split's K/V tiles
+// through the same TMA ring as pass 1, and computes them against the queries
+// of every member of the group at once, so each shared K/V element in shared
+// memory is used by n * G query rows.
+//  * Query rows r = member * G + head are the M side of mma.sync m16n8k16:
+//        S[rows, tokens] = Q[rows, D] . K^T[D, tokens]
+//        O[rows, D]     += P[rows, tokens] . V[tokens, D]
+//    Consumer warp w owns rows 16 w .. 16 w + 15 of the CTA's chunk and reads
+//    every stage; P goes from the S accumulators straight into A fragments
+//    (the two layouts coincide), split into bf16 high and residual parts as
+//    in pass 1.  MT consumer warps cover 16 MT rows; larger groups take
+//    several row chunks (blockIdx.y / Hkv).
+//  * Each warp finishes its own rows: the normalised partial row and (m, l)
+//    go to the prefix split's slot for the merge pass.  CTA (0, 0, g) also
+//    checks the group's description and stores each member's prefix length
+//    in seq_prefix for pass 1 and the merge; a description that breaks the
+//    preconditions is flagged and its group falls back to prefix 0 (pass 1
+//    then covers the whole sequences).
+// ---------------------------------------------------------------------------
+template <int D, int MT>
+__global__ void __launch_bounds__(32 * (1 + MT))
+    decode_prefix_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
+                             const __grid_constant__ CUtensorMap tmv) {
+    constexpr int SLABS = D / 64;
+    constexpr int SLAB_BYTES = kStageTokens * 128;
+    constexpr int STAGE_BYTES = SLABS * SLAB_BYTES;
+    constexpr int KSTEPS = D / 16;
+    constexpr int NTD = D / 8;  // 8-column tiles of the output row
+    constexpr int ROWS = 16 * MT;
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + p.stages;
+    int32_t* tbl = reinterpret_cast<int32_t*>(empty + p.stages);
+    uint8_t* ring = smem + p.ring_offset + ((1024u - (smem_addr(smem) & 1023u)) & 1023u);
+    __shared__ int s_start, s_n, s_prefix, s_bad;
+
+    if (threadIdx.x == 0) {
+        prefetch_tmap(&tmk);
+        prefetch_tmap(&tmv);
+    }
+    griddep_wait();  // q, lengths, tables and the pool may come from the kernel before
+    griddep_launch_dependents();
+    const int split = blockIdx.x;
+    const int kvh = blockIdx.y % p.num_kv_heads;
+    const int chunk = blockIdx.y / p.num_kv_heads;
+    const int grp = blockIdx.z;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int G = p.num_q_heads / p.num_kv_heads;
+    const bool reporter = split == 0 && blockIdx.y == 0;
+
+    // the group's description; every CTA of the group reaches the same verdict
+    if (threadIdx.x == 0) {
+        const int s = p.group_starts[grp], e = p.group_starts[grp + 1], P = p.group_prefix[grp];
+        const bool ok = s >= 0 && e >= s && e <= p.batch && e - s <= p.max_group && P >= 0 && P <= p.max_prefix &&
+                        P % p.block_size == 0;
+        s_start = ok ? s : 0;
+        s_n = ok ? e - s : 0;
+        s_prefix = ok ? P : 0;
+        s_bad = !ok;
+        if (reporter && ((grp == 0 && s != 0) || (grp == p.num_groups - 1 && e != p.batch)))
+            record_error(p.err, PA_ERR_BAD_BLOCK_ID);  // the groups do not cover the batch
+    }
+    __syncthreads();
+    for (int m = threadIdx.x; m < s_n; m += blockDim.x)
+        if (clamp_len(p, s_start + m, false) < s_prefix) s_bad = 1;  // a member shorter than the prefix
+    __syncthreads();
+    const int n = s_n;
+    const int P = s_bad ? 0 : s_prefix;
+    if (reporter) {
+        if (threadIdx.x == 0 && s_bad) record_error(p.err, PA_ERR_BAD_BLOCK_ID);
+        for (int m = threadIdx.x; m < n; m += blockDim.x) p.seq_prefix[s_start + m] = P;
+    }
+    const int tok_begin = split * p.prefix_partition;
+    const int rows_total = n * G;
+    const int row0 = chunk * ROWS;
+    if (tok_begin >= P || row0 >= rows_total) return;  // uniform over the CTA, before any barrier
+    const int ntok = min(P, tok_begin + p.prefix_partition) - tok_begin;
+    const int nstage = (ntok + kStageTokens - 1) / kStageTokens;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], MT);
+        }
+        fence_barrier_init();
+    }
+    {
+        // the shared blocks, from the first member's table
+        const int first_blk = tok_begin / p.block_size;
+        const int nblk = (ntok + p.block_size - 1) / p.block_size;
+        const int32_t* row = p.block_tables + (int64_t)s_start * p.max_blocks_per_seq + first_blk;
+        for (int i = threadIdx.x; i < nblk; i += blockDim.x) tbl[i] = row[i];
+    }
+    __syncthreads();
+
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        const uint64_t policy = l2_policy_evict_first();
+        const int bs = p.block_size;
+        const int tiles = kStageTokens / bs;
+        const uint32_t tile_bytes = (uint32_t)(SLABS * bs * 128);
+        for (int j = 0; j < nstage; ++j) {
+            const int slot = j % p.stages;
+            if (j >= p.stages) {
+                int ok = 1;
+                if (lane == 0) ok = mbar_wait(&empty[slot], ((j / p.stages) - 1) & 1, p.err);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            }
+            uint8_t* kdst = ring + (size_t)slot * 2 * STAGE_BYTES;
+            uint8_t* vdst = kdst + STAGE_BYTES;
+            const int t0 = j * kStageTokens;
+            const int rows = min(kStageTokens, ntok - t0);
+            if (rows < kStageTokens) {
+                // every consumer reads this stage: the producer zeroes the V
+                // rows past the prefix (0-weight * stale NaN would be NaN)
+                const int nchunks = (kStageTokens - rows) * SLABS * 8;
+                for (int c = lane; c < nchunks; c += 32) {
+                    const int row = rows + c / (SLABS * 8);
+                    const int rem = c % (SLABS * 8);
+                    *reinterpret_cast<uint4*>(vdst + (rem >> 3) * SLAB_BYTES + row * 128 + (rem & 7) * 16) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+                fence_proxy_async_smem();
+            }
+            const int r = lane * bs;
+            int y = 0;
+            uint32_t nbytes = 0;
+            if (lane < tiles && r < rows) {
+                const int32_t phys = tbl[(t0 + r) / bs];
+                if (phys < 0 || phys >= p.num_blocks) {
+                    record_error(p.err, PA_ERR_BAD_BLOCK_ID);
+                } else {
+                    nbytes = tile_bytes;
+                    y = (phys * p.num_kv_heads + kvh) * bs;
+                }
+            }
+            const uint32_t total = __reduce_add_sync(0xffffffffu, nbytes);
+            __syncwarp();
+            if (lane == 0) mbar_arrive_expect_tx(&full[slot], 2 * total);
+            __syncwarp();
+            if (nbytes) {
+#pragma unroll
+                for (int sl = 0; sl < SLABS; ++sl) {
+                    tma_load_2d(kdst + sl * SLAB_BYTES + r * 128, &tmk, sl * 64, y, &full[slot], policy);
+                    tma_load_2d(vdst + sl * SLAB_BYTES + r * 128, &tmv, sl * 64, y, &full[slot], policy);
+                }
+            }
+        }
+        return;
+    }
+
+    // ---------------- consumers ----------------
+    const int cw = warp - 1;
+    const int g = lane >> 2;  // fragment row group
+    const int t = lane & 3;   // fragment column pair
+    const int q4 = lane >> 3;
+    const int r8 = lane & 7;
+    const int rbase = row0 + 16 * cw;
+    // Q A-fragments of rows rbase + g and rbase + g + 8 (zero past the group)
+    uint32_t qa[KSTEPS][4];
+    {
+        const uint16_t* qv = static_cast<const uint16_t*>(p.q);
+        const uint16_t* qrow[2] = {nullptr, nullptr};
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int r = rbase + g + 8 * i;
+            if (r < rows_total)
+                qrow[i] = qv + ((int64_t)(s_start + r / G) * p.num_q_heads + (int64_t)kvh * G + r % G) * D;
+        }
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+            qa[kk][0] = qrow[0] ? *reinterpret_cast<const uint32_t*>(qrow[0] + kk * 16 + 2 * t) : 0u;
+            qa[kk][1] = qrow[1] ? *reinterpret_cast<const uint32_t*>(qrow[1] + kk * 16 + 2 * t) : 0u;
+            qa[kk][2] = qrow[0] ? *reinterpret_cast<const uint32_t*>(qrow[0] + kk * 16 + 8 + 2 * t) : 0u;
+            qa[kk][3] = qrow[1] ? *reinterpret_cast<const uint32_t*>(qrow[1] + kk * 16 + 8 + 2 * t) : 0u;
+        }
+    }
+    float o[NTD][4];
+#pragma unroll
+    for (int nd = 0; nd < NTD; ++nd)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) o[nd][c] = 0.f;
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+    bool aborted = false;
+    for (int j = 0; j < nstage; ++j) {
+        const int slot = j % p.stages;
+        if (!mbar_wait(&full[slot], (j / p.stages) & 1, p.err)) {
+            aborted = true;
+            break;
+        }
+        const uint32_t kst = smem_addr(ring + (size_t)slot * 2 * STAGE_BYTES);
+        const uint32_t vst = kst + STAGE_BYTES;
+        const int valid = min(kStageTokens, ntok - j * kStageTokens);
+        // S = Q . K^T over the stage's 32 tokens: four 8-token column tiles
+        float s[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) s[nt][c] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+            const uint32_t slab = kst + (kk >> 2) * SLAB_BYTES;
+            const int chunk16 = (kk & 3) * 2 + (q4 & 1);
+#pragma unroll
+            for (int pair = 0; pair < 2; ++pair) {
+                uint32_t b[4];
+                ldmatrix_x4(swizzled(slab, 8 * (2 * pair + (q4 >> 1)) + r8, chunk16), b[0], b[1], b[2], b[3]);
+                mma_bf16_16816(s[2 * pair], qa[kk], b[0], b[1]);
+                mma_bf16_16816(s[2 * pair + 1], qa[kk], b[2], b[3]);
+            }
+        }
+        // online softmax per row (this lane: rows g and g + 8, tokens
+        // 8 nt + 2 t and 8 nt + 2 t + 1), log2 domain, masked past the prefix
+        float alpha[2];
+        bool rescale = false;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            float mx = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const int tok = 8 * nt + 2 * t + c;
+                    const float v = tok < valid ? s[nt][2 * i + c] * p.scale_log2 : -INFINITY;
+                    s[nt][2 * i + c] = v;
+                    mx = fmaxf(mx, v);
+                }
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float m_new = fmaxf(m[i], mx);
+            float a = 1.f;
+            if (m_new == -INFINITY) {
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) s[nt][2 * i] = s[nt][2 * i + 1] = 0.f;
+            } else {
+                a = exp2f(m[i] - m_new);
+                float sum = 0.f;
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        const float e = exp2f(s[nt][2 * i + c] - m_new);
+                        s[nt][2 * i + c] = e;
+                        sum += e;
+                    }
+                l[i] = l[i] * a + sum;
+                m[i] = m_new;
+            }
+            alpha[i] = a;
+            rescale |= a != 1.f;
+        }
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+            for (int nd = 0; nd < NTD; ++nd) {
+                o[nd][0] *= alpha[0];
+                o[nd][1] *= alpha[0];
+                o[nd][2] *= alpha[1];
+                o[nd][3] *= alpha[1];
+            }
+        }
+        // O += P . V, one 16-token K step per pair of S column tiles
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            uint32_t ah[4], al[4];
+#pragma unroll
+            for (int f = 0; f < 4; ++f) {
+                // f = 0: row g, tile 2 ks; 1: row g + 8, tile 2 ks; 2, 3: tile 2 ks + 1
+                const float p0 = s[2 * ks + (f >> 1)][2 * (f & 1)], p1 = s[2 * ks + (f >> 1)][2 * (f & 1) + 1];
+                ah[f] = pack_bf16x2(p0, p1);
+                al[f] = pack_bf16x2(p0 - bf16_lo_to_f32(ah[f]), p1 - bf16_hi_to_f32(ah[f]));
+            }
+#pragma unroll
+            for (int ndp = 0; ndp < NTD / 2; ++ndp) {
+                const int nd = 2 * ndp + (q4 >> 1);
+                uint32_t b[4];
+                ldmatrix_x4_trans(swizzled(vst + (nd >> 3) * SLAB_BYTES, 16 * ks + 8 * (q4 & 1) + r8, nd & 7), b[0],
+                                  b[1], b[2], b[3]);
+                mma_bf16_16816(o[2 * ndp], ah, b[0], b[1]);
+                mma_bf16_16816(o[2 * ndp], al, b[0], b[1]);
+                mma_bf16_16816(o[2 * ndp + 1], ah, b[2], b[3]);
+                mma_bf16_16816(o[2 * ndp + 1], al, b[2], b[3]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+    }
+    if (aborted) return;
+    // l was summed per lane over its own columns: add the quad's four lanes
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        l[i] += __shfl_xor_sync(0xffffffffu, l[i], 1);
+        l[i] += __shfl_xor_sync(0xffffffffu, l[i], 2);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int r = rbase + g + 8 * i;
+        if (r >= rows_total) continue;
+        const int64_t qrow = (int64_t)(s_start + r / G) * p.num_q_heads + (int64_t)kvh * G + r % G;
+        const int64_t slotrow = qrow * p.max_splits + split;
+        float* dst = p.part_o + slotrow * D + 2 * t;
+#pragma unroll
+        for (int nd = 0; nd < NTD; ++nd) {
+            float2 v;
+            v.x = l[i] > 0.f ? o[nd][2 * i] / l[i] : 0.f;
+            v.y = l[i] > 0.f ? o[nd][2 * i + 1] / l[i] : 0.f;
+            *reinterpret_cast<float2*>(dst + 8 * nd) = v;
+        }
+        if (t == 0) {
+            p.part_ml[2 * slotrow] = m[i];
+            p.part_ml[2 * slotrow + 1] = l[i];
+        }
+    }
 }
 
 // Second pass: out = sum_s w_s o_s / sum_s w_s with w_s = l_s * 2^(m_s - max m),
@@ -907,8 +1296,10 @@ __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(const De
     const int64_t row = (int64_t)blockIdx.x * (kMergeWarps / kMergeWarpsPerRow) + warp / kMergeWarpsPerRow;
     int ns = 0;
     if (row < rows) {
-        const int L = clamp_len(p, (int)(row / p.num_q_heads), false);
-        ns = L > 0 ? (L + p.partition - 1) / p.partition : 1;
+        const int b = (int)(row / p.num_q_heads);
+        const int L = clamp_len(p, b, false);
+        int sp;
+        ns = row_splits(p, L, seq_prefix_len(p, b, L), &sp);
     }
     float m = -INFINITY, W = 0.f, acc[VPL];
 #pragma unroll
@@ -991,11 +1382,21 @@ __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(const De
 // ---------------------------------------------------------------------------
 struct Plan {
     int partition;
-    int max_splits;
+    int max_splits;     // partial-result slots per row (prefix splits + suffix splits)
+    int suffix_splits;  // pass 1's grid.x
     size_t part_o_bytes;
     size_t part_ml_bytes;
+    size_t seq_prefix_bytes;
     size_t workspace;
+    // shared-prefix calls only
+    int prefix_partition;
+    int prefix_splits;
+    int mt;      // 16-row query tiles per prefix CTA (consumer warps)
+    int chunks;  // prefix CTAs per (group, kv head) along the query rows
 };
+
+constexpr int kPrefixRingBytes = 64 * 1024;
+constexpr int kMinPrefixPartition = 256;
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -1014,23 +1415,45 @@ int auto_partition(int batch, int num_q_heads, int num_kv_heads, int max_context
     return P;
 }
 
+// Tokens per prefix split: as long as possible (4096) while the prefix pass
+// still has at least two CTAs per SM to run, halved down to 256 otherwise.
+int auto_prefix_partition(int num_groups, int num_kv_heads, int chunks, int max_prefix_len) {
+    int P = kMaxAutoPartition;
+    const int64_t want = 2ll * num_sms();
+    const int64_t L = max_prefix_len > 0 ? max_prefix_len : 1;
+    while (P > kMinPrefixPartition && (int64_t)num_groups * num_kv_heads * chunks * ((L + P - 1) / P) < want) P /= 2;
+    return P;
+}
+
+// num_groups == 0: plain decode.  Otherwise the shared-prefix layout: the
+// prefix pass's tiling and split size, prefix slots before suffix slots, and
+// the per-sequence prefix lengths after the partial results.
 int make_plan(int batch, int num_q_heads, int num_kv_heads, int head_dim, int max_context_len, int partition_size,
-              Plan* plan) {
+              Plan* plan, int num_groups = 0, int max_group = 0, int max_prefix = 0) {
     int P = partition_size;
     if (P == 0) P = auto_partition(batch, num_q_heads, num_kv_heads, max_context_len);
     if (P < kStageTokens || P > kMaxPartition || P % kStageTokens != 0) return PA_ERR_INVALID_ARG;
     const int L = max_context_len > 0 ? max_context_len : 1;
     const int splits = (L + P - 1) / P;
+    *plan = Plan{};
     plan->partition = P;
+    plan->suffix_splits = splits;
     plan->max_splits = splits;
-    if (splits > 1) {
-        const size_t rows = (size_t)batch * num_q_heads * splits;
+    if (num_groups > 0) {
+        const int rows = max_group * (num_q_heads / num_kv_heads);
+        plan->mt = rows <= 16 ? 1 : (rows <= 32 ? 2 : 4);
+        plan->chunks = (rows + 16 * plan->mt - 1) / (16 * plan->mt);
+        plan->prefix_partition = auto_prefix_partition(num_groups, num_kv_heads, plan->chunks, max_prefix);
+        plan->prefix_splits = max_prefix > 0 ? (max_prefix + plan->prefix_partition - 1) / plan->prefix_partition : 0;
+        plan->max_splits = plan->prefix_splits + splits;
+        plan->seq_prefix_bytes = align256((size_t)batch * sizeof(int32_t));
+    }
+    if (plan->max_splits > 1) {
+        const size_t rows = (size_t)batch * num_q_heads * plan->max_splits;
         plan->part_o_bytes = align256(rows * head_dim * sizeof(float));
         plan->part_ml_bytes = align256(rows * 2 * sizeof(float));
-    } else {
-        plan->part_o_bytes = plan->part_ml_bytes = 0;
     }
-    plan->workspace = plan->part_o_bytes + plan->part_ml_bytes;
+    plan->workspace = plan->part_o_bytes + plan->part_ml_bytes + plan->seq_prefix_bytes;
     return PA_OK;
 }
 
@@ -1080,6 +1503,22 @@ int launch_pass1_mma(const DecodeParams& p, const CUtensorMap& tmk, const CUtens
     return launch_pdl(decode_pass1_mma_kernel<D, NT>, grid, dim3(kDecodeThreads), smem, st, p, tmk, tmv);
 }
 
+template <int D, int MT>
+int launch_prefix_mma(const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, dim3 grid, size_t smem,
+                      cudaStream_t st) {
+    static std::atomic<unsigned long long> configured{0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(configured.load() & bit)) {
+        if (cudaFuncSetAttribute(decode_prefix_mma_kernel<D, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kMaxDynamicSmem) != cudaSuccess)
+            return PA_ERR_CUDA;
+        configured.fetch_or(bit);
+    }
+    return launch_pdl(decode_prefix_mma_kernel<D, MT>, grid, dim3(32 * (1 + MT)), smem, st, p, tmk, tmv);
+}
+
 template <typename T, int D, int G>
 int launch_pass1(const DecodeParams& p, dim3 grid, size_t smem, cudaStream_t st) {
     static std::atomic<unsigned long long> configured{0};
@@ -1106,22 +1545,31 @@ int dispatch_group(int G, const DecodeParams& p, dim3 grid, size_t smem, cudaStr
     }
 }
 
+// p.num_groups > 0: shared-prefix decode (bf16, paged), with the prefix pass
+// launched before pass 1.
 int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* workspace, size_t workspace_bytes,
                int max_context_len, int partition_size, cudaStream_t st) {
     const int G = p.num_q_heads / p.num_kv_heads;
     Plan plan;
-    int rc = make_plan(batch, p.num_q_heads, p.num_kv_heads, head_dim, max_context_len, partition_size, &plan);
+    int rc = make_plan(batch, p.num_q_heads, p.num_kv_heads, head_dim, max_context_len, partition_size, &plan,
+                       p.num_groups, p.max_group, p.max_prefix);
     if (rc) return rc;
     if (plan.workspace > 0) {
         if (!workspace || workspace_bytes < plan.workspace || !aligned16(workspace)) return PA_ERR_WORKSPACE;
-        p.part_o = static_cast<float*>(workspace);
-        p.part_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + plan.part_o_bytes);
+        char* ws = static_cast<char*>(workspace);
+        p.part_o = plan.part_o_bytes ? reinterpret_cast<float*>(ws) : nullptr;
+        p.part_ml = plan.part_ml_bytes ? reinterpret_cast<float*>(ws + plan.part_o_bytes) : nullptr;
+        p.seq_prefix = plan.seq_prefix_bytes
+                           ? reinterpret_cast<int32_t*>(ws + plan.part_o_bytes + plan.part_ml_bytes)
+                           : nullptr;
     } else {
         p.part_o = nullptr;
         p.part_ml = nullptr;
+        p.seq_prefix = nullptr;
     }
     p.partition = plan.partition;
     p.max_splits = plan.max_splits;
+    p.prefix_partition = plan.prefix_partition;
     p.batch = batch;
     p.longest_first = batch <= kLongestFirstMaxBatch;
     p.err = error_word_ptr();
@@ -1144,7 +1592,7 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
     const size_t smem = p.ring_offset + ring_bytes;
     if (smem > (size_t)kMaxDynamicSmem) return PA_ERR_UNSUPPORTED;
 
-    dim3 grid((unsigned)plan.max_splits, (unsigned)p.num_kv_heads, (unsigned)batch);
+    dim3 grid((unsigned)plan.suffix_splits, (unsigned)p.num_kv_heads, (unsigned)batch);
     if (kv_dtype == PA_BF16) {
         // tensor-core path: K/V tiles by tiled TMA, contractions by mma.sync
         const uint64_t rows = p.contiguous ? (uint64_t)batch * p.num_kv_heads * (uint64_t)p.L_pad
@@ -1153,6 +1601,29 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
         CUtensorMap tmk, tmv;
         if ((rc = encode_kv_map(&tmk, p.k, rows, head_dim, p.block_size))) return rc;
         if ((rc = encode_kv_map(&tmv, p.v, rows, head_dim, p.block_size))) return rc;
+        if (p.num_groups > 0) {
+            // the prefix pass: a deeper ring (few, long-lived CTAs), every
+            // consumer warp reads every stage
+            DecodeParams pp = p;
+            pp.stages = kPrefixRingBytes / stage_bytes;
+            const int ptable = (plan.prefix_partition / p.block_size) * 4;
+            pp.ring_offset = (int)((16 * pp.stages + ptable + 1023) & ~1023);
+            const size_t psmem = pp.ring_offset + (size_t)pp.stages * stage_bytes + 1024;
+            if (psmem > (size_t)kMaxDynamicSmem) return PA_ERR_UNSUPPORTED;
+            const int64_t gy = (int64_t)p.num_kv_heads * plan.chunks;
+            if (gy > 65535) return PA_ERR_UNSUPPORTED;
+            const dim3 pg((unsigned)(plan.prefix_splits > 0 ? plan.prefix_splits : 1), (unsigned)gy,
+                          (unsigned)p.num_groups);
+            if (head_dim == 128)
+                rc = plan.mt == 1 ? launch_prefix_mma<128, 1>(pp, tmk, tmv, pg, psmem, st)
+                     : plan.mt == 2 ? launch_prefix_mma<128, 2>(pp, tmk, tmv, pg, psmem, st)
+                                    : launch_prefix_mma<128, 4>(pp, tmk, tmv, pg, psmem, st);
+            else
+                rc = plan.mt == 1 ? launch_prefix_mma<64, 1>(pp, tmk, tmv, pg, psmem, st)
+                     : plan.mt == 2 ? launch_prefix_mma<64, 2>(pp, tmk, tmv, pg, psmem, st)
+                                    : launch_prefix_mma<64, 4>(pp, tmk, tmv, pg, psmem, st);
+            if (rc) return rc;
+        }
         p.ring_offset = (int)((16 * stages + table_bytes + 1023) & ~1023);
         const size_t smem_mma = p.ring_offset + ring_bytes + 1024;
         if (smem_mma > (size_t)kMaxDynamicSmem) return PA_ERR_UNSUPPORTED;
@@ -1310,6 +1781,67 @@ extern "C" int pa_paged_attention_decode_append(const void* q, const void* key, 
     p.v_new = value;
     p.slots = slot_mapping;
     p.append = 1;
+    return run_decode(p, head_dim, kv_dtype, batch, workspace, workspace_bytes, max_context_len, partition_size,
+                      static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int pa_paged_attention_shared_prefix_workspace_size(int batch, int num_q_heads, int num_kv_heads,
+                                                              int head_dim, int max_context_len, int block_size,
+                                                              int num_groups, int max_group_size, int max_prefix_len,
+                                                              int partition_size, size_t* workspace_bytes) {
+    if (!workspace_bytes) return PA_ERR_INVALID_ARG;
+    int rc = check_shapes(batch, num_q_heads, num_kv_heads, head_dim, block_size, PA_BF16, PA_F32, max_context_len);
+    if (rc) return rc;
+    if (num_groups < 1 || max_group_size < 1 || max_prefix_len < 0 || max_prefix_len > max_context_len)
+        return PA_ERR_INVALID_ARG;
+    Plan plan;
+    rc = make_plan(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, partition_size, &plan, num_groups,
+                   max_group_size, max_prefix_len);
+    if (rc) return rc;
+    *workspace_bytes = plan.workspace;
+    return PA_OK;
+}
+
+extern "C" int pa_paged_attention_decode_shared_prefix(
+    const void* q, const void* k_pool, const void* v_pool, const int32_t* block_tables, int max_blocks_per_seq,
+    const int32_t* context_lens, int max_context_len, float scale, int block_size, void* out, int out_dtype,
+    int batch, int num_q_heads, int num_kv_heads, int head_dim, int64_t num_blocks, int kv_dtype,
+    const int32_t* group_starts, const int32_t* group_prefix_lens, int num_groups, int max_group_size,
+    int max_prefix_len, int partition_size, void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_shapes(batch, num_q_heads, num_kv_heads, head_dim, block_size, kv_dtype, out_dtype,
+                          max_context_len);
+    if (rc) return rc;
+    if (kv_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+    if (max_blocks_per_seq < 0 || num_blocks < 0) return PA_ERR_INVALID_ARG;
+    if ((int64_t)max_context_len > (int64_t)max_blocks_per_seq * block_size) return PA_ERR_INVALID_ARG;
+    if (batch == 0) return PA_OK;
+    if (num_groups < 1 || num_groups > batch || max_group_size < 1 || max_group_size > batch ||
+        max_prefix_len < 0 || max_prefix_len > max_context_len)
+        return PA_ERR_INVALID_ARG;
+    if (!q || !k_pool || !v_pool || !block_tables || !context_lens || !out || !group_starts || !group_prefix_lens)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool)) return PA_ERR_INVALID_ARG;
+    DecodeParams p = {};
+    p.q = q;
+    p.k = k_pool;
+    p.v = v_pool;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.out = out;
+    p.num_blocks = num_blocks;
+    p.max_len = max_context_len;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.block_size = block_size;
+    p.out_bf16 = out_dtype == PA_BF16;
+    p.contiguous = 0;
+    p.scale_log2 = scale * kLog2e;
+    p.group_starts = group_starts;
+    p.group_prefix = group_prefix_lens;
+    p.num_groups = num_groups;
+    p.max_group = max_group_size;
+    p.max_prefix = max_prefix_len;
     return run_decode(p, head_dim, kv_dtype, batch, workspace, workspace_bytes, max_context_len, partition_size,
                       static_cast<cudaStream_t>(stream));
 }

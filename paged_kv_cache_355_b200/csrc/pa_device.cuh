@@ -45,6 +45,13 @@ __device__ __forceinline__ void griddep_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Order this thread's earlier generic-proxy writes to shared memory before
+// later async-proxy (TMA) accesses of the same bytes: a ring slot that the
+// threads wrote into (zeroed rows, patched rows) is refilled by TMA later.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Make barrier initialisation visible to the async (bulk-copy) proxy.
 __device__ __forceinline__ void fence_barrier_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");

@@ -59,6 +59,16 @@ static_assert(kTiles == 2, "the softmax warpgroups select their tile's values be
 constexpr int kStages = 4;     // K/V ring depth
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.f;  // lazy-rescale threshold of the running max (log2 units)
+// P.V with P as a bf16 high part plus a bf16 residual (two MMAs per key
+// step, ~16 significant bits of weight) or as the high part alone (one MMA,
+// 8 bits).  The library is built with the split; building with
+// -DPA_PREFILL_SINGLE_P gives the one-MMA form, for measuring what the split
+// costs and what it buys in accuracy.
+#ifdef PA_PREFILL_SINGLE_P
+constexpr bool kSplitP = false;
+#else
+constexpr bool kSplitP = true;
+#endif
 
 struct PrefillParams {
     const void* q;
@@ -366,7 +376,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint64_t db = umma_desc(v_base + kk * 2048, KV_SLAB, 1024);
                         umma_tmem_a(tmem + t * TILE_COLS + O_COL, p_col + kk * 8, db, IDESC_O,
                                     (jp > 0 || kk > 0) ? 1u : 0u);
-                        umma_tmem_a(tmem + t * TILE_COLS + O_COL, p_col + S_COLS / 2 + kk * 8, db, IDESC_O, 1u);
+                        if (kSplitP)
+                            umma_tmem_a(tmem + t * TILE_COLS + O_COL, p_col + S_COLS / 2 + kk * 8, db, IDESC_O, 1u);
                     }
                     umma_commit(&pv_done[t][jp & 1]);
                     umma_commit(&kv_empty[jp % kStages]);
@@ -473,10 +484,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < kKeys / 2; ++c) {
                 const float a = sv[2 * c], bb = sv[2 * c + 1];
                 hi[c] = pack_bf16x2(a, bb);
-                lo[c] = pack_bf16x2(a - bf16_lo_to_f32(hi[c]), bb - bf16_hi_to_f32(hi[c]));
+                if (kSplitP) lo[c] = pack_bf16x2(a - bf16_lo_to_f32(hi[c]), bb - bf16_hi_to_f32(hi[c]));
             }
             tmem_st32u(lane_base + s * S_COLS, hi);
-            tmem_st32u(lane_base + s * S_COLS + S_COLS / 2, lo);
+            if (kSplitP) tmem_st32u(lane_base + s * S_COLS + S_COLS / 2, lo);
             // keys past the sequence end carry weight 0, but 0 * NaN is NaN in
             // the MMA: zero those V rows of the CTA's last tile (both
             // warpgroups that use it do, each before it signals its P)

@@ -40,7 +40,8 @@ void* g_scratch_addr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device.  Resolved on the
 // first call per device (with that device current) and cached; NULL if the
-// lookup fails.
+// lookup fails.  The cache assumes the device's primary context lives until
+// the process exits: after a cudaDeviceReset the cached address is stale.
 void* scratch_address() {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;

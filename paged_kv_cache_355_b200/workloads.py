@@ -94,6 +94,9 @@ class DecodeCase:
     k_pool: torch.Tensor             # [NB, Hkv, bs, D]
     v_pool: torch.Tensor
     cow_pairs: torch.Tensor = field(default_factory=lambda: torch.zeros((0, 2), dtype=torch.int64))
+    # sequences [starts[g], starts[g + 1]) share their first prefix_len[g]
+    # tokens in the same physical blocks (None: no sharing)
+    prefix_groups: tuple | None = None
 
     @property
     def max_len(self) -> int:
@@ -153,8 +156,11 @@ def make_case(name: str, device="cpu", seed: int | None = None, batch: int | Non
     bs = w.block_size
 
     cow_pairs = torch.zeros((0, 2), dtype=torch.int64)
+    groups = None
     if w.lengths == "cow":
         tables, lengths, new_sid, new_pos, cow_pairs, nb = _cow_layout(w, host, place)
+        # the samples of a prompt are consecutive and share its full blocks
+        groups = ([p * w.samples for p in range(w.prompts + 1)], [(w.prompt_len // bs) * bs] * w.prompts)
     else:
         lengths = draw_lengths(w, host)
         need = [_blocks_for(L, bs) for L in lengths]
@@ -182,7 +188,15 @@ def make_case(name: str, device="cpu", seed: int | None = None, batch: int | Non
         new_sid = list(range(w.batch))
         new_pos = [L - 1 for L in lengths]
 
-    return build_case(w, lengths, tables, nb, new_sid, new_pos, cow_pairs, seed + 2, device)
+    case = build_case(w, lengths, tables, nb, new_sid, new_pos, cow_pairs, seed + 2, device)
+    case.prefix_groups = groups
+    return case
+
+
+def shared_prefix_groups(case: DecodeCase):
+    """(group_starts, prefix_len) lists of a case whose consecutive sequences
+    share their leading blocks, as its layout made them; None if none do."""
+    return case.prefix_groups
 
 
 def build_case(w: Workload, lengths, tables, num_blocks: int, new_sid, new_pos, cow_pairs=None, value_seed: int = 0,

@@ -134,3 +134,40 @@ def assert_bf16_output_matches_oracle(got, ref, what: str = ""):
     far = (steps > 1) & (err > F32_ATOL)
     assert not far.any(), f"{what}: {int(far.sum())} elements more than one bf16 step (and 1e-5) from the oracle"
     return float(err.max())
+
+
+def shared_prefix_case(groups, num_q_heads, num_kv_heads, head_dim, block_size, dtype, seed=0, extra_blocks=4):
+    """A decode case whose sequences come in groups sharing a prompt.
+
+    groups: list of (prefix_len, [member lengths]); prefix_len is a multiple
+    of block_size and at most every member's length.  Each group's first
+    prefix_len / block_size blocks are the same physical ids in every
+    member's table; every other block is private.  Blocks are scattered over
+    the pool.  Returns (case, group_starts, group_prefix_lens) with the two
+    lists as the shared-prefix call takes them."""
+    import torch
+
+    from paged_kv_cache_355_b200.workloads import Workload, build_case
+
+    bs = block_size
+    need = 0
+    for P, members in groups:
+        assert P % bs == 0 and all(L >= P for L in members)
+        need += P // bs + sum(-(-L // bs) - P // bs for L in members)
+    nb = need + extra_blocks
+    ids = iter(torch.randperm(nb, generator=torch.Generator().manual_seed(seed + 1)).tolist())
+    tables, lengths, starts, plens = [], [], [0], []
+    for P, members in groups:
+        shared = [next(ids) for _ in range(P // bs)]
+        for L in members:
+            t = list(shared)
+            while len(t) < -(-L // bs):
+                t.append(next(ids))
+            tables.append(t)
+            lengths.append(L)
+        starts.append(len(lengths))
+        plens.append(P)
+    w = Workload("shared", len(lengths), num_q_heads, num_kv_heads, head_dim, bs, dtype, "fixed")
+    sid = [b for b, L in enumerate(lengths) if L > 0]
+    case = build_case(w, lengths, tables, nb, sid, [lengths[b] - 1 for b in sid], None, seed + 2)
+    return case, starts, plens

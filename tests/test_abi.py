@@ -127,3 +127,63 @@ def test_cache_kernels_reject_bad_arguments(lib):
 def test_selftest_rejects_bad_limits(lib):
     assert lib.pa_selftest_wait_timeout(0, None) == INVALID
     assert lib.pa_selftest_wait_timeout(2_000_001, None) == INVALID
+
+
+def test_static_scratch_size_constant_matches_the_header():
+    """The binding's STATIC_SCRATCH_BYTES is the header's PA_STATIC_SCRATCH_BYTES."""
+    text = open(HEADER).read()
+    m = re.search(r"#define\s+PA_STATIC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", text)
+    assert m, "PA_STATIC_SCRATCH_BYTES not found in include/pa.h"
+    import paged_kv_cache_355_b200 as pa
+
+    assert pa.STATIC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
+
+
+def test_read_probe_rejects_bad_arguments(lib):
+    P = ctypes.c_void_p
+    lib.pa_hbm_read_probe.argtypes = [P, ctypes.c_size_t, P]
+    assert lib.pa_hbm_read_probe(P(16), 17, None) == INVALID   # not a multiple of 16 bytes
+    assert lib.pa_hbm_read_probe(P(24), 16, None) == INVALID   # not 16-byte aligned
+    assert lib.pa_hbm_read_probe(P(0), 16, None) == INVALID
+    assert lib.pa_hbm_read_probe(P(16), 0, None) == OK         # nothing to read, nothing launched
+
+
+def _shared(lib, **kw):
+    args = dict(q=16, k=16, v=16, bt=16, mbs=8, lens=16, maxlen=100, scale=0.1, bs=16, out=16, out_dtype=0,
+                batch=4, hq=8, hkv=2, d=128, nb=10, kv_dtype=1, gs=16, gl=16, ng=2, mg=2, mp=32, part=0, ws=0,
+                ws_bytes=0, stream=None)
+    args.update(kw)
+    P = ctypes.c_void_p
+    return lib.pa_paged_attention_decode_shared_prefix(
+        P(args["q"]), P(args["k"]), P(args["v"]), P(args["bt"]), args["mbs"], P(args["lens"]), args["maxlen"],
+        ctypes.c_float(args["scale"]), args["bs"], P(args["out"]), args["out_dtype"], args["batch"], args["hq"],
+        args["hkv"], args["d"], ctypes.c_int64(args["nb"]), args["kv_dtype"], P(args["gs"]), P(args["gl"]),
+        args["ng"], args["mg"], args["mp"], args["part"], P(args["ws"]), ctypes.c_size_t(args["ws_bytes"]),
+        P(args["stream"]))
+
+
+def test_shared_prefix_rejects_bad_arguments(lib):
+    assert _shared(lib, kv_dtype=0) == UNSUPPORTED        # bf16 only
+    assert _shared(lib, ng=0) == INVALID                  # no group
+    assert _shared(lib, ng=5) == INVALID                  # more groups than sequences
+    assert _shared(lib, mg=0) == INVALID
+    assert _shared(lib, mp=101) == INVALID                # prefix bound above max_context_len
+    assert _shared(lib, mp=-1) == INVALID
+    assert _shared(lib, gs=0) == INVALID
+    assert _shared(lib, gl=0) == INVALID
+    assert _shared(lib) == WORKSPACE                      # always needs scratch (prefix lengths at least)
+    assert _shared(lib, batch=0, q=0) == OK
+
+
+def test_shared_prefix_workspace_size(lib):
+    sz = ctypes.c_size_t(0)
+    f = lib.pa_paged_attention_shared_prefix_workspace_size
+    # no prefix, one suffix split: only the per-sequence prefix lengths
+    assert f(4, 8, 2, 128, 100, 16, 2, 2, 0, 128, ctypes.byref(sz)) == OK
+    assert sz.value == 256
+    # a prefix: prefix splits + suffix splits per row, then the lengths
+    assert f(4, 8, 2, 128, 100, 16, 2, 2, 64, 128, ctypes.byref(sz)) == OK
+    rows = 4 * 8 * 2
+    assert sz.value == -(-rows * 128 * 4 // 256) * 256 + -(-rows * 2 * 4 // 256) * 256 + 256
+    assert f(4, 8, 2, 128, 100, 16, 0, 2, 64, 128, ctypes.byref(sz)) == INVALID
+    assert f(4, 8, 2, 128, 100, 16, 2, 2, 101, 128, ctypes.byref(sz)) == INVALID

@@ -27,7 +27,7 @@ def bench():
 
 def _args(**kw):
     base = dict(gpus=1, steps=3, warmup=3, workload="llama7b", impl="ours", partition=0, batch=None,
-                no_cpu_baseline=True, op="decode")
+                no_cpu_baseline=True, op="decode", no_other_workloads=True)
     base.update(kw)
     return argparse.Namespace(**base)
 
@@ -60,10 +60,30 @@ def test_decode_bench_line_has_the_contract_fields(bench, capsys, workload, batc
     assert d["gpu_launches"] >= 2 * d["steps"]
     assert d["cache_part"]["ms"] > 0 and d["cache_part"]["bytes"] > 0
     assert {"sm_mhz", "sm_max_mhz", "reasons"} <= set(d["clocks"])
+    for k in ("step_ms", "decode_attention_ms"):
+        st = d[k]
+        assert st["p10"] <= st["median"] <= st["p90"] and st["n"] >= 3
+    assert d["decode_attention_ms"]["n"] >= 100
+    assert r["read_ceiling_gbs"] > 0 and abs(r["frac_of_read_ceiling"] - r["achieved"] / r["read_ceiling_gbs"]) < 1e-9
+    assert e["host_wall_ms_per_step"] > 0
+    assert d["other_workloads"] is None
     if workload == "cow":
         assert d["unique_kv"]["bytes_per_step"] < d["config"]["kv_bytes_per_step"]
     else:
         assert d["unique_kv"] is None
+
+
+def test_default_run_times_the_other_workloads(bench, capsys):
+    """The driver's default run (Llama-7B-shaped headline) also times the
+    GQA, long-context and shared-prefix decode calls in the same line."""
+    bench.run_ours(_args(steps=3, warmup=3, no_other_workloads=False))
+    d = _line(capsys)
+    o = d["other_workloads"]
+    for name in ("gqa", "long16", "cow"):
+        assert o[name]["gbs"] > 0 and o[name]["decode_ms"]["n"] >= 100, name
+        assert abs(o[name]["frac"] - o[name]["gbs"] / d["roofline"]["peak"]) < 1e-9
+    assert o["cow"]["unique_kv"]["bytes"] < o["cow"]["kv_bytes"]
+    assert "unique_kv" not in o["gqa"]
 
 
 def test_prefill_bench_line(bench, capsys):

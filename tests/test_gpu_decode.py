@@ -175,6 +175,60 @@ def test_decode_append_equals_write_then_decode(pa, dtype, D, bs, G, partition):
     assert pa.pa_read_error_flag() == 0
 
 
+@pytest.mark.parametrize("fault", ["length_over_max", "length_over_max_unmapped", "bad_last_block",
+                                   "negative_last_block", "negative_length", "bad_middle_block"])
+def test_decode_append_error_paths_match_two_calls(pa, fault):
+    """Bad inputs: the one-launch step leaves the pools, the slots and the
+    device error word exactly as pa_reshape_and_cache_decode followed by
+    pa_paged_attention_decode leave them, and the rows of the other
+    sequences agree at the bar."""
+    lengths = [40, 17, 65, 33]
+    B, Hkv, G, D, bs = 4, 2, 4, 128, 16
+    case = custom_case(lengths, Hkv * G, Hkv, D, bs, torch.bfloat16, seed=97, extra_blocks=10, table_width=8)
+    bt, lens, max_len = case.block_tables.clone(), case.lengths.clone(), case.max_len
+    bad = {"length_over_max": 2, "length_over_max_unmapped": 2, "bad_last_block": 1, "negative_last_block": 1,
+           "negative_length": 3, "bad_middle_block": 0}[fault]
+    if fault == "length_over_max":
+        max_len = 50  # sequence 2 (65 tokens) is longer; its token 64 still has a table entry
+    elif fault == "length_over_max_unmapped":
+        max_len = 50
+        bt[2, 4] = -1  # ... and here it has none
+    elif fault == "bad_last_block":
+        bt[1, 1] = case.num_blocks + 5  # the block of sequence 1's new token is outside the pool
+    elif fault == "negative_last_block":
+        bt[1, 1] = -3
+    elif fault == "negative_length":
+        lens[3] = -5
+    else:
+        bt[0, 1] = case.num_blocks + 2  # a block attention reads, not the written one
+    g = torch.Generator().manual_seed(98)
+    key = torch.randn(B, Hkv, D, generator=g).to(torch.bfloat16).cuda()
+    val = torch.randn(B, Hkv, D, generator=g).to(torch.bfloat16).cuda()
+    q, gbt, glens = case.q.cuda(), bt.cuda(), lens.cuda()
+    pa.pa_read_error_flag()
+
+    # two calls
+    k2, v2 = case.k_pool.cuda(), case.v_pool.cuda()
+    s2 = torch.full((B,), 7, dtype=torch.int64, device="cuda")
+    o2 = torch.zeros(B, Hkv * G, D, device="cuda")
+    pa.pa_reshape_and_cache_decode(key, val, k2, v2, gbt, glens, s2)
+    pa.pa_paged_attention_decode(q, k2, v2, gbt, glens, max_len, case.scale, o2)
+    flag2 = pa.pa_read_error_flag()
+    # one launch
+    k1, v1 = case.k_pool.cuda(), case.v_pool.cuda()
+    s1 = torch.full((B,), 7, dtype=torch.int64, device="cuda")
+    o1 = torch.zeros(B, Hkv * G, D, device="cuda")
+    pa.pa_paged_attention_decode_append(q, key, val, k1, v1, gbt, glens, max_len, case.scale, o1, slot_mapping=s1)
+    flag1 = pa.pa_read_error_flag()
+
+    assert flag2 == flag1 == 5, (flag2, flag1)
+    assert torch.equal(s1, s2), (s1.tolist(), s2.tolist())
+    assert torch.equal(k1.view(torch.int16), k2.view(torch.int16))
+    assert torch.equal(v1.view(torch.int16), v2.view(torch.int16))
+    keep = [b for b in range(B) if b != bad]
+    assert_matches_oracle(o1[keep], o2[keep].double().cpu().numpy(), True, f"{fault}: other sequences")
+
+
 def test_single_token_returns_value_bit_exactly(pa):
     case = custom_case([1, 1, 1], 8, 4, 128, 16, torch.float32, seed=11)
     out = run_gpu(pa, case)

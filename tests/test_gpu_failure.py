@@ -36,3 +36,13 @@ def test_wait_that_runs_out_reports_timeout_and_context_survives():
                                np_of(case.lengths), case.scale, 16)
     assert_matches_oracle(out, want, True, "decode after a timed-out wait")
     assert pa.pa_read_error_flag() == 0
+
+
+def test_read_probe_streams_a_buffer_without_errors():
+    import paged_kv_cache_355_b200 as pa
+
+    pa.pa_read_error_flag()
+    for nbytes in (16, 16384 + 48, 64 << 20):
+        buf = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+        pa.pa_hbm_read_probe(buf)
+        assert pa.pa_read_error_flag() == 0

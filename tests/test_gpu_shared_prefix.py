@@ -1,0 +1,160 @@
+"""GPU parity of pa_paged_attention_decode_shared_prefix: groups of sequences
+that share their prompt blocks, attended with one read of each shared block
+per group, against the fp64 oracle (which knows nothing of the sharing: it
+walks every sequence's own table), over head sizes, block sizes, group sizes
+(several row chunks per group included), prefix and suffix splits, members
+whose whole context is the prefix, and broken group descriptions."""
+from __future__ import annotations
+
+import pytest
+import torch
+
+import oracle
+from tests.helpers import assert_matches_oracle, np_of, shared_prefix_case
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def pa():
+    import paged_kv_cache_355_b200 as pa
+
+    assert torch.cuda.is_available()
+    pa.pa_read_error_flag()
+    return pa
+
+
+def _groups(bs):
+    r = lambda x: x - x % bs
+    return [
+        (r(64), [r(64) + 7, r(64) + 1, r(64) + 90]),
+        (0, [5]),
+        (bs, [bs, bs + 1]),  # the first member's whole context is the prefix
+        (r(640), [r(640) + k for k in (0, 1, 13, 31, 32, 33, 200, 7, 64)]),
+        (r(1000), [r(1000) + 3, r(1000) + 517]),
+    ]
+
+
+def run_shared(pa, case, starts, plens, partition=0, max_prefix=None, max_group=None, bt=None, kp=None, vp=None,
+               out_dtype=torch.float32):
+    B, Hq, D = case.q.shape
+    out = torch.full((B, Hq, D), float("nan"), dtype=out_dtype, device="cuda")
+    gs = torch.tensor(starts, dtype=torch.int32, device="cuda")
+    gl = torch.tensor(plens, dtype=torch.int32, device="cuda")
+    mp = max(plens) if max_prefix is None else max_prefix
+    mg = max(b - a for a, b in zip(starts[:-1], starts[1:])) if max_group is None else max_group
+    pa.pa_paged_attention_decode_shared_prefix(
+        case.q.cuda(), (case.k_pool if kp is None else kp).cuda(), (case.v_pool if vp is None else vp).cuda(),
+        (case.block_tables if bt is None else bt).cuda(), case.lengths.cuda(), case.max_len, case.scale, out, gs, gl,
+        mp, mg, partition_size=partition)
+    torch.cuda.synchronize()
+    return out
+
+
+def run_oracle(case, bt=None, kp=None, vp=None):
+    return oracle.paged_decode(np_of(case.q), np_of(case.k_pool if kp is None else kp),
+                               np_of(case.v_pool if vp is None else vp),
+                               np_of(case.block_tables if bt is None else bt), np_of(case.lengths), case.scale,
+                               case.workload.block_size)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("bs", [8, 16, 32])
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("partition", [0, 64])
+def test_shared_prefix_sweep(pa, D, bs, G, partition):
+    Hkv = 2
+    case, starts, plens = shared_prefix_case(_groups(bs), Hkv * G, Hkv, D, bs, torch.bfloat16, seed=D + bs + G)
+    out = run_shared(pa, case, starts, plens, partition)
+    assert_matches_oracle(out, run_oracle(case), True, f"shared prefix D{D} bs{bs} G{G} P{partition}")
+    assert pa.pa_read_error_flag() == 0
+
+
+def test_bf16_output(pa):
+    case, starts, plens = shared_prefix_case(_groups(16), 32, 8, 128, 16, torch.bfloat16, seed=5)
+    out = run_shared(pa, case, starts, plens, out_dtype=torch.bfloat16)
+    assert_matches_oracle(out, run_oracle(case), True, "shared prefix, bf16 out")
+
+
+def test_no_prefix_is_bit_identical_to_plain_decode(pa):
+    """With every prefix 0 the call is pass 1 and the merge of the plain
+    decode, with the same splits: the same bits."""
+    groups = [(0, [70, 5]), (0, [300]), (0, [1, 2, 1000])]
+    case, starts, plens = shared_prefix_case(groups, 16, 4, 128, 16, torch.bfloat16, seed=9)
+    for part in (0, 64):
+        out = run_shared(pa, case, starts, plens, part)
+        ref = torch.full_like(out, float("nan"))
+        pa.pa_paged_attention_decode(case.q.cuda(), case.k_pool.cuda(), case.v_pool.cuda(),
+                                     case.block_tables.cuda(), case.lengths.cuda(), case.max_len, case.scale, ref,
+                                     partition_size=part)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+
+
+def test_repeat_runs_and_physical_permutation_are_bit_identical(pa):
+    case, starts, plens = shared_prefix_case(_groups(16), 32, 8, 128, 16, torch.bfloat16, seed=13, extra_blocks=30)
+    a = run_shared(pa, case, starts, plens)
+    assert torch.equal(a, run_shared(pa, case, starts, plens))
+    perm = torch.randperm(case.num_blocks, generator=torch.Generator().manual_seed(14))
+    kp, vp = torch.empty_like(case.k_pool), torch.empty_like(case.v_pool)
+    kp[perm] = case.k_pool
+    vp[perm] = case.v_pool
+    bt = torch.where(case.block_tables >= 0, perm[case.block_tables.clamp(min=0).long()].to(torch.int32),
+                     case.block_tables)
+    assert torch.equal(a, run_shared(pa, case, starts, plens, bt=bt, kp=kp, vp=vp))
+
+
+def test_nan_poison_outside_the_sequences_is_never_read(pa):
+    case, starts, plens = shared_prefix_case(_groups(16), 16, 4, 128, 16, torch.bfloat16, seed=17, extra_blocks=12)
+    clean = run_shared(pa, case, starts, plens)
+    kp, vp = case.k_pool.clone(), case.v_pool.clone()
+    used = torch.zeros(case.num_blocks, 16, dtype=torch.bool)
+    for b, L in enumerate(case.lengths.tolist()):
+        for t in range(L):
+            used[case.block_tables[b, t // 16], t % 16] = True
+    kp.permute(0, 2, 1, 3)[~used] = float("nan")
+    vp.permute(0, 2, 1, 3)[~used] = float("nan")
+    bt = case.block_tables.clone()
+    bt[bt < 0] = case.num_blocks + 1000
+    assert torch.equal(clean, run_shared(pa, case, starts, plens, bt=bt, kp=kp, vp=vp))
+    assert pa.pa_read_error_flag() == 0
+
+
+@pytest.mark.parametrize("fault", ["not_whole_blocks", "longer_than_a_member", "above_max_prefix",
+                                   "group_above_max_size", "starts_out_of_order"])
+def test_broken_group_description_is_flagged_and_attended_without_sharing(pa, fault):
+    """A group whose description breaks the rules records
+    PA_ERR_BAD_BLOCK_ID and is attended as if nothing were shared, so the
+    output still matches the oracle."""
+    case, starts, plens = shared_prefix_case(_groups(16), 16, 4, 128, 16, torch.bfloat16, seed=23)
+    starts, plens = list(starts), list(plens)
+    kw = {}
+    if fault == "not_whole_blocks":
+        plens[0] = 56                     # not a multiple of 16
+    elif fault == "longer_than_a_member":
+        plens[2] = 32                     # the first member of group 2 has 16 tokens
+    elif fault == "above_max_prefix":
+        kw["max_prefix"] = 512            # group 3 declares 640
+    elif fault == "group_above_max_size":
+        kw["max_group"] = 3               # group 3 has 9 members
+    else:
+        starts[1], starts[2] = starts[2], starts[1]  # group 1 ends before it starts
+    pa.pa_read_error_flag()
+    out = run_shared(pa, case, starts, plens, **kw)
+    assert pa.pa_read_error_flag() == 5
+    if fault == "starts_out_of_order":
+        # groups 0 and 1 now overlap / are empty; only the untouched groups are specified
+        keep = list(range(starts[3], case.workload.batch))
+        assert_matches_oracle(out[keep], run_oracle(case)[keep], True, fault)
+    else:
+        assert_matches_oracle(out, run_oracle(case), True, fault)
+
+
+def test_groups_that_do_not_cover_the_batch_are_flagged(pa):
+    case, starts, plens = shared_prefix_case(_groups(16), 16, 4, 128, 16, torch.bfloat16, seed=29)
+    pa.pa_read_error_flag()
+    short = starts[:-1]
+    out = run_shared(pa, case, short, plens[:-1])  # the last group's sequences belong to no group
+    assert pa.pa_read_error_flag() == 5
+    covered = list(range(short[-1]))
+    assert_matches_oracle(out[covered], run_oracle(case)[covered], True, "covered sequences")
