@@ -568,7 +568,9 @@ def run_ours(args):
 
     max_splits = -(-max(max_len, 1) // part)
     cache_launches = (1 if pairs.numel() else 0) + (1 if plain_decode else 2)
-    decode_launches = (3 if groups is not None else 1 + (1 if max_splits > 1 else 0))
+    # shared prefixes: the prefix pass, pass 1 (which finishes rows whose own
+    # tokens are one split) and the merge pass only when a suffix can split
+    decode_launches = (1 if groups is not None else 0) + 1 + (1 if max_splits > 1 else 0)
     step_launches = decode_launches + (0 if plain_decode and w.dtype == torch.bfloat16 else cache_launches)
 
     # ---- device-resident timed region

@@ -102,8 +102,8 @@ int pa_selftest_wait_timeout(uint32_t limit_us, void* stream);
  * pa_hbm_read_probe -- read `bytes` of device memory at `buffer` as one
  * stream and discard them: the HBM read ceiling against which paged decode
  * attention, itself a read stream of K/V bytes, is judged.  No counterpart in
- * the pages: a measurement aid.  Each CTA (3 per SM) moves a grid-strided
- * series of 16 KB chunks of the buffer into a 4-stage shared-memory ring with
+ * the pages: a measurement aid.  Each CTA (2 per SM) moves a grid-strided
+ * series of 8 KB chunks of the buffer into a 6-stage shared-memory ring with
  * bulk TMA copies and never looks at them; nothing is written to global
  * memory.  buffer: device pointer, 16-byte aligned; bytes: a multiple of 16
  * (0 does nothing); else PA_ERR_INVALID_ARG.  Waits are bounded as everywhere.
@@ -333,13 +333,14 @@ int pa_paged_attention_shared_prefix_workspace_size(int batch, int num_q_heads, 
  *   max_prefix_len     host-side upper bound of the P_g (<= max_context_len)
  *   workspace          pa_paged_attention_shared_prefix_workspace_size bytes
  * Other arguments as for pa_paged_attention_decode.  bf16 only (kv_dtype
- * PA_BF16, else PA_ERR_UNSUPPORTED).  A group whose description breaks these
- * rules (a prefix that is not whole blocks, longer than a member or than
- * max_prefix_len, a group larger than max_group_size, starts out of order)
- * records PA_ERR_BAD_BLOCK_ID and is attended without sharing (prefix 0);
- * groups that do not cover the batch record it too, and the uncovered
- * sequences' outputs are unspecified.  Equal table entries are the caller's
- * precondition and are not checked.
+ * PA_BF16, else PA_ERR_UNSUPPORTED).  A group whose prefix breaks these
+ * rules (not whole blocks, longer than a member or than max_prefix_len) or
+ * that is larger than max_group_size records PA_ERR_BAD_BLOCK_ID and is
+ * attended without sharing (prefix 0), with the correct result.  Starts out
+ * of order or out of range, and groups that do not cover the batch, record it
+ * too; the outputs of the sequences that no well-formed group covers are then
+ * unspecified (but nothing outside the arrays is read or written).  Equal
+ * table entries are the caller's precondition and are not checked.
  */
 int pa_paged_attention_decode_shared_prefix(const void* q, const void* k_pool, const void* v_pool,
                                             const int32_t* block_tables, int max_blocks_per_seq,
@@ -455,6 +456,27 @@ int pa_bm_block_tables(const pa_block_manager* bm, const int64_t* seq_ids, int64
 /* The free list in hand-out order: the first min(cap, free) ids into out,
  * the number of free blocks into *n. */
 int pa_bm_free_list(const pa_block_manager* bm, int64_t* out, int64_t cap, int64_t* n);
+
+/*
+ * The sharing structure of a batch as pa_paged_attention_decode_shared_prefix
+ * takes it (reference-counted prompt blocks shared by parallel samples,
+ * [P2] "Key terms in this lesson"; [P1] "Key takeaways").  seq_ids[0..n) in
+ * batch order are cut into groups of consecutive sequences whose tables begin
+ * with the same physical block; a sequence with no block, or whose first
+ * block differs from its predecessor's, starts a new group.  A group's prefix
+ * is the run of leading table entries that are equal in every member, cut to
+ * the blocks that are full in every member, times block_size (0 when the
+ * members share nothing full).
+ *   group_starts   int32 [n + 1] output: group g is batch rows
+ *                  group_starts[g] .. group_starts[g + 1] - 1
+ *   prefix_lens    int32 [n] output: the first *num_groups entries are used
+ *   num_groups, max_group_size, max_prefix_len  outputs (the host-side
+ *                  bounds the decode call takes)
+ * PA_ERR_INVALID_ARG for an unknown sequence id or a null output.
+ */
+int pa_bm_shared_prefix_groups(const pa_block_manager* bm, const int64_t* seq_ids, int64_t n,
+                               int32_t* group_starts, int32_t* prefix_lens, int64_t* num_groups,
+                               int32_t* max_group_size, int32_t* max_prefix_len);
 
 /*
  * pa_paged_attention_decode_static_scratch -- pa_paged_attention_decode for

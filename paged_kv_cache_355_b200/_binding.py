@@ -69,6 +69,7 @@ _SIGS = {
     "pa_bm_length": ([_P, _I64], _I64),
     "pa_bm_block_tables": ([_P, _P, _I64, _I, _P, _P], _I),
     "pa_bm_free_list": ([_P, _P, _I64, _P], _I),
+    "pa_bm_shared_prefix_groups": ([_P, _P, _I64, _P, _P, _P, _P, _P], _I),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)

@@ -94,3 +94,18 @@ class BlockManager:
         out = np.empty(self.num_blocks, np.int64)
         self._check("pa_bm_free_list", _lib.pa_bm_free_list(self._h, _p(out), self.num_blocks, ctypes.byref(n)))
         return out[: n.value].tolist()
+
+    def shared_prefix_groups(self, seq_ids):
+        """(group_starts int32 [G + 1], prefix_lens int32 [G], max_group_size,
+        max_prefix_len) of a batch in the order given: the inputs of
+        pa_paged_attention_decode_shared_prefix (copy the two arrays to the
+        device)."""
+        ids = np.ascontiguousarray(np.asarray(seq_ids, np.int64))
+        n = ids.shape[0]
+        starts = np.empty(n + 1, np.int32)
+        plens = np.empty(max(n, 1), np.int32)
+        ng, mg, mp = ctypes.c_int64(0), ctypes.c_int32(0), ctypes.c_int32(0)
+        self._check("pa_bm_shared_prefix_groups", _lib.pa_bm_shared_prefix_groups(
+            self._h, _p(ids), n, _p(starts), _p(plens), ctypes.byref(ng), ctypes.byref(mg), ctypes.byref(mp)))
+        g = ng.value
+        return starts[: g + 1].copy(), plens[:g].copy(), int(mg.value), int(mp.value)

@@ -162,3 +162,52 @@ extern "C" int pa_bm_free_list(const pa_block_manager* bm, int64_t* out, int64_t
     for (int64_t i = 0; i < bm->count && i < cap; ++i) out[i] = bm->ring[(bm->head + i) % bm->num_blocks];
     return PA_OK;
 }
+
+// The sharing structure of a batch, in the form the shared-prefix decode takes
+// it: consecutive sequences (in the order given) whose tables begin with the
+// same physical block form a group; the group's prefix is the run of leading
+// table entries equal in every member, cut to the blocks that are full in
+// every member (entry i counts only if every member has at least
+// (i + 1) * block_size tokens).  A sequence with no block, or one whose first
+// block differs from its predecessor's, starts a new group.
+extern "C" int pa_bm_shared_prefix_groups(const pa_block_manager* bm, const int64_t* seq_ids, int64_t n,
+                                          int32_t* group_starts, int32_t* prefix_lens, int64_t* num_groups,
+                                          int32_t* max_group_size, int32_t* max_prefix_len) {
+    if (!bm || n < 0 || !num_groups || !max_group_size || !max_prefix_len ||
+        (n > 0 && (!seq_ids || !group_starts || !prefix_lens)) || n > INT32_MAX)
+        return PA_ERR_INVALID_ARG;
+    std::vector<const pa_block_manager::Seq*> seqs((size_t)n);
+    for (int64_t i = 0; i < n; ++i) {
+        auto it = bm->seqs.find(seq_ids[i]);
+        if (it == bm->seqs.end()) return PA_ERR_INVALID_ARG;
+        seqs[(size_t)i] = &it->second;
+    }
+    int64_t g = 0;
+    *max_group_size = 0;
+    *max_prefix_len = 0;
+    for (int64_t a = 0; a < n;) {
+        const auto& lead = seqs[(size_t)a]->table;
+        int64_t e = a + 1;
+        if (!lead.empty())
+            while (e < n && !seqs[(size_t)e]->table.empty() && seqs[(size_t)e]->table[0] == lead[0]) ++e;
+        // common leading entries, full in every member
+        int64_t k = (int64_t)lead.size();
+        for (int64_t m = a; m < e; ++m) {
+            const auto& t = seqs[(size_t)m]->table;
+            int64_t c = 0;
+            while (c < k && c < (int64_t)t.size() && t[(size_t)c] == lead[(size_t)c]) ++c;
+            k = c;
+            const int64_t full = seqs[(size_t)m]->length / bm->block_size;
+            if (full < k) k = full;
+        }
+        group_starts[g] = (int32_t)a;
+        prefix_lens[g] = (int32_t)(k * bm->block_size);
+        if (e - a > *max_group_size) *max_group_size = (int32_t)(e - a);
+        if (prefix_lens[g] > *max_prefix_len) *max_prefix_len = prefix_lens[g];
+        ++g;
+        a = e;
+    }
+    if (n > 0) group_starts[g] = (int32_t)n;
+    *num_groups = g;
+    return PA_OK;
+}

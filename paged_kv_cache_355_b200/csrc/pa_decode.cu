@@ -200,9 +200,14 @@ __device__ __forceinline__ void store_out(const DecodeParams& p, int64_t idx, fl
 // Combine the consumer warps' (m, l, o) states of one work item, held in
 // shared memory as o[w][h][d], m[w][h], l[w][h], and write the final row (one
 // split) or the normalised partial row plus (m, l) for the merge kernel.
+// When the row's only other splits are prefix splits (written by the prefix
+// pass, which has completed), the row is finished here: the prefix partials
+// are folded in with the same log-sum-exp rescale the merge pass applies, and
+// the merge pass skips the row.
 __device__ __forceinline__ void merge_warps_and_store(const DecodeParams& p, const float* sm_o, const float* sm_m,
                                                       const float* sm_l, int G, int D, int b, int kvh, int split,
-                                                      int num_splits_b) {
+                                                      int num_splits_b, int prefix_splits = 0) {
+    const bool fold_prefix = prefix_splits > 0 && num_splits_b == prefix_splits + 1;
     for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
         const int h = idx / D;
         const int d = idx - h * D;
@@ -219,8 +224,31 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeParams& p, con
                 ot += sm_o[(w * G + h) * D + d] * a;
             }
         }
-        const float val = lt > 0.f ? ot / lt : 0.f;
         const int64_t qrow = (int64_t)b * p.num_q_heads + (int64_t)kvh * G + h;
+        if (fold_prefix) {
+            const float* ml = p.part_ml + qrow * p.max_splits * 2;
+            const float* po = p.part_o + qrow * p.max_splits * D + d;
+            float Mt = M;
+            for (int s = 0; s < prefix_splits; ++s) Mt = fmaxf(Mt, ml[2 * s]);
+            float W = 0.f, acc = 0.f;
+            if (Mt != -INFINITY) {
+                if (M != -INFINITY) {
+                    const float a = exp2f(M - Mt);
+                    W = lt * a;
+                    acc = ot * a;
+                }
+                for (int s = 0; s < prefix_splits; ++s) {
+                    const float ms = ml[2 * s];
+                    if (ms == -INFINITY) continue;
+                    const float w = ml[2 * s + 1] * exp2f(ms - Mt);
+                    W += w;
+                    acc = fmaf(w, po[(int64_t)s * D], acc);
+                }
+            }
+            store_out(p, qrow * D + d, W > 0.f ? acc / W : 0.f);
+            continue;
+        }
+        const float val = lt > 0.f ? ot / lt : 0.f;
         if (num_splits_b == 1) {
             store_out(p, qrow * D + d, val);
         } else {
@@ -943,7 +971,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
         }
     }
     __syncthreads();
-    merge_warps_and_store(p, sm_o, sm_m, sm_l, G, D, b, kvh, prefix_splits + split, num_splits_b);
+    merge_warps_and_store(p, sm_o, sm_m, sm_l, G, D, b, kvh, prefix_splits + split, num_splits_b, prefix_splits);
 }
 
 // ---------------------------------------------------------------------------
@@ -1009,10 +1037,13 @@ __global__ void __launch_bounds__(32 * (1 + MT))
     // the group's description; every CTA of the group reaches the same verdict
     if (threadIdx.x == 0) {
         const int s = p.group_starts[grp], e = p.group_starts[grp + 1], P = p.group_prefix[grp];
-        const bool ok = s >= 0 && e >= s && e <= p.batch && e - s <= p.max_group && P >= 0 && P <= p.max_prefix &&
-                        P % p.block_size == 0;
-        s_start = ok ? s : 0;
-        s_n = ok ? e - s : 0;
+        // a well-formed span gets its members' prefix lengths written in any
+        // case (0 when the group cannot share); a malformed one names no
+        // members, and the sequences it should have covered stay unspecified
+        const bool span_ok = s >= 0 && e >= s && e <= p.batch;
+        const bool ok = span_ok && e - s <= p.max_group && P >= 0 && P <= p.max_prefix && P % p.block_size == 0;
+        s_start = span_ok ? s : 0;
+        s_n = span_ok ? e - s : 0;
         s_prefix = ok ? P : 0;
         s_bad = !ok;
         if (reporter && ((grp == 0 && s != 0) || (grp == p.num_groups - 1 && e != p.batch)))
@@ -1300,6 +1331,7 @@ __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(const De
         const int L = clamp_len(p, b, false);
         int sp;
         ns = row_splits(p, L, seq_prefix_len(p, b, L), &sp);
+        if (sp > 0 && ns == sp + 1) ns = 1;  // pass 1 folded the prefix in and wrote the row
     }
     float m = -INFINITY, W = 0.f, acc[VPL];
 #pragma unroll
@@ -1638,7 +1670,9 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
                              : dispatch_group<float, 64>(G, p, grid, smem, st);
     }
     if (rc) return rc;
-    if (plan.max_splits > 1) {
+    // with shared prefixes, rows whose suffix is one split are finished by
+    // pass 1; the merge pass is needed only when a suffix can be split
+    if (p.num_groups > 0 ? plan.suffix_splits > 1 : plan.max_splits > 1) {
         const int64_t rows = (int64_t)batch * p.num_q_heads;
         // four warps per row, or all eight of a CTA when rows carry many splits
         // and there are too few rows to fill the GPU with four-warp groups

@@ -130,3 +130,84 @@ def test_bad_arguments(native):
         bm.append_token(7)
     with pytest.raises(native.OutOfBlocks):
         bm.append_token(7)
+
+
+def _check_groups(nat, order, starts, plens, mg, mp):
+    """The defining properties of the shared-prefix description."""
+    bs = nat.block_size
+    tables = [nat.block_table(s) for s in order]
+    lens = [nat.length(s) for s in order]
+    n = len(order)
+    assert starts[0] == 0 and starts[-1] == n and all(a < b for a, b in zip(starts[:-1], starts[1:]))
+    assert len(plens) == len(starts) - 1
+    assert mg == max(b - a for a, b in zip(starts[:-1], starts[1:])) and mp == max(plens)
+    for g, (a, e) in enumerate(zip(starts[:-1], starts[1:])):
+        members = range(a, e)
+        first = tables[a][0] if tables[a] else None
+        # members begin on the same block; the next group does not
+        if e - a > 1:
+            assert first is not None and all(tables[m] and tables[m][0] == first for m in members)
+        if e < n and first is not None and tables[e]:
+            assert tables[e][0] != first
+        # the prefix: whole blocks, equal in every member, full in every member, and maximal
+        P = int(plens[g])
+        k = P // bs
+        assert P % bs == 0
+        assert all(tables[m][:k] == tables[a][:k] and lens[m] >= P for m in members)
+        extendable = all(len(tables[m]) > k and len(tables[a]) > k and tables[m][k] == tables[a][k]
+                         and lens[m] >= (k + 1) * bs for m in members)
+        assert not extendable
+
+
+@pytest.mark.parametrize("bs", [1, 4, 16])
+def test_shared_prefix_groups_on_random_fork_trees(native, bs):
+    rng = np.random.default_rng(40 + bs)
+    nat = native.BlockManager(4000, bs)
+    seqs, next_id = [], 0
+    for prompt in range(12):
+        root = next_id
+        next_id += 1
+        nat.add_sequence(root)
+        for _ in range(int(rng.integers(0, 120))):
+            nat.append_token(root)
+        family = [root]
+        for _ in range(int(rng.integers(0, 6))):  # samples forked from the prompt or from each other
+            nat.fork(int(rng.choice(family)), next_id)
+            family.append(next_id)
+            next_id += 1
+        for _ in range(200):
+            nat.append_token(int(rng.choice(family)))
+        seqs += family
+    for trial in range(3):
+        order = list(seqs) if trial == 0 else [int(x) for x in rng.permutation(seqs)]
+        starts, plens, mg, mp = nat.shared_prefix_groups(order)
+        _check_groups(nat, order, starts.tolist(), plens.tolist(), mg, mp)
+
+
+def test_shared_prefix_groups_of_parallel_samples(native):
+    """3 prompts of 40 tokens (bs 16: 2 full blocks + 8 tokens) x 4 samples,
+    each sample then writing its own tokens: the samples of a prompt form a
+    group sharing the 32 tokens of the full prompt blocks (the partial block
+    is copied on the first write)."""
+    nat = native.BlockManager(200, 16)
+    order = []
+    for p in range(3):
+        root = 10 * p
+        nat.add_sequence(root)
+        for _ in range(40):
+            nat.append_token(root)
+        order.append(root)
+        for s in range(1, 4):
+            nat.fork(root, root + s)
+            order.append(root + s)
+    for s in order:
+        for _ in range(1 + s % 5):
+            nat.append_token(s)
+    starts, plens, mg, mp = nat.shared_prefix_groups(order)
+    assert starts.tolist() == [0, 4, 8, 12] and plens.tolist() == [32, 32, 32] and (mg, mp) == (4, 32)
+    _check_groups(nat, order, starts.tolist(), plens.tolist(), mg, mp)
+    # a sequence that shares nothing is a group of one with prefix 0
+    nat.add_sequence(99)
+    nat.append_token(99)
+    starts, plens, _, _ = nat.shared_prefix_groups(order[:4] + [99] + order[4:])
+    assert starts.tolist() == [0, 4, 5, 9, 13] and plens.tolist() == [32, 0, 32, 32]

@@ -158,3 +158,40 @@ def test_groups_that_do_not_cover_the_batch_are_flagged(pa):
     assert pa.pa_read_error_flag() == 5
     covered = list(range(short[-1]))
     assert_matches_oracle(out[covered], run_oracle(case)[covered], True, "covered sequences")
+
+
+def test_block_manager_groups_drive_the_shared_prefix_call(pa):
+    """Prompts forked into samples by the native block manager, each sample
+    then writing its own tokens (copy-on-write of the partial prompt block):
+    the manager's group description drives the shared-prefix call, which
+    matches the oracle walking every sample's own table."""
+    import numpy as np
+
+    from paged_kv_cache_355_b200.block_manager import BlockManager
+    from paged_kv_cache_355_b200.workloads import Workload, build_case
+
+    bs, Hkv, G, D = 16, 2, 4, 128
+    bm = BlockManager(900, bs)
+    rng = np.random.default_rng(5)
+    order = []
+    for p in range(5):
+        root = 100 * p
+        bm.add_sequence(root)
+        for _ in range(int(rng.integers(20, 400))):
+            bm.append_token(root)
+        order.append(root)
+        for s in range(1, int(rng.integers(1, 10))):
+            bm.fork(root, root + s)
+            order.append(root + s)
+    for s in order:
+        for _ in range(int(rng.integers(1, 60))):
+            bm.append_token(s)
+    starts, plens, mg, mp = bm.shared_prefix_groups(order)
+    assert mp > 0 and mg > 1
+    tables = [bm.block_table(s) for s in order]
+    lengths = [bm.length(s) for s in order]
+    w = Workload("bm", len(order), Hkv * G, Hkv, D, bs, torch.bfloat16, "fixed")
+    case = build_case(w, lengths, tables, 900, [], [], None, 77)
+    out = run_shared(pa, case, starts.tolist(), plens.tolist(), max_prefix=mp, max_group=mg)
+    assert_matches_oracle(out, run_oracle(case), True, "block-manager groups")
+    assert pa.pa_read_error_flag() == 0
