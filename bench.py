@@ -64,7 +64,10 @@ if ROOT not in sys.path:
 METRIC = "Paged decode attn: achieved HBM GB/s vs peak; decode tokens/s per batch"
 FALLBACK_HBM_GBS = 6650.0
 FLUSH_BYTES = 256 << 20
-SPIN_CYCLES = 2_000_000  # ~1 ms at 1.9 GHz
+# ~4 ms at 1.965 GHz.  With a 1 ms spin the step's first H2D copy measured
+# 0.126 ms instead of 0.038 ms on the B200 (the same copy with no spin, or
+# after a 4 ms one, takes 0.038-0.040 ms), which inflated the e2e time.
+SPIN_CYCLES = 8_000_000
 
 DESCRIPTIONS = {
     "tiny": "tiny: batch 4, lengths 1,7,16,33 (+1 appended), 4/4 heads, head_dim 64, block_size 16, fp32",
@@ -705,7 +708,7 @@ def run_ours(args):
     e2e_ev = []
     for i in range(args.warmup + args.steps):
         flush_l2()
-        # a 1 ms spin on the device before the start event: the host enqueues
+        # a 4 ms spin on the device before the start event: the host enqueues
         # the whole step (copies, API calls, read-back) while it runs, so the
         # events time the step's device work, not Python's issue rate
         torch.cuda._sleep(SPIN_CYCLES)

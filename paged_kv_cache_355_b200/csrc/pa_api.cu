@@ -2,6 +2,8 @@
 // strings, the version string and the per-device caches the entry points use.
 #include <cuda_runtime.h>
 
+#include <stdlib.h>
+
 #include <mutex>
 
 #include "pa.h"
@@ -41,6 +43,14 @@ int* error_word_ptr() {
     return g_error_ptr[dev];
 }
 
+bool nvtx_enabled() {
+    static const bool on = [] {
+        const char* v = getenv("PA_NVTX");
+        return v && v[0] == '1' && v[1] == 0;
+    }();
+    return on;
+}
+
 int num_sms() {
     const int dev = current_device();
     if (dev < 0) return 148;
@@ -70,6 +80,7 @@ __global__ void wait_selftest_kernel(int* err, uint64_t limit_ns) {
 }  // namespace pa
 
 extern "C" int pa_selftest_wait_timeout(uint32_t limit_us, void* stream) {
+    PA_NVTX_RANGE("pa_selftest_wait_timeout");
     if (limit_us == 0 || limit_us > 2000000u) return PA_ERR_INVALID_ARG;
     int* err = pa::error_word_ptr();
     if (!err) return PA_ERR_CUDA;
@@ -93,6 +104,7 @@ extern "C" const char* pa_status_string(int status) {
 extern "C" const char* pa_version(void) { return "0.1.0"; }
 
 extern "C" int pa_read_error_flag(void* stream) {
+    PA_NVTX_RANGE("pa_read_error_flag");
     int* err = pa::error_word_ptr();
     if (!err) return PA_ERR_CUDA;
     int value = 0;

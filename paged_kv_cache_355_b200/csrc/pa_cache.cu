@@ -203,6 +203,7 @@ using namespace pa;
 extern "C" int pa_slot_mapping(const int32_t* block_tables, int max_blocks_per_seq, int batch,
                                const int32_t* seq_ids, const int32_t* positions, int64_t num_tokens,
                                int block_size, int64_t* slot_mapping, void* stream) {
+    PA_NVTX_RANGE("pa_slot_mapping");
     if (num_tokens < 0 || batch < 0 || max_blocks_per_seq < 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
     if (num_tokens == 0) return PA_OK;
     if (!block_tables || !seq_ids || !positions || !slot_mapping) return PA_ERR_INVALID_ARG;
@@ -216,6 +217,7 @@ extern "C" int pa_slot_mapping(const int32_t* block_tables, int max_blocks_per_s
 extern "C" int pa_decode_slot_mapping(const int32_t* block_tables, int max_blocks_per_seq,
                                       const int32_t* context_lens, int batch, int block_size,
                                       int64_t* slot_mapping, void* stream) {
+    PA_NVTX_RANGE("pa_decode_slot_mapping");
     if (batch < 0 || max_blocks_per_seq < 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
     if (batch == 0) return PA_OK;
     if (!block_tables || !context_lens || !slot_mapping) return PA_ERR_INVALID_ARG;
@@ -230,6 +232,7 @@ extern "C" int pa_reshape_and_cache(const void* key, const void* value, void* k_
                                     const int64_t* slot_mapping, int64_t num_tokens, int num_kv_heads,
                                     int head_dim, int block_size, int64_t num_blocks, int dtype,
                                     void* stream) {
+    PA_NVTX_RANGE("pa_reshape_and_cache");
     if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks < 0 ||
         !valid_dtype(dtype))
         return PA_ERR_INVALID_ARG;
@@ -253,6 +256,7 @@ extern "C" int pa_reshape_and_cache_decode(const void* key, const void* value, v
                                            const int32_t* context_lens, int batch, int num_kv_heads, int head_dim,
                                            int block_size, int64_t num_blocks, int dtype, int64_t* slot_mapping,
                                            void* stream) {
+    PA_NVTX_RANGE("pa_reshape_and_cache_decode");
     if (batch < 0 || max_blocks_per_seq < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
         num_blocks < 0 || !valid_dtype(dtype))
         return PA_ERR_INVALID_ARG;
@@ -273,6 +277,7 @@ extern "C" int pa_reshape_and_cache_decode(const void* key, const void* value, v
 extern "C" int pa_copy_blocks(void* k_pool, void* v_pool, const int64_t* block_mapping, int64_t num_pairs,
                               int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, int dtype,
                               void* stream) {
+    PA_NVTX_RANGE("pa_copy_blocks");
     if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks < 0 ||
         !valid_dtype(dtype))
         return PA_ERR_INVALID_ARG;
@@ -288,6 +293,7 @@ extern "C" int pa_swap_blocks(const void* src_k, const void* src_v, void* dst_k,
                               const int64_t* block_mapping, int64_t num_pairs, int num_kv_heads, int head_dim,
                               int block_size, int64_t src_num_blocks, int64_t dst_num_blocks, int dtype,
                               void* stream) {
+    PA_NVTX_RANGE("pa_swap_blocks");
     if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || src_num_blocks < 0 ||
         dst_num_blocks < 0 || !valid_dtype(dtype))
         return PA_ERR_INVALID_ARG;

@@ -1737,6 +1737,7 @@ extern "C" int pa_paged_attention_decode(const void* q, const void* k_pool, cons
                                          int num_kv_heads, int head_dim, int64_t num_blocks, int kv_dtype,
                                          int partition_size, void* workspace, size_t workspace_bytes,
                                          void* stream) {
+    PA_NVTX_RANGE("pa_paged_attention_decode");
     int rc = check_shapes(batch, num_q_heads, num_kv_heads, head_dim, block_size, kv_dtype, out_dtype,
                           max_context_len);
     if (rc) return rc;
@@ -1773,6 +1774,7 @@ extern "C" int pa_paged_attention_decode_append(const void* q, const void* key, 
                                                 int num_kv_heads, int head_dim, int64_t num_blocks, int kv_dtype,
                                                 int partition_size, void* workspace, size_t workspace_bytes,
                                                 int64_t* slot_mapping, void* stream) {
+    PA_NVTX_RANGE("pa_paged_attention_decode_append");
     int rc = check_shapes(batch, num_q_heads, num_kv_heads, head_dim, block_size, kv_dtype, out_dtype,
                           max_context_len);
     if (rc) return rc;
@@ -1842,6 +1844,7 @@ extern "C" int pa_paged_attention_decode_shared_prefix(
     int batch, int num_q_heads, int num_kv_heads, int head_dim, int64_t num_blocks, int kv_dtype,
     const int32_t* group_starts, const int32_t* group_prefix_lens, int num_groups, int max_group_size,
     int max_prefix_len, int partition_size, void* workspace, size_t workspace_bytes, void* stream) {
+    PA_NVTX_RANGE("pa_paged_attention_decode_shared_prefix");
     int rc = check_shapes(batch, num_q_heads, num_kv_heads, head_dim, block_size, kv_dtype, out_dtype,
                           max_context_len);
     if (rc) return rc;
@@ -1886,6 +1889,7 @@ extern "C" int pa_paged_attention_decode_contiguous(const void* q, const void* k
                                                     int num_q_heads, int num_kv_heads, int head_dim, int kv_dtype,
                                                     int partition_size, void* workspace, size_t workspace_bytes,
                                                     void* stream) {
+    PA_NVTX_RANGE("pa_paged_attention_decode_contiguous");
     int rc = check_shapes(batch, num_q_heads, num_kv_heads, head_dim, block_size, kv_dtype, out_dtype,
                           max_context_len);
     if (rc) return rc;

@@ -5,11 +5,28 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <utility>
 
 #include "pa.h"
 
 namespace pa {
+
+// NVTX ranges around the entry points that launch work, for timeline
+// profilers: on when the environment has PA_NVTX=1 (read once per process),
+// otherwise one predictable branch per call.
+bool nvtx_enabled();
+
+struct NvtxRange {
+    bool on;
+    explicit NvtxRange(const char* name) : on(nvtx_enabled()) {
+        if (on) nvtxRangePushA(name);
+    }
+    ~NvtxRange() {
+        if (on) nvtxRangePop();
+    }
+};
 
 // Device address of the current device's error word (resolved once per
 // device with cudaGetSymbolAddress).  NULL if the lookup failed.
@@ -58,3 +75,5 @@ inline int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
 }
 
 }  // namespace pa
+
+#define PA_NVTX_RANGE(name) ::pa::NvtxRange pa_nvtx_range_(name)

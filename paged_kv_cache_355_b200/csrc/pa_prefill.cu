@@ -615,6 +615,7 @@ extern "C" int pa_paged_attention_prefill(const void* q, const void* k_pool, con
                                           int out_dtype, int batch, int num_q_heads, int num_kv_heads,
                                           int head_dim, int64_t num_tokens, int64_t num_blocks, int kv_dtype,
                                           void* stream) {
+    PA_NVTX_RANGE("pa_paged_attention_prefill");
     if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
         max_query_len < 0 || num_tokens < 0 || num_blocks < 0 || max_blocks_per_seq < 0 || !valid_dtype(kv_dtype) ||
         !valid_dtype(out_dtype) || num_q_heads % num_kv_heads != 0)

@@ -57,6 +57,7 @@ __global__ void __launch_bounds__(32) hbm_read_probe_kernel(const uint8_t* __res
 }  // namespace pa
 
 extern "C" int pa_hbm_read_probe(const void* buffer, size_t bytes, void* stream) {
+    PA_NVTX_RANGE("pa_hbm_read_probe");
     if (bytes == 0) return PA_OK;
     if (!buffer || !pa::aligned16(buffer) || bytes % 16 != 0) return PA_ERR_INVALID_ARG;
     int* err = pa::error_word_ptr();

@@ -26,6 +26,7 @@
 #include <mutex>
 
 #include "pa.h"
+#include "pa_internal.h"
 
 namespace pa {
 namespace {
@@ -62,6 +63,7 @@ extern "C" int pa_paged_attention_decode_static_scratch(
     const int32_t* context_lens, int max_context_len, float scale, int block_size, void* out, int out_dtype,
     int batch, int num_q_heads, int num_kv_heads, int head_dim, int64_t num_blocks, int kv_dtype, int partition_size,
     void* stream) {
+    PA_NVTX_RANGE("pa_paged_attention_decode_static_scratch");
     size_t need = 0;
     int rc = pa_paged_attention_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, max_context_len,
                                                block_size, partition_size, &need);

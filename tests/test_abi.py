@@ -187,3 +187,22 @@ def test_shared_prefix_workspace_size(lib):
     assert sz.value == -(-rows * 128 * 4 // 256) * 256 + -(-rows * 2 * 4 // 256) * 256 + 256
     assert f(4, 8, 2, 128, 100, 16, 0, 2, 64, 128, ctypes.byref(sz)) == INVALID
     assert f(4, 8, 2, 128, 100, 16, 2, 2, 101, 128, ctypes.byref(sz)) == INVALID
+
+
+def test_nvtx_ranges_leave_the_calls_unchanged(lib):
+    """With PA_NVTX=1 every launching entry point opens and closes an NVTX
+    range; with no profiler attached that changes nothing the caller sees."""
+    import subprocess
+    import sys
+
+    code = ("import ctypes; lib = ctypes.CDLL(%r); P = ctypes.c_void_p; "
+            "lib.pa_hbm_read_probe.argtypes = [P, ctypes.c_size_t, P]; "
+            "print(lib.pa_hbm_read_probe(P(24), 16, None), lib.pa_hbm_read_probe(P(16), 0, None), "
+            "lib.pa_copy_blocks(P(16), P(16), P(0), ctypes.c_int64(3), 2, 128, 16, ctypes.c_int64(8), 1, None))"
+            % os.path.join(ROOT, "paged_kv_cache_355_b200", "libpa.so"))
+    outs = []
+    for flag in ("0", "1"):
+        env = dict(os.environ, PA_NVTX=flag)
+        outs.append(subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                                   check=True).stdout.split())
+    assert outs[0] == outs[1] == [str(INVALID), str(OK), str(INVALID)]
