@@ -172,12 +172,15 @@ __device__ __forceinline__ int clamp_len(const DecodeParams& p, int b, bool repo
 // shared prefixes), clamped to [0, min(L, max_prefix)] and to whole blocks, so
 // that a value left unwritten under a violated precondition can never send
 // pass 1 or the merge outside the table or the partial-result slots.
-__device__ __forceinline__ int seq_prefix_len(const DecodeParams& p, int b, int L) {
+__device__ __forceinline__ int clamp_prefix(const DecodeParams& p, int v, int L) {
     if (!p.seq_prefix) return 0;
-    int v = p.seq_prefix[b];
     const int hi = L < p.max_prefix ? L : p.max_prefix;
     v = v < 0 ? 0 : (v > hi ? hi : v);
     return v - v % p.block_size;
+}
+
+__device__ __forceinline__ int seq_prefix_len(const DecodeParams& p, int b, int L) {
+    return p.seq_prefix ? clamp_prefix(p, p.seq_prefix[b], L) : 0;
 }
 
 // Partial-result slots of sequence b (prefix splits, then suffix splits; at
@@ -197,17 +200,113 @@ __device__ __forceinline__ void store_out(const DecodeParams& p, int64_t idx, fl
         static_cast<float*>(p.out)[idx] = v;
 }
 
+// Prefix splits that pass 1 folds into a row itself (more are left to the
+// merge pass).
+constexpr int kMaxFoldSplits = 16;
+
+// A row whose only other splits are prefix splits (written by the prefix
+// pass, which has completed) is finished in pass 1: the prefix partials are
+// combined with the CTA's own state by the log-sum-exp rescale the merge
+// pass applies.  First the rows' coefficients (one thread per row, all
+// (m, l) loads issued together), then the output elements, four per thread
+// at a time with all their partial-row loads issued before any is used.
+__device__ __forceinline__ void fold_prefix_and_store(const DecodeParams& p, const float* sm_o, const float* sm_m,
+                                                      const float* sm_l, float* coef, int G, int D, int b, int kvh,
+                                                      int sp) {
+    constexpr int K = kMaxFoldSplits;
+    for (int h = threadIdx.x; h < G; h += blockDim.x) {
+        const int64_t qrow = (int64_t)b * p.num_q_heads + (int64_t)kvh * G + h;
+        const float* ml = p.part_ml + qrow * p.max_splits * 2;
+        float mv[K], lv[K];
+#pragma unroll
+        for (int s = 0; s < K; ++s) {
+            mv[s] = s < sp ? ml[2 * s] : -INFINITY;
+            lv[s] = s < sp ? ml[2 * s + 1] : 0.f;
+        }
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_m[w * G + h]);
+        float lt = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) {
+                const float mw = sm_m[w * G + h];
+                lt += mw == -INFINITY ? 0.f : sm_l[w * G + h] * exp2f(mw - M);
+            }
+        }
+        float Mt = M;
+#pragma unroll
+        for (int s = 0; s < K; ++s) Mt = fmaxf(Mt, mv[s]);
+        float W = 0.f, own = 0.f, ws[K];
+#pragma unroll
+        for (int s = 0; s < K; ++s) ws[s] = 0.f;
+        if (Mt != -INFINITY) {
+            if (M != -INFINITY) {
+                own = exp2f(M - Mt);
+                W = lt * own;
+            }
+#pragma unroll
+            for (int s = 0; s < K; ++s) {
+                ws[s] = mv[s] == -INFINITY ? 0.f : lv[s] * exp2f(mv[s] - Mt);
+                W += ws[s];
+            }
+        }
+        const float inv = W > 0.f ? 1.f / W : 0.f;
+        coef[h * (K + 1)] = own * inv;
+#pragma unroll
+        for (int s = 0; s < K; ++s) coef[h * (K + 1) + 1 + s] = ws[s] * inv;
+    }
+    __syncthreads();
+    constexpr int E = 4;
+    for (int base = threadIdx.x; base < G * D; base += E * blockDim.x) {
+        float pv[E][K];
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int idx = base + e * blockDim.x;
+            const int h = idx / D;
+            const int d = idx - h * D;
+            const float* po = p.part_o + ((int64_t)b * p.num_q_heads + (int64_t)kvh * G + h) * p.max_splits * D + d;
+#pragma unroll
+            for (int s = 0; s < K; ++s) pv[e][s] = (idx < G * D && s < sp) ? po[(int64_t)s * D] : 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int idx = base + e * blockDim.x;
+            if (idx >= G * D) break;
+            const int h = idx / D;
+            const int d = idx - h * D;
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_m[w * G + h]);
+            float ot = 0.f;
+            if (M != -INFINITY) {
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) {
+                    const float mw = sm_m[w * G + h];
+                    ot += mw == -INFINITY ? 0.f : sm_o[(w * G + h) * D + d] * exp2f(mw - M);
+                }
+            }
+            float acc = ot * coef[h * (K + 1)];
+#pragma unroll
+            for (int s = 0; s < K; ++s) acc = fmaf(coef[h * (K + 1) + 1 + s], pv[e][s], acc);
+            store_out(p, ((int64_t)b * p.num_q_heads + (int64_t)kvh * G + h) * D + d, acc);
+        }
+    }
+}
+
 // Combine the consumer warps' (m, l, o) states of one work item, held in
 // shared memory as o[w][h][d], m[w][h], l[w][h], and write the final row (one
-// split) or the normalised partial row plus (m, l) for the merge kernel.
-// When the row's only other splits are prefix splits (written by the prefix
-// pass, which has completed), the row is finished here: the prefix partials
-// are folded in with the same log-sum-exp rescale the merge pass applies, and
-// the merge pass skips the row.
+// split) or the normalised partial row plus (m, l) for the merge kernel; with
+// prefix splits and one own split, fold the prefix in (above).  `coef` is
+// shared scratch of G * (kMaxFoldSplits + 1) floats.
 __device__ __forceinline__ void merge_warps_and_store(const DecodeParams& p, const float* sm_o, const float* sm_m,
                                                       const float* sm_l, int G, int D, int b, int kvh, int split,
-                                                      int num_splits_b, int prefix_splits = 0) {
-    const bool fold_prefix = prefix_splits > 0 && num_splits_b == prefix_splits + 1;
+                                                      int num_splits_b, int prefix_splits = 0,
+                                                      float* coef = nullptr) {
+    if (coef && prefix_splits > 0 && prefix_splits <= kMaxFoldSplits && num_splits_b == prefix_splits + 1) {
+        fold_prefix_and_store(p, sm_o, sm_m, sm_l, coef, G, D, b, kvh, prefix_splits);
+        return;
+    }
     for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
         const int h = idx / D;
         const int d = idx - h * D;
@@ -224,31 +323,8 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeParams& p, con
                 ot += sm_o[(w * G + h) * D + d] * a;
             }
         }
-        const int64_t qrow = (int64_t)b * p.num_q_heads + (int64_t)kvh * G + h;
-        if (fold_prefix) {
-            const float* ml = p.part_ml + qrow * p.max_splits * 2;
-            const float* po = p.part_o + qrow * p.max_splits * D + d;
-            float Mt = M;
-            for (int s = 0; s < prefix_splits; ++s) Mt = fmaxf(Mt, ml[2 * s]);
-            float W = 0.f, acc = 0.f;
-            if (Mt != -INFINITY) {
-                if (M != -INFINITY) {
-                    const float a = exp2f(M - Mt);
-                    W = lt * a;
-                    acc = ot * a;
-                }
-                for (int s = 0; s < prefix_splits; ++s) {
-                    const float ms = ml[2 * s];
-                    if (ms == -INFINITY) continue;
-                    const float w = ml[2 * s + 1] * exp2f(ms - Mt);
-                    W += w;
-                    acc = fmaf(w, po[(int64_t)s * D], acc);
-                }
-            }
-            store_out(p, qrow * D + d, W > 0.f ? acc / W : 0.f);
-            continue;
-        }
         const float val = lt > 0.f ? ot / lt : 0.f;
+        const int64_t qrow = (int64_t)b * p.num_q_heads + (int64_t)kvh * G + h;
         if (num_splits_b == 1) {
             store_out(p, qrow * D + d, val);
         } else {
@@ -284,14 +360,29 @@ __device__ __forceinline__ int schedule_sequence(const DecodeParams& p, uint8_t*
     for (int k = tid; k < 64; k += blockDim.x) hist[k] = 0;
     if (tid == 0) s_seq = rank;
     __syncthreads();
-    for (int b = tid; b < p.batch; b += blockDim.x) {
-        int L = p.context_lens[b];
-        L = L < 0 ? 0 : ((int64_t)L > p.max_len ? (int)p.max_len : L);
-        L -= seq_prefix_len(p, b, L);  // the tokens this pass reads
-        int k = (int)(((int64_t)L * 64) / (p.max_len + 1));
-        k = 63 - (k > 63 ? 63 : k);  // longer sequences get lower keys
-        key[b] = (uint8_t)k;
-        atomicAdd(&hist[k], 1);
+    // the loads of four sequences per thread are issued before any is used:
+    // one memory round trip for batches up to four times the block size
+    constexpr int U = 4;
+    for (int b0 = tid; b0 < p.batch; b0 += U * blockDim.x) {
+        int lv[U], pv[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int b = b0 + u * blockDim.x;
+            lv[u] = b < p.batch ? p.context_lens[b] : 0;
+            pv[u] = (b < p.batch && p.seq_prefix) ? p.seq_prefix[b] : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int b = b0 + u * blockDim.x;
+            if (b >= p.batch) break;
+            int L = lv[u];
+            L = L < 0 ? 0 : ((int64_t)L > p.max_len ? (int)p.max_len : L);
+            L -= clamp_prefix(p, pv[u], L);  // the tokens this pass reads
+            int k = (int)(((int64_t)L * 64) / (p.max_len + 1));
+            k = 63 - (k > 63 ? 63 : k);  // longer sequences get lower keys
+            key[b] = (uint8_t)k;
+            atomicAdd(&hist[k], 1);
+        }
     }
     __syncthreads();
     if (tid < 32) {
@@ -913,16 +1004,26 @@ __global__ void __launch_bounds__(kDecodeThreads)
                         bl[nt][half] = movmatrix_trans(lo);
                     }
                 }
+                // two row tiles at a time: both high-part MMAs, then both
+                // residual ones, so no MMA waits on the one just issued into
+                // the same accumulator
 #pragma unroll
-                for (int mt = 0; mt < KSTEPS; ++mt) {
-                    const uint32_t slab = vst + (mt >> 2) * SLAB_BYTES;
-                    const int chunk = (mt & 3) * 2 + (q4 & 1);
-                    uint32_t a[4];
-                    ldmatrix_x4_trans(swizzled(slab, 16 * ks + r8 + 8 * (q4 >> 1), chunk), a[0], a[1], a[2], a[3]);
+                for (int mp = 0; mp < KSTEPS; mp += 2) {
+                    uint32_t a[2][4];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int mt = mp + u;
+                        const uint32_t slab = vst + (mt >> 2) * SLAB_BYTES;
+                        const int chunk = (mt & 3) * 2 + (q4 & 1);
+                        ldmatrix_x4_trans(swizzled(slab, 16 * ks + r8 + 8 * (q4 >> 1), chunk), a[u][0], a[u][1],
+                                          a[u][2], a[u][3]);
+                    }
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        mma_bf16_16816(o[mt][nt], a, bh[nt][0], bh[nt][1]);
-                        mma_bf16_16816(o[mt][nt], a, bl[nt][0], bl[nt][1]);
+                        mma_bf16_16816(o[mp][nt], a[0], bh[nt][0], bh[nt][1]);
+                        mma_bf16_16816(o[mp + 1][nt], a[1], bh[nt][0], bh[nt][1]);
+                        mma_bf16_16816(o[mp][nt], a[0], bl[nt][0], bl[nt][1]);
+                        mma_bf16_16816(o[mp + 1][nt], a[1], bl[nt][0], bl[nt][1]);
                     }
                 }
             }
@@ -971,7 +1072,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
         }
     }
     __syncthreads();
-    merge_warps_and_store(p, sm_o, sm_m, sm_l, G, D, b, kvh, prefix_splits + split, num_splits_b, prefix_splits);
+    merge_warps_and_store(p, sm_o, sm_m, sm_l, G, D, b, kvh, prefix_splits + split, num_splits_b, prefix_splits,
+                          sm_l + kConsumerWarps * G);
 }
 
 // ---------------------------------------------------------------------------
@@ -989,20 +1091,28 @@ __global__ void __launch_bounds__(kDecodeThreads)
 //  * Query rows r = member * G + head are the M side of mma.sync m16n8k16:
 //        S[rows, tokens] = Q[rows, D] . K^T[D, tokens]
 //        O[rows, D]     += P[rows, tokens] . V[tokens, D]
-//    Consumer warp w owns rows 16 w .. 16 w + 15 of the CTA's chunk and reads
-//    every stage; P goes from the S accumulators straight into A fragments
-//    (the two layouts coincide), split into bf16 high and residual parts as
-//    in pass 1.  MT consumer warps cover 16 MT rows; larger groups take
-//    several row chunks (blockIdx.y / Hkv).
-//  * Each warp finishes its own rows: the normalised partial row and (m, l)
-//    go to the prefix split's slot for the merge pass.  CTA (0, 0, g) also
-//    checks the group's description and stores each member's prefix length
-//    in seq_prefix for pass 1 and the merge; a description that breaks the
-//    preconditions is flagged and its group falls back to prefix 0 (pass 1
-//    then covers the whole sequences).
+//    P goes from the S accumulators straight into A fragments (the two
+//    layouts coincide), split into bf16 high and residual parts as in pass 1.
+//  * The CTA's 16 MT query rows are staged once in shared memory (128-byte
+//    swizzle, read by ldmatrix), which keeps registers for two CTAs' worth of
+//    latency hiding.  Consumer warp (tile t, parity q) owns rows 16 t ..
+//    16 t + 15 and the stages j with j % PAR == q: PAR groups of MT warps
+//    work on alternate stages, and at the end each group's (m, l, o) is
+//    combined with the others' through shared memory (same lane layout, so
+//    lane by lane).  Larger groups take several row chunks (blockIdx.y / Hkv).
+//  * The first consumer group writes its rows' normalised partial and (m, l)
+//    to the prefix split's slot for pass 1 (which folds them into the row) or
+//    the merge pass.  CTA (0, 0, g) also checks the group's description and
+//    stores each member's prefix length in seq_prefix; a description that
+//    breaks the preconditions is flagged and its group falls back to prefix 0
+//    (pass 1 then covers the whole sequences).
 // ---------------------------------------------------------------------------
-template <int D, int MT>
-__global__ void __launch_bounds__(32 * (1 + MT))
+__device__ __forceinline__ void consumer_barrier(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+template <int D, int MT, int PAR>
+__global__ void __launch_bounds__(32 * (1 + MT * PAR), 3)
     decode_prefix_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
                              const __grid_constant__ CUtensorMap tmv) {
     constexpr int SLABS = D / 64;
@@ -1011,12 +1121,15 @@ __global__ void __launch_bounds__(32 * (1 + MT))
     constexpr int KSTEPS = D / 16;
     constexpr int NTD = D / 8;  // 8-column tiles of the output row
     constexpr int ROWS = 16 * MT;
+    constexpr int QSLAB = ROWS * 128;  // bytes of one 64-column slab of the Q tile
+    constexpr int CONSUMERS = 32 * MT * PAR;
 
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + p.stages;
     int32_t* tbl = reinterpret_cast<int32_t*>(empty + p.stages);
     uint8_t* ring = smem + p.ring_offset + ((1024u - (smem_addr(smem) & 1023u)) & 1023u);
+    uint8_t* qtile = ring + (size_t)p.stages * 2 * STAGE_BYTES;  // [SLABS][ROWS][128 B], swizzled
     __shared__ int s_start, s_n, s_prefix, s_bad;
 
     if (threadIdx.x == 0) {
@@ -1079,6 +1192,19 @@ __global__ void __launch_bounds__(32 * (1 + MT))
         const int nblk = (ntok + p.block_size - 1) / p.block_size;
         const int32_t* row = p.block_tables + (int64_t)s_start * p.max_blocks_per_seq + first_blk;
         for (int i = threadIdx.x; i < nblk; i += blockDim.x) tbl[i] = row[i];
+        // the chunk's query rows (zero past the group), 16-byte chunk c of
+        // row r of a slab at chunk c ^ (r & 7)
+        const uint16_t* qv = static_cast<const uint16_t*>(p.q);
+        for (int i = threadIdx.x; i < ROWS * (D / 8); i += blockDim.x) {
+            const int r = i / (D / 8);
+            const int c = i % (D / 8);
+            const int gr = row0 + r;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (gr < rows_total)
+                v = *reinterpret_cast<const uint4*>(
+                    qv + ((int64_t)(s_start + gr / G) * p.num_q_heads + (int64_t)kvh * G + gr % G) * D + c * 8);
+            *reinterpret_cast<uint4*>(qtile + (c >> 3) * QSLAB + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
+        }
     }
     __syncthreads();
 
@@ -1100,8 +1226,9 @@ __global__ void __launch_bounds__(32 * (1 + MT))
             const int t0 = j * kStageTokens;
             const int rows = min(kStageTokens, ntok - t0);
             if (rows < kStageTokens) {
-                // every consumer reads this stage: the producer zeroes the V
-                // rows past the prefix (0-weight * stale NaN would be NaN)
+                // every consumer of this stage reads all its rows: the
+                // producer zeroes the V rows past the prefix (0-weight * stale
+                // NaN would be NaN)
                 const int nchunks = (kStageTokens - rows) * SLABS * 8;
                 for (int c = lane; c < nchunks; c += 32) {
                     const int row = rows + c / (SLABS * 8);
@@ -1140,30 +1267,14 @@ __global__ void __launch_bounds__(32 * (1 + MT))
 
     // ---------------- consumers ----------------
     const int cw = warp - 1;
-    const int g = lane >> 2;  // fragment row group
-    const int t = lane & 3;   // fragment column pair
+    const int mtile = cw % MT;  // 16-row tile of the chunk
+    const int par = cw / MT;    // stages j with j % PAR == par
+    const int g = lane >> 2;    // fragment row group
+    const int t = lane & 3;     // fragment column pair
     const int q4 = lane >> 3;
     const int r8 = lane & 7;
-    const int rbase = row0 + 16 * cw;
-    // Q A-fragments of rows rbase + g and rbase + g + 8 (zero past the group)
-    uint32_t qa[KSTEPS][4];
-    {
-        const uint16_t* qv = static_cast<const uint16_t*>(p.q);
-        const uint16_t* qrow[2] = {nullptr, nullptr};
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const int r = rbase + g + 8 * i;
-            if (r < rows_total)
-                qrow[i] = qv + ((int64_t)(s_start + r / G) * p.num_q_heads + (int64_t)kvh * G + r % G) * D;
-        }
-#pragma unroll
-        for (int kk = 0; kk < KSTEPS; ++kk) {
-            qa[kk][0] = qrow[0] ? *reinterpret_cast<const uint32_t*>(qrow[0] + kk * 16 + 2 * t) : 0u;
-            qa[kk][1] = qrow[1] ? *reinterpret_cast<const uint32_t*>(qrow[1] + kk * 16 + 2 * t) : 0u;
-            qa[kk][2] = qrow[0] ? *reinterpret_cast<const uint32_t*>(qrow[0] + kk * 16 + 8 + 2 * t) : 0u;
-            qa[kk][3] = qrow[1] ? *reinterpret_cast<const uint32_t*>(qrow[1] + kk * 16 + 8 + 2 * t) : 0u;
-        }
-    }
+    const int rbase = row0 + 16 * mtile;
+    const uint32_t qbase = smem_addr(qtile);
     float o[NTD][4];
 #pragma unroll
     for (int nd = 0; nd < NTD; ++nd)
@@ -1171,7 +1282,7 @@ __global__ void __launch_bounds__(32 * (1 + MT))
         for (int c = 0; c < 4; ++c) o[nd][c] = 0.f;
     float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
     bool aborted = false;
-    for (int j = 0; j < nstage; ++j) {
+    for (int j = par; j < nstage; j += PAR) {
         const int slot = j % p.stages;
         if (!mbar_wait(&full[slot], (j / p.stages) & 1, p.err)) {
             aborted = true;
@@ -1180,24 +1291,43 @@ __global__ void __launch_bounds__(32 * (1 + MT))
         const uint32_t kst = smem_addr(ring + (size_t)slot * 2 * STAGE_BYTES);
         const uint32_t vst = kst + STAGE_BYTES;
         const int valid = min(kStageTokens, ntok - j * kStageTokens);
-        // S = Q . K^T over the stage's 32 tokens: four 8-token column tiles
-        float s[4][4];
+        // S = Q . K^T over the stage's 32 tokens: four 8-token column tiles;
+        // the head dimension in two halves with their own accumulators, so
+        // each MMA waits on the one eight issues back, not four
+        float s[4][4], s2[4][4];
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) s[nt][c] = 0.f;
+            for (int c = 0; c < 4; ++c) s[nt][c] = s2[nt][c] = 0.f;
 #pragma unroll
-        for (int kk = 0; kk < KSTEPS; ++kk) {
-            const uint32_t slab = kst + (kk >> 2) * SLAB_BYTES;
-            const int chunk16 = (kk & 3) * 2 + (q4 & 1);
+        for (int kh = 0; kh < KSTEPS / 2; ++kh) {
+            uint32_t a[2][4], b[2][2][4];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int kk = kh + half * (KSTEPS / 2);
+                // Q rows 16 mtile + {0..15}, columns 16 kk .. 16 kk + 15
+                ldmatrix_x4(swizzled(qbase + (kk >> 2) * QSLAB, 16 * mtile + r8 + 8 * (q4 & 1),
+                                     (kk & 3) * 2 + (q4 >> 1)),
+                            a[half][0], a[half][1], a[half][2], a[half][3]);
+                const uint32_t slab = kst + (kk >> 2) * SLAB_BYTES;
+                const int chunk16 = (kk & 3) * 2 + (q4 & 1);
+#pragma unroll
+                for (int pair = 0; pair < 2; ++pair)
+                    ldmatrix_x4(swizzled(slab, 8 * (2 * pair + (q4 >> 1)) + r8, chunk16), b[half][pair][0],
+                                b[half][pair][1], b[half][pair][2], b[half][pair][3]);
+            }
 #pragma unroll
             for (int pair = 0; pair < 2; ++pair) {
-                uint32_t b[4];
-                ldmatrix_x4(swizzled(slab, 8 * (2 * pair + (q4 >> 1)) + r8, chunk16), b[0], b[1], b[2], b[3]);
-                mma_bf16_16816(s[2 * pair], qa[kk], b[0], b[1]);
-                mma_bf16_16816(s[2 * pair + 1], qa[kk], b[2], b[3]);
+                mma_bf16_16816(s[2 * pair], a[0], b[0][pair][0], b[0][pair][1]);
+                mma_bf16_16816(s[2 * pair + 1], a[0], b[0][pair][2], b[0][pair][3]);
+                mma_bf16_16816(s2[2 * pair], a[1], b[1][pair][0], b[1][pair][1]);
+                mma_bf16_16816(s2[2 * pair + 1], a[1], b[1][pair][2], b[1][pair][3]);
             }
         }
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) s[nt][c] += s2[nt][c];
         // online softmax per row (this lane: rows g and g + 8, tokens
         // 8 nt + 2 t and 8 nt + 2 t + 1), log2 domain, masked past the prefix
         float alpha[2];
@@ -1258,20 +1388,70 @@ __global__ void __launch_bounds__(32 * (1 + MT))
                 ah[f] = pack_bf16x2(p0, p1);
                 al[f] = pack_bf16x2(p0 - bf16_lo_to_f32(ah[f]), p1 - bf16_hi_to_f32(ah[f]));
             }
+            // four column-tile pairs at a time: their eight high-part MMAs,
+            // then the eight residual ones, so no MMA waits on the one just
+            // issued into the same accumulator
 #pragma unroll
-            for (int ndp = 0; ndp < NTD / 2; ++ndp) {
-                const int nd = 2 * ndp + (q4 >> 1);
-                uint32_t b[4];
-                ldmatrix_x4_trans(swizzled(vst + (nd >> 3) * SLAB_BYTES, 16 * ks + 8 * (q4 & 1) + r8, nd & 7), b[0],
-                                  b[1], b[2], b[3]);
-                mma_bf16_16816(o[2 * ndp], ah, b[0], b[1]);
-                mma_bf16_16816(o[2 * ndp], al, b[0], b[1]);
-                mma_bf16_16816(o[2 * ndp + 1], ah, b[2], b[3]);
-                mma_bf16_16816(o[2 * ndp + 1], al, b[2], b[3]);
+            for (int ng = 0; ng < NTD / 8; ++ng) {
+                uint32_t b[4][4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int nd = 2 * (4 * ng + u) + (q4 >> 1);
+                    ldmatrix_x4_trans(swizzled(vst + (nd >> 3) * SLAB_BYTES, 16 * ks + 8 * (q4 & 1) + r8, nd & 7),
+                                      b[u][0], b[u][1], b[u][2], b[u][3]);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    mma_bf16_16816(o[2 * (4 * ng + u)], ah, b[u][0], b[u][1]);
+                    mma_bf16_16816(o[2 * (4 * ng + u) + 1], ah, b[u][2], b[u][3]);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    mma_bf16_16816(o[2 * (4 * ng + u)], al, b[u][0], b[u][1]);
+                    mma_bf16_16816(o[2 * (4 * ng + u) + 1], al, b[u][2], b[u][3]);
+                }
             }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[slot]);
+    }
+    if (PAR > 1) {
+        // combine the parity groups lane by lane through the (drained) ring:
+        // every consumer has finished its stages before anything is written
+        consumer_barrier(1, CONSUMERS);
+        constexpr int REC = NTD * 4 + 4;  // floats per lane: o, m[2], l[2]
+        float* xch = reinterpret_cast<float*>(ring);
+        if (par > 0) {
+            float* dst = xch + ((size_t)((par - 1) * MT + mtile) * 32 + lane) * REC;
+#pragma unroll
+            for (int nd = 0; nd < NTD; ++nd)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) dst[nd * 4 + c] = o[nd][c];
+            dst[NTD * 4] = m[0];
+            dst[NTD * 4 + 1] = m[1];
+            dst[NTD * 4 + 2] = l[0];
+            dst[NTD * 4 + 3] = l[1];
+        }
+        consumer_barrier(1, CONSUMERS);
+        if (par > 0) return;
+#pragma unroll
+        for (int q = 1; q < PAR; ++q) {
+            const float* src = xch + ((size_t)((q - 1) * MT + mtile) * 32 + lane) * REC;
+            float a0[2], a1[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const float mq = src[NTD * 4 + i];
+                const float M = fmaxf(m[i], mq);
+                a0[i] = m[i] == -INFINITY ? 0.f : exp2f(m[i] - M);
+                a1[i] = mq == -INFINITY ? 0.f : exp2f(mq - M);
+                l[i] = l[i] * a0[i] + src[NTD * 4 + 2 + i] * a1[i];
+                m[i] = M;
+            }
+#pragma unroll
+            for (int nd = 0; nd < NTD; ++nd)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) o[nd][c] = o[nd][c] * a0[c >> 1] + src[nd * 4 + c] * a1[c >> 1];
+        }
     }
     if (aborted) return;
     // l was summed per lane over its own columns: add the quad's four lanes
@@ -1331,7 +1511,7 @@ __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(const De
         const int L = clamp_len(p, b, false);
         int sp;
         ns = row_splits(p, L, seq_prefix_len(p, b, L), &sp);
-        if (sp > 0 && ns == sp + 1) ns = 1;  // pass 1 folded the prefix in and wrote the row
+        if (sp > 0 && sp <= kMaxFoldSplits && ns == sp + 1) ns = 1;  // pass 1 folded the prefix in and wrote the row
     }
     float m = -INFINITY, W = 0.f, acc[VPL];
 #pragma unroll
@@ -1448,10 +1628,11 @@ int auto_partition(int batch, int num_q_heads, int num_kv_heads, int max_context
 }
 
 // Tokens per prefix split: as long as possible (4096) while the prefix pass
-// still has at least two CTAs per SM to run, halved down to 256 otherwise.
+// still has at least four CTAs per SM to run, halved down to 256 otherwise
+// (its consumer warps read every stage, so it needs CTAs to hide latency).
 int auto_prefix_partition(int num_groups, int num_kv_heads, int chunks, int max_prefix_len) {
     int P = kMaxAutoPartition;
-    const int64_t want = 2ll * num_sms();
+    const int64_t want = 4ll * num_sms();
     const int64_t L = max_prefix_len > 0 ? max_prefix_len : 1;
     while (P > kMinPrefixPartition && (int64_t)num_groups * num_kv_heads * chunks * ((L + P - 1) / P) < want) P /= 2;
     return P;
@@ -1535,7 +1716,7 @@ int launch_pass1_mma(const DecodeParams& p, const CUtensorMap& tmk, const CUtens
     return launch_pdl(decode_pass1_mma_kernel<D, NT>, grid, dim3(kDecodeThreads), smem, st, p, tmk, tmv);
 }
 
-template <int D, int MT>
+template <int D, int MT, int PAR>
 int launch_prefix_mma(const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, dim3 grid, size_t smem,
                       cudaStream_t st) {
     static std::atomic<unsigned long long> configured{0};
@@ -1543,12 +1724,22 @@ int launch_prefix_mma(const DecodeParams& p, const CUtensorMap& tmk, const CUten
     cudaGetDevice(&dev);
     const unsigned long long bit = 1ull << (dev & 63);
     if (!(configured.load() & bit)) {
-        if (cudaFuncSetAttribute(decode_prefix_mma_kernel<D, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(decode_prefix_mma_kernel<D, MT, PAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kMaxDynamicSmem) != cudaSuccess)
             return PA_ERR_CUDA;
         configured.fetch_or(bit);
     }
-    return launch_pdl(decode_prefix_mma_kernel<D, MT>, grid, dim3(32 * (1 + MT)), smem, st, p, tmk, tmv);
+    return launch_pdl(decode_prefix_mma_kernel<D, MT, PAR>, grid, dim3(32 * (1 + MT * PAR)), smem, st, p, tmk, tmv);
+}
+
+// Consumer groups of the prefix pass: two parity groups for 16 or 32 query
+// rows per CTA, one for 64 (the block stays at five warps or fewer).
+template <int D>
+int launch_prefix_for_rows(int mt, const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, dim3 grid,
+                           size_t smem, cudaStream_t st) {
+    return mt == 1 ? launch_prefix_mma<D, 1, 2>(p, tmk, tmv, grid, smem, st)
+         : mt == 2 ? launch_prefix_mma<D, 2, 2>(p, tmk, tmv, grid, smem, st)
+                   : launch_prefix_mma<D, 4, 1>(p, tmk, tmv, grid, smem, st);
 }
 
 template <typename T, int D, int G>
@@ -1619,7 +1810,8 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
     const int table_bytes = p.contiguous ? 0 : (plan.partition / p.block_size) * 4;
     p.ring_offset = (int)((16 * stages + table_bytes + 127) & ~127);
     const size_t ring_bytes = (size_t)stages * stage_bytes;
-    const size_t merge_bytes = (size_t)kConsumerWarps * G * (head_dim + 2) * sizeof(float);
+    const size_t merge_bytes = ((size_t)kConsumerWarps * G * (head_dim + 2) + (size_t)G * (kMaxFoldSplits + 1)) *
+                               sizeof(float);
     if (merge_bytes > ring_bytes) return PA_ERR_UNSUPPORTED;
     const size_t smem = p.ring_offset + ring_bytes;
     if (smem > (size_t)kMaxDynamicSmem) return PA_ERR_UNSUPPORTED;
@@ -1640,20 +1832,17 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
             pp.stages = kPrefixRingBytes / stage_bytes;
             const int ptable = (plan.prefix_partition / p.block_size) * 4;
             pp.ring_offset = (int)((16 * pp.stages + ptable + 1023) & ~1023);
-            const size_t psmem = pp.ring_offset + (size_t)pp.stages * stage_bytes + 1024;
-            if (psmem > (size_t)kMaxDynamicSmem) return PA_ERR_UNSUPPORTED;
+            // ring (a multiple of two stages: two consumer parity groups),
+            // then the chunk's query rows
+            const size_t qbytes = (size_t)16 * plan.mt * head_dim * 2;
+            const size_t psmem = pp.ring_offset + (size_t)pp.stages * stage_bytes + qbytes + 1024;
+            if (psmem > (size_t)kMaxDynamicSmem || pp.stages % 2) return PA_ERR_UNSUPPORTED;
             const int64_t gy = (int64_t)p.num_kv_heads * plan.chunks;
             if (gy > 65535) return PA_ERR_UNSUPPORTED;
             const dim3 pg((unsigned)(plan.prefix_splits > 0 ? plan.prefix_splits : 1), (unsigned)gy,
                           (unsigned)p.num_groups);
-            if (head_dim == 128)
-                rc = plan.mt == 1 ? launch_prefix_mma<128, 1>(pp, tmk, tmv, pg, psmem, st)
-                     : plan.mt == 2 ? launch_prefix_mma<128, 2>(pp, tmk, tmv, pg, psmem, st)
-                                    : launch_prefix_mma<128, 4>(pp, tmk, tmv, pg, psmem, st);
-            else
-                rc = plan.mt == 1 ? launch_prefix_mma<64, 1>(pp, tmk, tmv, pg, psmem, st)
-                     : plan.mt == 2 ? launch_prefix_mma<64, 2>(pp, tmk, tmv, pg, psmem, st)
-                                    : launch_prefix_mma<64, 4>(pp, tmk, tmv, pg, psmem, st);
+            rc = head_dim == 128 ? launch_prefix_for_rows<128>(plan.mt, pp, tmk, tmv, pg, psmem, st)
+                                 : launch_prefix_for_rows<64>(plan.mt, pp, tmk, tmv, pg, psmem, st);
             if (rc) return rc;
         }
         p.ring_offset = (int)((16 * stages + table_bytes + 1023) & ~1023);
@@ -1672,7 +1861,7 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
     if (rc) return rc;
     // with shared prefixes, rows whose suffix is one split are finished by
     // pass 1; the merge pass is needed only when a suffix can be split
-    if (p.num_groups > 0 ? plan.suffix_splits > 1 : plan.max_splits > 1) {
+    if (p.num_groups > 0 ? (plan.suffix_splits > 1 || plan.prefix_splits > kMaxFoldSplits) : plan.max_splits > 1) {
         const int64_t rows = (int64_t)batch * p.num_q_heads;
         // four warps per row, or all eight of a CTA when rows carry many splits
         // and there are too few rows to fill the GPU with four-warp groups
