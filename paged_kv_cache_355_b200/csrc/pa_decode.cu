@@ -13,7 +13,7 @@
 //    token positions, so the result is independent of where the blocks sit
 //    in the pool and bit-identical from run to run (no atomics).
 //  * Sequences are taken longest first: every CTA's prologue ranks the
-//    batch's lengths with a counting sort (64 length buckets) and maps its
+//    batch's lengths into 64 length buckets (a counting sort) and maps its
 //    blockIdx.z to the sequence of that rank, so the grid's tail holds the
 //    short sequences.
 //  * Warp 0 is the producer: the CTA's slice of the block table is staged
@@ -344,17 +344,19 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeParams& p, con
 // decreasing length (64 length buckets, ties by index).  This is
 // longest-processing-time-first list scheduling; it keeps the tail of the
 // grid short when lengths vary.  All threads read each length once into a
-// shared-memory key and a bucket histogram; then one warp walks the keys in
-// index order, placing each lane among equal keys with match_any (a counting
-// sort, O(batch) shared-memory work).  `scratch` is shared memory that is
-// free at this point (at least 512 + batch bytes).  With longest_first == 0
-// the rank is the sequence index.
+// shared-memory key and a bucket histogram; then one warp scans the histogram,
+// finds the bucket holding the CTA's rank and the rank's position in it, and
+// picks the sequence at that position among the bucket's members in index
+// order with ballots, 32 keys at a time.  Only this CTA's sequence is
+// selected (every CTA computes the same order, so the mapping is a
+// bijection).  `scratch` is shared memory that is free at this point (at
+// least 512 + batch bytes).  With longest_first == 0 the rank is the sequence
+// index.
 __device__ __forceinline__ int schedule_sequence(const DecodeParams& p, uint8_t* scratch) {
     const int rank = blockIdx.z;
     if (!p.longest_first) return rank;
     __shared__ int s_seq;
-    int* hist = reinterpret_cast<int*>(scratch);  // [64], then running positions [64]
-    int* run = hist + 64;
+    int* hist = reinterpret_cast<int*>(scratch);  // [64]
     uint8_t* key = scratch + 512;                 // [batch]
     const int tid = threadIdx.x;
     for (int k = tid; k < 64; k += blockDim.x) hist[k] = 0;
@@ -395,20 +397,24 @@ __device__ __forceinline__ int schedule_sequence(const DecodeParams& p, uint8_t*
             if (lane >= off) incl += y;
         }
         const int excl = incl - a0 - a1;
-        run[2 * lane] = excl;
-        run[2 * lane + 1] = excl + a0;
-        __syncwarp();
-        for (int c = 0; c < p.batch; c += 32) {
+        // the bucket holding this rank (the lane owning it broadcasts the
+        // bucket and the rank's position inside it), then that position's
+        // sequence among the bucket's members in index order, 32 at a time
+        const bool in0 = rank >= excl && rank < excl + a0;
+        const bool in1 = rank >= excl + a0 && rank < incl;
+        const unsigned owner = __ballot_sync(0xffffffffu, in0 || in1);
+        const int src = owner ? __ffs(owner) - 1 : 0;
+        const int kb = __shfl_sync(0xffffffffu, in0 ? 2 * lane : 2 * lane + 1, src);
+        int pos = rank - __shfl_sync(0xffffffffu, in0 ? excl : excl + a0, src);
+        for (int c = 0; owner && c < p.batch; c += 32) {
             const int b = c + lane;
-            const bool valid = b < p.batch;
-            const int k = valid ? key[b] : 64 + lane;
-            const unsigned peers = __match_any_sync(0xffffffffu, k);
-            const int before = __popc(peers & ((1u << lane) - 1u));
-            const int pos = valid ? run[k] + before : -1;
-            __syncwarp();
-            if (valid && before == 0) run[k] += __popc(peers);
-            if (pos == rank) s_seq = b;
-            __syncwarp();
+            const unsigned m = __ballot_sync(0xffffffffu, b < p.batch && key[b] == kb);
+            const int cnt = __popc(m);
+            if (pos < cnt) {
+                if (((m >> lane) & 1u) && __popc(m & ((1u << lane) - 1u)) == pos) s_seq = b;
+                break;
+            }
+            pos -= cnt;
         }
     }
     __syncthreads();
