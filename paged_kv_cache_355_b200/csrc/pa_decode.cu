@@ -61,6 +61,7 @@
 #include "pa.h"
 #include "pa_device.cuh"
 #include "pa_internal.h"
+#include "pa_tc.cuh"
 
 namespace pa {
 namespace {
@@ -1117,6 +1118,45 @@ __device__ __forceinline__ void consumer_barrier(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// A shared-prefix group as the prefix passes use it: first member, member
+// count and the prefix length it can share (0 when it cannot).
+struct PrefixGroup {
+    int start;
+    int n;
+    int prefix;
+};
+
+// Check group grp's description; every CTA of the group reaches the same
+// verdict.  The reporter CTA (one per group) flags a bad description and
+// writes each member's prefix length to seq_prefix.  Called by all threads.
+__device__ PrefixGroup prefix_group_setup(const DecodeParams& p, int grp, bool reporter) {
+    __shared__ int s_start, s_n, s_prefix, s_bad;
+    if (threadIdx.x == 0) {
+        const int s = p.group_starts[grp], e = p.group_starts[grp + 1], P = p.group_prefix[grp];
+        // a well-formed span gets its members' prefix lengths written in any
+        // case (0 when the group cannot share); a malformed one names no
+        // members, and the sequences it should have covered stay unspecified
+        const bool span_ok = s >= 0 && e >= s && e <= p.batch;
+        const bool ok = span_ok && e - s <= p.max_group && P >= 0 && P <= p.max_prefix && P % p.block_size == 0;
+        s_start = span_ok ? s : 0;
+        s_n = span_ok ? e - s : 0;
+        s_prefix = ok ? P : 0;
+        s_bad = !ok;
+        if (reporter && ((grp == 0 && s != 0) || (grp == p.num_groups - 1 && e != p.batch)))
+            record_error(p.err, PA_ERR_BAD_BLOCK_ID);  // the groups do not cover the batch
+    }
+    __syncthreads();
+    for (int m = threadIdx.x; m < s_n; m += blockDim.x)
+        if (clamp_len(p, s_start + m, false) < s_prefix) s_bad = 1;  // a member shorter than the prefix
+    __syncthreads();
+    const PrefixGroup g{s_start, s_n, s_bad ? 0 : s_prefix};
+    if (reporter) {
+        if (threadIdx.x == 0 && s_bad) record_error(p.err, PA_ERR_BAD_BLOCK_ID);
+        for (int m = threadIdx.x; m < g.n; m += blockDim.x) p.seq_prefix[g.start + m] = g.prefix;
+    }
+    return g;
+}
+
 template <int D, int MT, int PAR>
 __global__ void __launch_bounds__(32 * (1 + MT * PAR), 3)
     decode_prefix_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
@@ -1136,8 +1176,6 @@ __global__ void __launch_bounds__(32 * (1 + MT * PAR), 3)
     int32_t* tbl = reinterpret_cast<int32_t*>(empty + p.stages);
     uint8_t* ring = smem + p.ring_offset + ((1024u - (smem_addr(smem) & 1023u)) & 1023u);
     uint8_t* qtile = ring + (size_t)p.stages * 2 * STAGE_BYTES;  // [SLABS][ROWS][128 B], swizzled
-    __shared__ int s_start, s_n, s_prefix, s_bad;
-
     if (threadIdx.x == 0) {
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
@@ -1151,33 +1189,10 @@ __global__ void __launch_bounds__(32 * (1 + MT * PAR), 3)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int G = p.num_q_heads / p.num_kv_heads;
-    const bool reporter = split == 0 && blockIdx.y == 0;
-
-    // the group's description; every CTA of the group reaches the same verdict
-    if (threadIdx.x == 0) {
-        const int s = p.group_starts[grp], e = p.group_starts[grp + 1], P = p.group_prefix[grp];
-        // a well-formed span gets its members' prefix lengths written in any
-        // case (0 when the group cannot share); a malformed one names no
-        // members, and the sequences it should have covered stay unspecified
-        const bool span_ok = s >= 0 && e >= s && e <= p.batch;
-        const bool ok = span_ok && e - s <= p.max_group && P >= 0 && P <= p.max_prefix && P % p.block_size == 0;
-        s_start = span_ok ? s : 0;
-        s_n = span_ok ? e - s : 0;
-        s_prefix = ok ? P : 0;
-        s_bad = !ok;
-        if (reporter && ((grp == 0 && s != 0) || (grp == p.num_groups - 1 && e != p.batch)))
-            record_error(p.err, PA_ERR_BAD_BLOCK_ID);  // the groups do not cover the batch
-    }
-    __syncthreads();
-    for (int m = threadIdx.x; m < s_n; m += blockDim.x)
-        if (clamp_len(p, s_start + m, false) < s_prefix) s_bad = 1;  // a member shorter than the prefix
-    __syncthreads();
-    const int n = s_n;
-    const int P = s_bad ? 0 : s_prefix;
-    if (reporter) {
-        if (threadIdx.x == 0 && s_bad) record_error(p.err, PA_ERR_BAD_BLOCK_ID);
-        for (int m = threadIdx.x; m < n; m += blockDim.x) p.seq_prefix[s_start + m] = P;
-    }
+    const PrefixGroup pgrp = prefix_group_setup(p, grp, split == 0 && blockIdx.y == 0);
+    const int s_start = pgrp.start;
+    const int n = pgrp.n;
+    const int P = pgrp.prefix;
     const int tok_begin = split * p.prefix_partition;
     const int rows_total = n * G;
     const int row0 = chunk * ROWS;
@@ -1487,6 +1502,438 @@ __global__ void __launch_bounds__(32 * (1 + MT * PAR), 3)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Shared-prefix pass on the 5th-generation tensor cores (head_dim 128).
+//
+// Same work item, inputs and outputs as the mma.sync pass above, with 32 query
+// rows per CTA.  The shared tokens are the M side of tcgen05 MMAs, so one
+// 128-token tile of K and V feeds all the rows at once:
+//     S^T[tokens, rows] = K[tokens, D] . Q^T[D, rows]         (M = 128 tokens)
+//     O^T[D, rows]     += V^T[D, tokens] . P^T[tokens, rows]  (M = D = 128)
+// K is the A operand as it lands from TMA (K-major, 128-byte swizzle); V is the
+// A operand read M-major from the same kind of tile; Q (staged once) and P are
+// the B operands; S^T (double-buffered) and O^T live in tensor memory.
+//  * warp 0 streams K and V tiles of 128 shared tokens (tiled TMA boxes of
+//    block_size rows, one pool block per lane) into one K and one V buffer: K
+//    of the next tile is requested as soon as S of this one is computed, V as
+//    soon as its P.V is.  With one buffer each a CTA takes ~90 KB of shared
+//    memory, so two run on an SM: one's start-up and epilogue overlap the
+//    other's stream, and the GPU holds the whole grid of a typical call;
+//  * warp 1 owns the tensor memory and issues the MMAs from one thread:
+//    P_{j-1}.V_{j-1} once the softmax has written P_{j-1}, then S_j;
+//  * warps 2..5 (one per TMEM lane quarter) run the softmax: thread t holds
+//    token t's scores for all 32 rows.  Every thread keeps the rows' running
+//    maxima; they move only when a score exceeds them by more than 2^8
+//    (found with one barrier reduction per tile), so most tiles need no
+//    cross-thread max.  When they move, the tile's exact row maxima come
+//    from a transposing shuffle reduction and O^T is rescaled in tensor
+//    memory.  Each thread keeps partial row sums over its own tokens
+//    (combined once at the end) and writes its token's row of P^T, as bf16
+//    high and residual parts (M/N-major, 64-byte swizzle), for the next P.V;
+//  * at the end they stage O^T through shared memory and write each row's
+//    normalised partial (as float4 rows) and (m, l), as the mma.sync pass
+//    does.
+// ---------------------------------------------------------------------------
+constexpr int kTcTokens = 128;         // shared tokens per tile (M of S^T)
+constexpr int kTcRows = 32;            // query rows per CTA (N of both MMAs)
+constexpr int kTcThreads = 64 + 128;   // producer, MMA issuer, softmax warpgroup
+constexpr float kTcRescaleLog2 = 8.f;  // lazy-rescale threshold of the running max (log2 units)
+constexpr int kTcSlab = kTcTokens * 128;        // one 64-column slab of a K or V tile
+constexpr int kTcTile = 2 * kTcSlab;            // a K or V tile of 128 tokens x 128 columns
+constexpr int kTcQSlab = kTcRows * 128;         // one 64-column slab of the Q tile
+constexpr int kTcPRow = kTcRows * 2;            // bytes of one token's row of P^T
+constexpr int kTcPBytes = kTcTokens * kTcPRow;  // one part (high or residual) of P^T
+constexpr uint32_t kTcTmemCols = 128;           // O^T in [0, 32), S^T buffers in [32, 96)
+static_assert(kTcRows * kTcTokens * 4 <= kTcTile, "the epilogue stages O^T in the K buffer");
+
+// Dynamic shared memory of the tensor-core prefix pass: the K and V buffers,
+// P^T (high + residual), the Q tile, the reduction scratch and the split's
+// block-table slice, after 1024-byte alignment.
+inline size_t prefix_tc_smem_bytes(int table_entries) {
+    return 1024 + 2 * (size_t)kTcTile + 2 * (size_t)kTcPBytes + 2 * (size_t)kTcQSlab + 4 * kTcRows * sizeof(float) +
+           (size_t)table_entries * sizeof(int32_t);
+}
+
+// OR of a predicate over the 128 softmax threads (named barrier 1).
+__device__ __forceinline__ bool softmax_any(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.or.pred po, 1, 128, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return r != 0;
+}
+
+// Reduce v[0..31] element-wise over the warp's 32 lanes so that lane i ends
+// with the result for element i (max or sum): five exchange steps, each
+// halving the elements a lane keeps, 31 shuffles in all.  Destroys v.
+template <bool kMax>
+__device__ __forceinline__ float warp_transpose_reduce(float (&v)[32], int lane) {
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1) {
+        const bool upper = (lane & w) != 0;
+#pragma unroll
+        for (int i = 0; i < w; ++i) {
+            const float send = upper ? v[i] : v[i + w];
+            const float keep = upper ? v[i + w] : v[i];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, w);
+            v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+        }
+    }
+    return v[0];
+}
+
+__global__ void __launch_bounds__(kTcThreads, 2)
+    decode_prefix_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
+                            const __grid_constant__ CUtensorMap tmv) {
+    constexpr int D = 128;
+    constexpr int N = kTcRows;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    uint8_t* sK = smem;                                        // K tile (the epilogue's O staging after)
+    uint8_t* sV = sK + kTcTile;                                // V tile
+    uint8_t* sP = sV + kTcTile;                                // P^T: high part, residual part
+    uint8_t* sQ = sP + 2 * kTcPBytes;                          // [2 slabs][kTcQSlab]
+    float* red = reinterpret_cast<float*>(sQ + 2 * kTcQSlab);  // [4 warps][N]
+    int32_t* tbl = reinterpret_cast<int32_t*>(red + 4 * N);
+    __shared__ uint64_t k_full, k_empty, v_full, v_empty, s_full[2], p_full, pv_done;
+    __shared__ uint32_t tmem_base;
+    __shared__ int64_t row_off[N];  // epilogue: element offset of row r's partial, or -1
+    __shared__ float row_inv[N];    //           1 / row sum
+
+    if (threadIdx.x == 0) {
+        prefetch_tmap(&tmk);
+        prefetch_tmap(&tmv);
+    }
+    griddep_wait();  // q, lengths, tables and the pool may come from the kernel before
+    griddep_launch_dependents();
+    const int split = blockIdx.x;
+    const int kvh = blockIdx.y % p.num_kv_heads;
+    const int chunk = blockIdx.y / p.num_kv_heads;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int G = p.num_q_heads / p.num_kv_heads;
+    const PrefixGroup grp = prefix_group_setup(p, blockIdx.z, split == 0 && blockIdx.y == 0);
+    const int tok_begin = split * p.prefix_partition;
+    const int rows_total = grp.n * G;
+    const int row0 = chunk * N;
+    if (tok_begin >= grp.prefix || row0 >= rows_total) return;  // uniform over the CTA, before any barrier
+    const int ntok = min(grp.prefix, tok_begin + p.prefix_partition) - tok_begin;
+    const int nt = (ntok + kTcTokens - 1) / kTcTokens;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&k_full, 1);
+        mbar_init(&k_empty, 1);
+        mbar_init(&v_full, 1);
+        mbar_init(&v_empty, 1);
+        mbar_init(&s_full[0], 1);
+        mbar_init(&s_full[1], 1);
+        mbar_init(&p_full, 4);
+        mbar_init(&pv_done, 1);
+        fence_barrier_init();
+    }
+    {
+        // the shared blocks, from the first member's table
+        const int first_blk = tok_begin / p.block_size;
+        const int nblk = (ntok + p.block_size - 1) / p.block_size;
+        const int32_t* row = p.block_tables + (int64_t)grp.start * p.max_blocks_per_seq + first_blk;
+        for (int i = threadIdx.x; i < nblk; i += blockDim.x) tbl[i] = row[i];
+        // the chunk's query rows (zero past the group), K-major with the
+        // 128-byte swizzle: 16-byte chunk c of row r of a slab at c ^ (r & 7)
+        const uint16_t* qv = static_cast<const uint16_t*>(p.q);
+        for (int i = threadIdx.x; i < N * (D / 8); i += blockDim.x) {
+            const int r = i / (D / 8);
+            const int c = i % (D / 8);
+            const int gr = row0 + r;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (gr < rows_total)
+                v = *reinterpret_cast<const uint4*>(
+                    qv + ((int64_t)(grp.start + gr / G) * p.num_q_heads + (int64_t)kvh * G + gr % G) * D + c * 8);
+            *reinterpret_cast<uint4*>(sQ + (c >> 3) * kTcQSlab + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
+        }
+        fence_proxy_async_smem();  // the tensor core reads Q through the async proxy
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&tmem_base)),
+                     "r"(kTcTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base;
+
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        const uint64_t policy = l2_policy_evict_first();
+        const int bs = p.block_size;
+        const int boxes = kTcTokens / bs;  // pool blocks per tile
+        bool streamed = true;
+        for (int j = 0; j < nt; ++j) {
+            const int t0 = j * kTcTokens;
+            const int valid = min(kTcTokens, ntok - t0);
+            const int r = lane * bs;
+            int y = 0;
+            uint32_t nbytes = 0;
+            if (lane < boxes && r < valid) {
+                const int32_t phys = tbl[(t0 + r) / bs];
+                if (phys < 0 || phys >= p.num_blocks) {
+                    record_error(p.err, PA_ERR_BAD_BLOCK_ID);
+                } else {
+                    nbytes = (uint32_t)(2 * bs * 128);
+                    y = (phys * p.num_kv_heads + kvh) * bs;
+                }
+            }
+            const uint32_t total = __reduce_add_sync(0xffffffffu, nbytes);
+            // K_j once S_{j-1} has read the K buffer
+            if (j >= 1) {
+                int ok = 1;
+                if (lane == 0) ok = mbar_wait(&k_empty, (j - 1) & 1, p.err);
+                if (!(streamed = __shfl_sync(0xffffffffu, ok, 0))) break;
+            }
+            if (lane == 0) mbar_arrive_expect_tx(&k_full, total);
+            __syncwarp();
+            if (nbytes) {
+                tma_load_2d(sK + r * 128, &tmk, 0, y, &k_full, policy);
+                tma_load_2d(sK + kTcSlab + r * 128, &tmk, 64, y, &k_full, policy);
+            }
+            // V_j once P_{j-1}.V_{j-1} has read the V buffer
+            if (j >= 1) {
+                int ok = 1;
+                if (lane == 0) ok = mbar_wait(&v_empty, (j - 1) & 1, p.err);
+                if (!(streamed = __shfl_sync(0xffffffffu, ok, 0))) break;
+            }
+            if (valid < kTcTokens) {
+                // the tile's tokens past the split carry weight 0, but 0 * NaN
+                // is NaN in the MMA: zero those V rows (stale or never loaded)
+                const int nch = (kTcTokens - valid) * 16;
+                for (int c = lane; c < nch; c += 32) {
+                    const int row = valid + c / 16;
+                    const int rem = c % 16;
+                    *reinterpret_cast<uint4*>(sV + (rem >> 3) * kTcSlab + row * 128 + (rem & 7) * 16) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
+            if (lane == 0) mbar_arrive_expect_tx(&v_full, total);
+            __syncwarp();
+            if (nbytes) {
+                tma_load_2d(sV + r * 128, &tmv, 0, y, &v_full, policy);
+                tma_load_2d(sV + kTcSlab + r * 128, &tmv, 64, y, &v_full, policy);
+            }
+        }
+        // the last tile's releases are tensor-core commits that land in this
+        // CTA's shared memory: wait for them before the CTA may exit
+        if (lane == 0 && streamed && mbar_wait(&k_empty, (nt - 1) & 1, p.err))
+            mbar_wait(&v_empty, (nt - 1) & 1, p.err);
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            constexpr uint32_t IDESC_S = umma_idesc(kTcTokens, N, false, false);
+            constexpr uint32_t IDESC_O = umma_idesc(D, N, true, true);
+            const uint32_t q_base = smem_addr(sQ);
+            const uint32_t k_base = smem_addr(sK);
+            const uint32_t v_base = smem_addr(sV);
+            const uint32_t p_base = smem_addr(sP);
+            for (int j = 0; j <= nt; ++j) {
+                if (j >= 1) {
+                    // O^T += V_{j-1}^T . P_{j-1}^T, high part then residual,
+                    // 16 tokens per step
+                    const int jp = j - 1;
+                    if (!mbar_wait(&p_full, jp & 1, p.err)) break;
+                    if (!mbar_wait(&v_full, jp & 1, p.err)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kTcTokens / 16; ++kk) {
+                        const uint64_t da = umma_desc(v_base + kk * 16 * 128, kTcSlab, 1024);
+                        const uint32_t pk = p_base + kk * 16 * kTcPRow;
+                        umma(tmem, da, umma_desc_sw(pk, kTcPBytes, 8 * kTcPRow, kUmmaSwizzle64), IDESC_O,
+                             (jp > 0 || kk > 0) ? 1u : 0u);
+                        umma(tmem, da, umma_desc_sw(pk + kTcPBytes, kTcPBytes, 8 * kTcPRow, kUmmaSwizzle64), IDESC_O,
+                             1u);
+                    }
+                    umma_commit(&pv_done);
+                    umma_commit(&v_empty);
+                }
+                if (j < nt) {
+                    // S_j^T = K_j . Q^T into S buffer j & 1 (the softmax
+                    // loaded S_{j-2} before it signalled P_{j-2})
+                    if (!mbar_wait(&k_full, j & 1, p.err)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * kTcSlab + (kk & 3) * 32;
+                        const uint32_t qoff = (kk >> 2) * kTcQSlab + (kk & 3) * 32;
+                        umma(tmem + N + (j & 1) * N, umma_desc(k_base + off, 16, 1024),
+                             umma_desc(q_base + qoff, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&s_full[j & 1]);
+                    umma_commit(&k_empty);
+                }
+            }
+        }
+    } else {
+        // ---------------- softmax: one token per thread ----------------
+        const int q4 = warp & 3;         // TMEM lane quarter this warp may access
+        const int tok = q4 * 32 + lane;  // token of the tile = TMEM lane
+        const int st = threadIdx.x - 64; // thread index within the softmax warpgroup
+        const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
+        float m[N], l[N];  // reference maxima (log2 units, scaled; the same in every thread), partial sums
+#pragma unroll
+        for (int r = 0; r < N; ++r) {
+            m[r] = -INFINITY;
+            l[r] = 0.f;
+        }
+        bool ok = true;
+        for (int j = 0; j < nt; ++j) {
+            // S_j is ready, and P.V of tile j - 1 is done: O^T holds the tiles
+            // before j (for a rescale) and the P buffer is free
+            bool wok = mbar_wait(&s_full[j & 1], (j >> 1) & 1, p.err);
+            if (wok && j >= 1) wok = mbar_wait(&pv_done, (j - 1) & 1, p.err);
+            if (softmax_any(!wok)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t s_col = lane_base + N + (j & 1) * N;
+            const bool tvalid = j * kTcTokens + tok < ntok;
+            float x[N];
+            bool grow = false;
+            tmem_ld32(s_col, x);
+            tmem_wait_ld();
+#pragma unroll
+            for (int r = 0; r < N; ++r) grow |= tvalid && x[r] * p.scale_log2 > m[r] + kTcRescaleLog2;
+            if (softmax_any(grow)) {
+                // the tile's exact row maxima: over this warp's 32 tokens by
+                // a transposing shuffle reduction (lane i gets row i), then
+                // over the four warps through shared memory
+#pragma unroll
+                for (int r = 0; r < N; ++r) x[r] = tvalid ? x[r] * p.scale_log2 : -INFINITY;
+                red[q4 * N + lane] = warp_transpose_reduce<true>(x, lane);
+                consumer_barrier(1, 128);
+                const float mt = fmaxf(fmaxf(red[lane], red[N + lane]), fmaxf(red[2 * N + lane], red[3 * N + lane]));
+                // O^T (lane = output element, column = row) holds the tiles
+                // before j: rescale it with the partial sums
+                float ov[32];
+                if (j >= 1) {
+                    tmem_ld32(lane_base, ov);
+                    tmem_wait_ld();
+                }
+#pragma unroll
+                for (int r = 0; r < N; ++r) {
+                    const float mn = fmaxf(m[r], __shfl_sync(0xffffffffu, mt, r));
+                    const float alpha = m[r] == -INFINITY ? 0.f : ex2_approx(m[r] - mn);
+                    m[r] = mn;
+                    l[r] *= alpha;
+                    ov[r] *= alpha;
+                }
+                if (j >= 1) {
+                    tmem_st32(lane_base, ov);
+                    tmem_wait_st();
+                }
+                // the reduction consumed the scores: read them again
+                tmem_ld32(s_col, x);
+                tmem_wait_ld();
+            }
+#pragma unroll
+            for (int r = 0; r < N; ++r) x[r] = tvalid ? x[r] * p.scale_log2 : -INFINITY;
+            // weights of this token for every row, split into bf16 high and
+            // residual parts, written as token tok's row of P^T: rows
+            // 8c..8c+7 form 16-byte chunk c, stored at chunk c ^ ((tok & 7) >> 1)
+            // (the 64-byte swizzle)
+            uint8_t* prow = sP + tok * kTcPRow;
+#pragma unroll
+            for (int c = 0; c < kTcPRow / 16; ++c) {
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = 8 * c + 2 * i;
+                    const float e0 = m[r] == -INFINITY ? 0.f : ex2_approx(x[r] - m[r]);
+                    const float e1 = m[r + 1] == -INFINITY ? 0.f : ex2_approx(x[r + 1] - m[r + 1]);
+                    l[r] += e0;
+                    l[r + 1] += e1;
+                    hi[i] = pack_bf16x2(e0, e1);
+                    lo[i] = pack_bf16x2(e0 - bf16_lo_to_f32(hi[i]), e1 - bf16_hi_to_f32(hi[i]));
+                }
+                const int pc = c ^ ((tok & 7) >> 1);
+                *reinterpret_cast<uint4*>(prow + pc * 16) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4*>(prow + kTcPBytes + pc * 16) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+            fence_proxy_async_smem();  // P is read by the tensor core
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full);
+        }
+        // the last P.V done: O^T is complete (and every MMA has read its
+        // operands, so the K buffer is free for the epilogue)
+        if (ok) {
+            const bool wok = mbar_wait(&pv_done, (nt - 1) & 1, p.err);
+            ok = !softmax_any(!wok);
+        }
+        if (ok) {
+            tc_fence_after();
+            // row sums: each thread's over its tokens, added over the warp
+            // (lane i gets row i) and then over the four warps
+            float v[32];
+#pragma unroll
+            for (int r = 0; r < N; ++r) v[r] = l[r];
+            red[q4 * N + lane] = warp_transpose_reduce<false>(v, lane);
+            // O^T column tok (output element tok of every row) into the K
+            // buffer as rows [N][D]
+            float* so = reinterpret_cast<float*>(sK);
+            float ov[32];
+            tmem_ld32(lane_base, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int r = 0; r < N; ++r) so[r * D + tok] = ov[r];
+            consumer_barrier(1, 128);
+            if (q4 == 0) {
+                // row `lane`: its slot, 1 / l, and (m, l)
+                const float lt = (red[lane] + red[N + lane]) + (red[2 * N + lane] + red[3 * N + lane]);
+                float mr = m[0];
+#pragma unroll
+                for (int r = 1; r < N; ++r) mr = lane == r ? m[r] : mr;
+                const int gr = row0 + lane;
+                int64_t off = -1;
+                if (gr < rows_total) {
+                    const int64_t qrow = (int64_t)(grp.start + gr / G) * p.num_q_heads + (int64_t)kvh * G + gr % G;
+                    const int64_t slotrow = qrow * p.max_splits + split;
+                    off = slotrow * D;
+                    p.part_ml[2 * slotrow] = mr;
+                    p.part_ml[2 * slotrow + 1] = lt;
+                }
+                row_off[lane] = off;
+                row_inv[lane] = lt > 0.f ? 1.f / lt : 0.f;
+            }
+            consumer_barrier(1, 128);
+            // each row's 128 elements as 32 float4, one row per warp step
+            const float4* so4 = reinterpret_cast<const float4*>(so);
+            for (int i = st; i < N * (D / 4); i += 128) {
+                const int r = i / (D / 4);
+                const int64_t off = row_off[r];
+                if (off >= 0) {
+                    float4 o = so4[i];
+                    const float inv = row_inv[r];
+                    o.x *= inv;
+                    o.y *= inv;
+                    o.z *= inv;
+                    o.w *= inv;
+                    *reinterpret_cast<float4*>(p.part_o + off + (i % (D / 4)) * 4) = o;
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcTmemCols));
+    }
+}
+
 // Second pass: out = sum_s w_s o_s / sum_s w_s with w_s = l_s * 2^(m_s - max m),
 // for sequences that were cut into more than one split.  W warps share a
 // (sequence, query head) row: W = 4 with two rows per CTA, or W = 8 with one
@@ -1609,7 +2056,8 @@ struct Plan {
     // shared-prefix calls only
     int prefix_partition;
     int prefix_splits;
-    int mt;      // 16-row query tiles per prefix CTA (consumer warps)
+    int tc;      // head_dim 128: the tensor-core (tcgen05) prefix pass, 32 query rows per CTA
+    int mt;      // otherwise: 16-row query tiles per prefix CTA (consumer warps)
     int chunks;  // prefix CTAs per (group, kv head) along the query rows
 };
 
@@ -1662,8 +2110,10 @@ int make_plan(int batch, int num_q_heads, int num_kv_heads, int head_dim, int ma
     plan->max_splits = splits;
     if (num_groups > 0) {
         const int rows = max_group * (num_q_heads / num_kv_heads);
+        plan->tc = head_dim == 128;
         plan->mt = rows <= 16 ? 1 : (rows <= 32 ? 2 : 4);
-        plan->chunks = (rows + 16 * plan->mt - 1) / (16 * plan->mt);
+        const int rows_per_cta = plan->tc ? kTcRows : 16 * plan->mt;
+        plan->chunks = (rows + rows_per_cta - 1) / rows_per_cta;
         plan->prefix_partition = auto_prefix_partition(num_groups, num_kv_heads, plan->chunks, max_prefix);
         plan->prefix_splits = max_prefix > 0 ? (max_prefix + plan->prefix_partition - 1) / plan->prefix_partition : 0;
         plan->max_splits = plan->prefix_splits + splits;
@@ -1738,6 +2188,21 @@ int launch_prefix_mma(const DecodeParams& p, const CUtensorMap& tmk, const CUten
         configured.fetch_or(bit);
     }
     return launch_pdl(decode_prefix_mma_kernel<D, MT, PAR>, grid, dim3(32 * (1 + MT * PAR)), smem, st, p, tmk, tmv);
+}
+
+int launch_prefix_tc(const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, dim3 grid, size_t smem,
+                     cudaStream_t st) {
+    static std::atomic<unsigned long long> configured{0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(configured.load() & bit)) {
+        if (cudaFuncSetAttribute(decode_prefix_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kMaxDynamicSmem) != cudaSuccess)
+            return PA_ERR_CUDA;
+        configured.fetch_or(bit);
+    }
+    return launch_pdl(decode_prefix_tc_kernel, grid, dim3(kTcThreads), smem, st, p, tmk, tmv);
 }
 
 // Consumer groups of the prefix pass: two parity groups for 16 or 32 query
@@ -1836,7 +2301,17 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
         CUtensorMap tmk, tmv;
         if ((rc = encode_kv_map(&tmk, p.k, rows, head_dim, p.block_size))) return rc;
         if ((rc = encode_kv_map(&tmv, p.v, rows, head_dim, p.block_size))) return rc;
-        if (p.num_groups > 0) {
+        if (p.num_groups > 0 && plan.tc) {
+            // the prefix pass on the tensor cores: 128-token tiles, its own
+            // buffers and tensor memory
+            const size_t psmem = prefix_tc_smem_bytes(plan.prefix_partition / p.block_size);
+            if (psmem > (size_t)kMaxDynamicSmem) return PA_ERR_UNSUPPORTED;
+            const int64_t gy = (int64_t)p.num_kv_heads * plan.chunks;
+            if (gy > 65535) return PA_ERR_UNSUPPORTED;
+            const dim3 pg((unsigned)(plan.prefix_splits > 0 ? plan.prefix_splits : 1), (unsigned)gy,
+                          (unsigned)p.num_groups);
+            if ((rc = launch_prefix_tc(p, tmk, tmv, pg, psmem, st))) return rc;
+        } else if (p.num_groups > 0) {
             // the prefix pass: a deeper ring (few, long-lived CTAs), every
             // consumer warp reads every stage
             DecodeParams pp = p;

@@ -195,3 +195,107 @@ def test_block_manager_groups_drive_the_shared_prefix_call(pa):
     out = run_shared(pa, case, starts.tolist(), plens.tolist(), max_prefix=mp, max_group=mg)
     assert_matches_oracle(out, run_oracle(case), True, "block-manager groups")
     assert pa.pa_read_error_flag() == 0
+
+
+# ---- many groups (the GPU-filling case), head_dim 128 ---------------------
+# 16 copies of the five groups above with 2 kv heads: 80 groups x 2 kv heads x
+# the row chunks >= 160 prefix CTAs, so every group's prefix is one split (the
+# tensor-core pass's widest tiling) and pass 1 folds it into each row.
+MANY_COPIES = 16
+
+
+def _many_case(bs, G, seed, extra=(), extra_blocks=4):
+    groups = _groups(bs) * MANY_COPIES + list(extra)
+    return shared_prefix_case(groups, 2 * G, 2, 128, bs, torch.bfloat16, seed=seed, extra_blocks=extra_blocks)
+
+
+@pytest.mark.parametrize("bs", [8, 16, 32])
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
+def test_many_groups_sweep(pa, bs, G):
+    """Own parts of 0..517 tokens, members whose context is the prefix, a
+    group without a prefix; several row chunks per group for G >= 4."""
+    case, starts, plens = _many_case(bs, G, seed=100 + bs + G)
+    out = run_shared(pa, case, starts, plens)
+    assert_matches_oracle(out, run_oracle(case), True, f"many groups bs{bs} G{G}")
+    assert pa.pa_read_error_flag() == 0
+
+
+def test_many_groups_bf16_output_and_empty_sequences(pa):
+    """bf16 rows; groups without a prefix whose members are empty (rows of
+    zeros) or mixed with a non-empty one."""
+    case, starts, plens = _many_case(16, 4, seed=131, extra=[(0, [0, 0]), (0, [0, 9])])
+    out = run_shared(pa, case, starts, plens, out_dtype=torch.bfloat16)
+    ref = run_oracle(case)
+    assert_matches_oracle(out, ref, True, "many groups, bf16 out")
+    empty = [b for b, L in enumerate(case.lengths.tolist()) if L == 0]
+    assert len(empty) == 3 and torch.all(out[empty] == 0)
+    assert pa.pa_read_error_flag() == 0
+
+
+def test_many_groups_are_deterministic_and_placement_free(pa):
+    case, starts, plens = _many_case(16, 4, seed=137, extra_blocks=40)
+    a = run_shared(pa, case, starts, plens)
+    assert torch.equal(a, run_shared(pa, case, starts, plens))
+    perm = torch.randperm(case.num_blocks, generator=torch.Generator().manual_seed(138))
+    kp, vp = torch.empty_like(case.k_pool), torch.empty_like(case.v_pool)
+    kp[perm] = case.k_pool
+    vp[perm] = case.v_pool
+    bt = torch.where(case.block_tables >= 0, perm[case.block_tables.clamp(min=0).long()].to(torch.int32),
+                     case.block_tables)
+    assert torch.equal(a, run_shared(pa, case, starts, plens, bt=bt, kp=kp, vp=vp))
+
+
+def test_many_groups_never_read_outside_the_sequences(pa):
+    """NaN in every pool slot no sequence uses (the rest of each partly used
+    block included) and junk block ids past each table's used entries."""
+    case, starts, plens = _many_case(16, 2, seed=139, extra_blocks=24)
+    clean = run_shared(pa, case, starts, plens)
+    kp, vp = case.k_pool.clone(), case.v_pool.clone()
+    used = torch.zeros(case.num_blocks, 16, dtype=torch.bool)
+    for b, L in enumerate(case.lengths.tolist()):
+        for t in range(L):
+            used[case.block_tables[b, t // 16], t % 16] = True
+    kp.permute(0, 2, 1, 3)[~used] = float("nan")
+    vp.permute(0, 2, 1, 3)[~used] = float("nan")
+    bt = case.block_tables.clone()
+    bt[bt < 0] = case.num_blocks + 1000
+    assert torch.equal(clean, run_shared(pa, case, starts, plens, bt=bt, kp=kp, vp=vp))
+    assert pa.pa_read_error_flag() == 0
+
+
+@pytest.mark.parametrize("fault", ["longer_than_a_member", "above_max_prefix", "not_whole_blocks"])
+def test_many_groups_broken_group_is_flagged_and_attended_without_sharing(pa, fault):
+    case, starts, plens = _many_case(16, 4, seed=149)
+    starts, plens = list(starts), list(plens)
+    kw = {}
+    if fault == "longer_than_a_member":
+        plens[7] = 32                     # a copy of group 2: its first member has 16 tokens
+    elif fault == "above_max_prefix":
+        kw["max_prefix"] = 512            # the copies of group 3 declare 640
+    else:
+        plens[5] = 56                     # not a multiple of 16
+    pa.pa_read_error_flag()
+    out = run_shared(pa, case, starts, plens, **kw)
+    assert pa.pa_read_error_flag() == 5
+    assert_matches_oracle(out, run_oracle(case), True, f"many groups, {fault}")
+
+
+def test_many_groups_flag_lengths_above_max_context(pa):
+    """A length above max_context_len is clamped to it and flagged, as the
+    plain decode does."""
+    case, starts, plens = _many_case(16, 4, seed=151)
+    lens = case.lengths.clone()
+    b = int(torch.argmax(lens))
+    L = int(lens[b])
+    lens[b] = L + 5  # the call is told max_context_len = L
+    pa.pa_read_error_flag()
+    out = torch.full_like(case.q, float("nan"), dtype=torch.float32, device="cuda")
+    gs = torch.tensor(starts, dtype=torch.int32, device="cuda")
+    gl = torch.tensor(plens, dtype=torch.int32, device="cuda")
+    mg = max(e - s for s, e in zip(starts[:-1], starts[1:]))
+    pa.pa_paged_attention_decode_shared_prefix(case.q.cuda(), case.k_pool.cuda(), case.v_pool.cuda(),
+                                               case.block_tables.cuda(), lens.cuda(), L, case.scale, out, gs, gl,
+                                               max(plens), mg)
+    torch.cuda.synchronize()
+    assert pa.pa_read_error_flag() == 5
+    assert_matches_oracle(out, run_oracle(case), True, "many groups, clamped length")
