@@ -26,11 +26,10 @@ value  = K/V bytes attention reads (tokens < length, K and V) / step time,
 e2e    = the same metric through the public API with the step's inputs in
          pinned host memory: one H2D copy of q, new K/V, block tables and
          lengths packed together, the step (direct calls on views of the
-         device copy), and D2H of the output, all inside the timed
-         events; a device spin before each step lets the host enqueue it
-         ahead, so host issue latency stays out.  host_wall_ms_per_step
-         times the same calls by the host clock with no spin (issue to a
-         synchronize after the read-back).
+         device copy), and D2H of the output, timed by the host clock from
+         the first issue to a synchronize after the read-back (what a
+         caller without graphs waits).  device_ms_per_step times the same
+         calls by CUDA events with a device spin ahead of each step.
 roofline = the decode call alone (pass 1 + merge; at least 100 timed replays,
          mean, median, p10 and p90 reported) against the measured HBM copy
          bandwidth, and against the read ceiling that pa_hbm_read_probe (a
@@ -798,14 +797,16 @@ def run_ours(args):
                                   if plain_decode and w.dtype == torch.bfloat16 else "")},
         "paging_overhead": {"paged_ms_median": paged_med, "contiguous_ms_median": contig_med,
                             "overhead": paged_med / contig_med - 1.0, "contiguous_ms_mean_max_ranks": ms_contig},
-        "e2e": {"value": world * kv_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e, "ms_stats": time_stats(e2e_ms),
-                "host_wall_ms_per_step": ms_host, "host_wall_ms_stats": time_stats(host_ms),
-                "host_wall_gbs": world * kv_bytes / (ms_host * 1e-3) / 1e9,
-                "timing": "device time from before the H2D copies to after the D2H read-back, direct API calls "
-                          "(no graph); a device spin ahead of each step keeps host issue latency out. "
-                          "host_wall: the same calls timed by the host clock from the first issue to a "
-                          "synchronize after the read-back, with no spin (what a caller without graphs waits)"},
+        "e2e": {"value": world * kv_bytes / (ms_host * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": ms_host, "ms_stats": time_stats(host_ms),
+                "device_ms_per_step": ms_e2e, "device_ms_stats": time_stats(e2e_ms),
+                "device_gbs": world * kv_bytes / (ms_e2e * 1e-3) / 1e9,
+                "timing": "host clock from the first issue (the H2D copies of the step's inputs from pinned "
+                          "memory) to a synchronize after the D2H read-back of the result, direct API calls, no "
+                          "graph, max over ranks: what a caller without graphs waits. device_*: the same calls "
+                          "timed by CUDA events with a device spin ahead of each step (host issue latency "
+                          "hidden); on some boxes the GPU idling through the spin slows the step after it, so "
+                          "that figure can exceed the host's"},
         "other_workloads": others,
         "gpu_launches": step_launches * args.steps,
         "gpu_launches_decode_roofline_loop": decode_launches * n_dec,

@@ -65,7 +65,7 @@ def test_decode_bench_line_has_the_contract_fields(bench, capsys, workload, batc
         assert st["p10"] <= st["median"] <= st["p90"] and st["n"] >= 3
     assert d["decode_attention_ms"]["n"] >= 100
     assert r["read_ceiling_gbs"] > 0 and abs(r["frac_of_read_ceiling"] - r["achieved"] / r["read_ceiling_gbs"]) < 1e-9
-    assert e["host_wall_ms_per_step"] > 0
+    assert e["device_ms_per_step"] > 0 and e["ms_stats"]["n"] == d["steps"]
     assert d["other_workloads"] is None
     if workload == "cow":
         assert d["unique_kv"]["bytes_per_step"] < d["config"]["kv_bytes_per_step"]
