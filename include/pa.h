@@ -315,9 +315,12 @@ int pa_paged_attention_shared_prefix_workspace_size(int batch, int num_q_heads, 
  * tables and lengths (within rounding: the softmax is split at different
  * points), but each shared block is read from memory once per group instead
  * of once per member: a prefix pass attends the group's shared tokens for
- * all its members' query heads at once (tensor cores, queries stacked on the
- * MMA's M side), pass 1 attends each member's own tokens after the prefix,
- * and the merge pass combines the two.
+ * all its members' query heads at once (tensor cores: for head_dim 128 the
+ * shared tokens are the M side of tcgen05 MMAs and the query heads their N
+ * side; for 64 the query heads are stacked on the M side of mma.sync), pass
+ * 1 attends each member's own tokens after the prefix and folds the prefix
+ * in, and the merge pass combines the two where a member's own tokens span
+ * several splits.
  *   group_starts       int32 [num_groups + 1], device: group g is sequences
  *                      group_starts[g] .. group_starts[g + 1] - 1, with
  *                      group_starts[0] = 0, non-decreasing,
