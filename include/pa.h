@@ -295,7 +295,8 @@ int pa_paged_attention_decode_append(const void* q, const void* key, const void*
 /*
  * pa_paged_attention_shared_prefix_workspace_size -- bytes of scratch that
  * pa_paged_attention_decode_shared_prefix needs for these sizes (always > 0:
- * the prefix pass's partial results and each sequence's prefix length).
+ * the partial results, each sequence's prefix length and, when the prefix
+ * pass runs last, one counter).
  * num_groups >= 1, max_group_size >= 1, 0 <= max_prefix_len <=
  * max_context_len; partition_size as for pa_paged_attention_decode.
  */
@@ -317,10 +318,17 @@ int pa_paged_attention_shared_prefix_workspace_size(int batch, int num_q_heads, 
  * of once per member: a prefix pass attends the group's shared tokens for
  * all its members' query heads at once (tensor cores: for head_dim 128 the
  * shared tokens are the M side of tcgen05 MMAs and the query heads their N
- * side; for 64 the query heads are stacked on the M side of mma.sync), pass
- * 1 attends each member's own tokens after the prefix and folds the prefix
- * in, and the merge pass combines the two where a member's own tokens span
- * several splits.
+ * side; for 64 the query heads are stacked on the M side of mma.sync), and
+ * pass 1 attends each member's own tokens after the prefix.  For head_dim
+ * 128, when the prefix is one split (at most the prefix partition, 4096
+ * tokens by default) and the own tokens one split, a one-CTA set-up kernel
+ * checks the groups and stores each sequence's prefix length, pass 1 runs
+ * next and stores each own part's partial result, and the prefix pass runs
+ * last -- its CTAs start as pass 1's last wave drains -- and writes every
+ * shared row, its own state combined with pass 1's partial by the
+ * log-sum-exp rescale.  Otherwise the prefix pass runs first, pass 1 folds
+ * the prefix in, and the merge pass combines the two where a member's own
+ * tokens span several splits.
  *   group_starts       int32 [num_groups + 1], device: group g is sequences
  *                      group_starts[g] .. group_starts[g + 1] - 1, with
  *                      group_starts[0] = 0, non-decreasing,

@@ -113,6 +113,17 @@ struct DecodeParams {
     const void* v_new;
     int64_t* slots;
     int append;
+    // shared-prefix calls: pass 1 has room after its ring for the one prefix
+    // partial it folds into a row (G rows of D floats, then their (m, l))
+    int fold_prefetch;
+    // shared-prefix calls with one prefix split and one own split, head_dim
+    // 128: a set-up kernel checks the groups and writes seq_prefix, pass 1
+    // runs next and stores each own part's partial in slot 1, and the
+    // tensor-core prefix pass runs last, beside pass 1's tail, and finishes
+    // every row (its own state folded with slot 1).  done_count counts the
+    // prefix pass's finished CTAs.
+    int prefix_last;
+    int* done_count;
     // shared-prefix decode: sequences [group_starts[g], group_starts[g + 1])
     // share their first group_prefix[g] tokens (whole blocks, the same
     // physical ids in every member's table).  The prefix pass attends each
@@ -160,6 +171,14 @@ struct Elt<__nv_bfloat16> {
     }
 };
 
+__device__ __forceinline__ int clamp_len_value(const DecodeParams& p, int L, bool report) {
+    if (L < 0 || (int64_t)L > p.max_len) {
+        if (report) record_error(p.err, PA_ERR_BAD_BLOCK_ID);
+        L = L < 0 ? 0 : (int)p.max_len;
+    }
+    return L;
+}
+
 __device__ __forceinline__ int clamp_len(const DecodeParams& p, int b, bool report) {
     int L = p.context_lens[b];
     if (L < 0 || (int64_t)L > p.max_len) {
@@ -205,137 +224,95 @@ __device__ __forceinline__ void store_out(const DecodeParams& p, int64_t idx, fl
 // merge pass).
 constexpr int kMaxFoldSplits = 16;
 
-// A row whose only other splits are prefix splits (written by the prefix
-// pass, which has completed) is finished in pass 1: the prefix partials are
-// combined with the CTA's own state by the log-sum-exp rescale the merge
-// pass applies.  First the rows' coefficients (one thread per row, all
-// (m, l) loads issued together), then the output elements, four per thread
-// at a time with all their partial-row loads issued before any is used.
-__device__ __forceinline__ void fold_prefix_and_store(const DecodeParams& p, const float* sm_o, const float* sm_m,
-                                                      const float* sm_l, float* coef, int G, int D, int b, int kvh,
-                                                      int sp) {
-    constexpr int K = kMaxFoldSplits;
-    for (int h = threadIdx.x; h < G; h += blockDim.x) {
-        const int64_t qrow = (int64_t)b * p.num_q_heads + (int64_t)kvh * G + h;
-        const float* ml = p.part_ml + qrow * p.max_splits * 2;
-        float mv[K], lv[K];
-#pragma unroll
-        for (int s = 0; s < K; ++s) {
-            mv[s] = s < sp ? ml[2 * s] : -INFINITY;
-            lv[s] = s < sp ? ml[2 * s + 1] : 0.f;
-        }
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_m[w * G + h]);
-        float lt = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) {
-                const float mw = sm_m[w * G + h];
-                lt += mw == -INFINITY ? 0.f : sm_l[w * G + h] * exp2f(mw - M);
-            }
-        }
-        float Mt = M;
-#pragma unroll
-        for (int s = 0; s < K; ++s) Mt = fmaxf(Mt, mv[s]);
-        float W = 0.f, own = 0.f, ws[K];
-#pragma unroll
-        for (int s = 0; s < K; ++s) ws[s] = 0.f;
-        if (Mt != -INFINITY) {
-            if (M != -INFINITY) {
-                own = exp2f(M - Mt);
-                W = lt * own;
-            }
-#pragma unroll
-            for (int s = 0; s < K; ++s) {
-                ws[s] = mv[s] == -INFINITY ? 0.f : lv[s] * exp2f(mv[s] - Mt);
-                W += ws[s];
-            }
-        }
-        const float inv = W > 0.f ? 1.f / W : 0.f;
-        coef[h * (K + 1)] = own * inv;
-#pragma unroll
-        for (int s = 0; s < K; ++s) coef[h * (K + 1) + 1 + s] = ws[s] * inv;
-    }
-    __syncthreads();
-    constexpr int E = 4;
-    for (int base = threadIdx.x; base < G * D; base += E * blockDim.x) {
-        float pv[E][K];
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-            const int idx = base + e * blockDim.x;
-            const int h = idx / D;
-            const int d = idx - h * D;
-            const float* po = p.part_o + ((int64_t)b * p.num_q_heads + (int64_t)kvh * G + h) * p.max_splits * D + d;
-#pragma unroll
-            for (int s = 0; s < K; ++s) pv[e][s] = (idx < G * D && s < sp) ? po[(int64_t)s * D] : 0.f;
-        }
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-            const int idx = base + e * blockDim.x;
-            if (idx >= G * D) break;
-            const int h = idx / D;
-            const int d = idx - h * D;
-            float M = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_m[w * G + h]);
-            float ot = 0.f;
-            if (M != -INFINITY) {
-#pragma unroll
-                for (int w = 0; w < kConsumerWarps; ++w) {
-                    const float mw = sm_m[w * G + h];
-                    ot += mw == -INFINITY ? 0.f : sm_o[(w * G + h) * D + d] * exp2f(mw - M);
-                }
-            }
-            float acc = ot * coef[h * (K + 1)];
-#pragma unroll
-            for (int s = 0; s < K; ++s) acc = fmaf(coef[h * (K + 1) + 1 + s], pv[e][s], acc);
-            store_out(p, ((int64_t)b * p.num_q_heads + (int64_t)kvh * G + h) * D + d, acc);
-        }
-    }
-}
+// Shared scratch of the epilogue merge, per query head: one factor per
+// consumer warp's accumulator, then one per prefix split folded in.
+constexpr int kCoefStride = kConsumerWarps + kMaxFoldSplits;
 
 // Combine the consumer warps' (m, l, o) states of one work item, held in
 // shared memory as o[w][h][d], m[w][h], l[w][h], and write the final row (one
-// split) or the normalised partial row plus (m, l) for the merge kernel; with
-// prefix splits and one own split, fold the prefix in (above).  `coef` is
-// shared scratch of G * (kMaxFoldSplits + 1) floats.
+// split) or the normalised partial row plus (m, l) for the merge kernel.
+// First one thread per row turns the row's maxima and sums into one factor
+// per warp (and per folded prefix split), then every output element is a
+// short dot product of the warps' (and splits') values with those factors.
+// With prefix splits and one own split (`fold`), the row is finished here:
+// the prefix pass's partials (complete before this grid started) are
+// combined with the CTA's own state by the log-sum-exp rescale the merge
+// pass applies.  `pf` (one prefix split only): that split's partial already
+// copied into shared memory as G rows of D floats followed by the rows'
+// (m, l).  `coef` is shared scratch of G * kCoefStride floats.
 __device__ __forceinline__ void merge_warps_and_store(const DecodeParams& p, const float* sm_o, const float* sm_m,
-                                                      const float* sm_l, int G, int D, int b, int kvh, int split,
-                                                      int num_splits_b, int prefix_splits = 0,
-                                                      float* coef = nullptr) {
-    if (coef && prefix_splits > 0 && prefix_splits <= kMaxFoldSplits && num_splits_b == prefix_splits + 1) {
-        fold_prefix_and_store(p, sm_o, sm_m, sm_l, coef, G, D, b, kvh, prefix_splits);
-        return;
-    }
-    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-        const int h = idx / D;
-        const int d = idx - h * D;
+                                                      const float* sm_l, float* coef, int G, int D, int b, int kvh,
+                                                      int split, int num_splits_b, int prefix_splits = 0,
+                                                      bool fold = false, const float* pf = nullptr) {
+    const int sp = (fold && prefix_splits > 0 && prefix_splits <= kMaxFoldSplits && num_splits_b == prefix_splits + 1)
+                       ? prefix_splits
+                       : 0;
+    const bool final_row = num_splits_b == 1 || sp > 0;
+    for (int h = threadIdx.x; h < G; h += blockDim.x) {
+        const int64_t qrow = (int64_t)b * p.num_q_heads + (int64_t)kvh * G + h;
+        float* c = coef + h * kCoefStride;
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_m[w * G + h]);
-        float lt = 0.f, ot = 0.f;
-        if (M != -INFINITY) {
+        float a[kConsumerWarps], lt = 0.f;
 #pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) {
-                const float mw = sm_m[w * G + h];
-                const float a = mw == -INFINITY ? 0.f : exp2f(mw - M);
-                lt += sm_l[w * G + h] * a;
-                ot += sm_o[(w * G + h) * D + d] * a;
-            }
+        for (int w = 0; w < kConsumerWarps; ++w) {
+            const float mw = sm_m[w * G + h];
+            a[w] = mw == -INFINITY ? 0.f : exp2f(mw - M);
+            lt += sm_l[w * G + h] * a[w];
         }
-        const float val = lt > 0.f ? ot / lt : 0.f;
-        const int64_t qrow = (int64_t)b * p.num_q_heads + (int64_t)kvh * G + h;
-        if (num_splits_b == 1) {
-            store_out(p, qrow * D + d, val);
-        } else {
-            const int64_t r = qrow * p.max_splits + split;
-            p.part_o[r * D + d] = val;
-            if (d == 0) {
+        if (sp == 0) {
+            const float inv = lt > 0.f ? 1.f / lt : 0.f;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) c[w] = a[w] * inv;
+            if (!final_row) {
+                const int64_t r = qrow * p.max_splits + split;
                 p.part_ml[2 * r] = M;
                 p.part_ml[2 * r + 1] = lt;
             }
+        } else {
+            const float* ml = pf ? pf + G * D + 2 * h : p.part_ml + qrow * p.max_splits * 2;
+            float Mt = M;
+            for (int s = 0; s < sp; ++s) Mt = fmaxf(Mt, ml[2 * s]);
+            const float own = M == -INFINITY ? 0.f : exp2f(M - Mt);
+            float W = lt * own;
+            for (int s = 0; s < sp; ++s) {
+                const float ms = ml[2 * s];
+                const float ws = ms == -INFINITY ? 0.f : ml[2 * s + 1] * exp2f(ms - Mt);
+                c[kConsumerWarps + s] = ws;
+                W += ws;
+            }
+            const float inv = W > 0.f ? 1.f / W : 0.f;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) c[w] = a[w] * own * inv;
+            for (int s = 0; s < sp; ++s) c[kConsumerWarps + s] *= inv;
         }
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+        const int h = idx / D;
+        const int d = idx - h * D;
+        const int64_t qrow = (int64_t)b * p.num_q_heads + (int64_t)kvh * G + h;
+        const float* c = coef + h * kCoefStride;
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) acc = fmaf(sm_o[(w * G + h) * D + d], c[w], acc);
+        if (sp > 0) {
+            const float* po = pf ? pf + h * D + d : p.part_o + qrow * p.max_splits * D + d;
+            // four splits' loads in flight at a time
+            for (int s0 = 0; s0 < sp; s0 += 4) {
+                float v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) v[u] = s0 + u < sp ? po[(int64_t)(s0 + u) * D] : 0.f;
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (s0 + u < sp) acc = fmaf(c[kConsumerWarps + s0 + u], v[u], acc);
+            }
+        }
+        if (final_row)
+            store_out(p, qrow * D + d, acc);
+        else
+            p.part_o[(qrow * p.max_splits + split) * D + d] = acc;
     }
 }
 
@@ -665,7 +642,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const Deco
         }
     }
     __syncthreads();
-    merge_warps_and_store(p, sm_o, sm_m, sm_l, G, D, b, kvh, split, num_splits_b);
+    merge_warps_and_store(p, sm_o, sm_m, sm_l, sm_l + kConsumerWarps * G, G, D, b, kvh, split, num_splits_b);
 }
 
 // ---------------------------------------------------------------------------
@@ -723,22 +700,30 @@ __global__ void __launch_bounds__(kDecodeThreads)
     const int lane = threadIdx.x & 31;
     const int G = p.num_q_heads / p.num_kv_heads;
 
-    const int L = clamp_len(p, b, threadIdx.x == 0 && split == 0 && kvh == 0);
+    // the length and the prefix length, loaded together
+    const int len_raw = p.context_lens[b];
+    const int pre_raw = p.seq_prefix ? p.seq_prefix[b] : 0;
+    const int L = clamp_len_value(p, len_raw, threadIdx.x == 0 && split == 0 && kvh == 0);
     // A length beyond max_context_len is clamped for the attention (and
     // flagged), but the folded write still goes to the slot of the length as
     // given, where pa_reshape_and_cache_decode puts it: split 0 writes it
     // directly, outside the (clamped) range any CTA of this launch reads.
-    const bool overflow = p.append && p.context_lens[b] > p.max_len;
+    const bool overflow = p.append && len_raw > p.max_len;
     if (p.append && !overflow && L == 0 && split == 0 && kvh == 0 && threadIdx.x == 0 && p.slots) p.slots[b] = -1;
     // with shared prefixes this pass covers the tokens after the sequence's
     // prefix, and its splits' partial results follow the prefix splits' slots
-    const int pre = seq_prefix_len(p, b, L);
+    const int pre = clamp_prefix(p, pre_raw, L);
     const int tok_begin = pre + split * p.partition;
     if (split > 0 && tok_begin >= L) return;
     const int ntok = max(0, min(L, tok_begin + p.partition) - tok_begin);
     const int nstage = (ntok + kStageTokens - 1) / kStageTokens;
     int prefix_splits;
     const int num_splits_b = row_splits(p, L, pre, &prefix_splits);
+    // one prefix split to fold in: its partial is copied to shared memory
+    // (after the ring) while the last stages are consumed
+    float* pf = (p.fold_prefetch && prefix_splits == 1 && num_splits_b == 2)
+                    ? reinterpret_cast<float*>(ring + (size_t)p.stages * 2 * STAGE_BYTES)
+                    : nullptr;
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -838,6 +823,26 @@ __global__ void __launch_bounds__(kDecodeThreads)
                     tma_load_2d(vdst + sl * SLAB_BYTES + r * 128, &tmv, sl * 64, y, &full[slot], policy);
                 }
             }
+        }
+        if (pf) {
+            // the prefix partial (complete before this grid started): rows of
+            // the G heads, four float4 per lane in flight, then their (m, l)
+            const int64_t qrow0 = (int64_t)b * p.num_q_heads + (int64_t)kvh * G;
+            const int nv = G * D / 4;
+            for (int i0 = lane; i0 < nv; i0 += 4 * 32) {
+                float4 v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int i = i0 + 32 * u;
+                    if (i < nv)
+                        v[u] = *reinterpret_cast<const float4*>(p.part_o + (qrow0 + i / (D / 4)) * p.max_splits * D +
+                                                                (i % (D / 4)) * 4);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (i0 + 32 * u < nv) reinterpret_cast<float4*>(pf)[i0 + 32 * u] = v[u];
+            }
+            if (lane < 2 * G) pf[G * D + lane] = p.part_ml[(qrow0 + lane / 2) * p.max_splits * 2 + (lane & 1)];
         }
     } else {
         // ---------------- consumers ----------------
@@ -1079,8 +1084,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
         }
     }
     __syncthreads();
-    merge_warps_and_store(p, sm_o, sm_m, sm_l, G, D, b, kvh, prefix_splits + split, num_splits_b, prefix_splits,
-                          sm_l + kConsumerWarps * G);
+    merge_warps_and_store(p, sm_o, sm_m, sm_l, sm_l + kConsumerWarps * G, G, D, b, kvh, prefix_splits + split,
+                          num_splits_b, prefix_splits, !p.prefix_last, pf);
 }
 
 // ---------------------------------------------------------------------------
@@ -1126,35 +1131,81 @@ struct PrefixGroup {
     int prefix;
 };
 
+// Group grp's description as given (one thread): its span, its prefix length
+// if the description keeps the rules that need no member's length (else 0
+// and `bad`).  A well-formed span gets its members' prefix lengths written in
+// any case (0 when the group cannot share); a malformed one names no
+// members, and the sequences it should have covered stay unspecified.  The
+// reporter CTA flags groups that do not cover the batch.
+__device__ __forceinline__ void prefix_group_describe(const DecodeParams& p, int grp, bool reporter, int& start,
+                                                      int& n, int& prefix, int& bad) {
+    const int s = p.group_starts[grp], e = p.group_starts[grp + 1], P = p.group_prefix[grp];
+    const bool span_ok = s >= 0 && e >= s && e <= p.batch;
+    const bool ok = span_ok && e - s <= p.max_group && P >= 0 && P <= p.max_prefix && P % p.block_size == 0;
+    start = span_ok ? s : 0;
+    n = span_ok ? e - s : 0;
+    prefix = ok ? P : 0;
+    bad = !ok;
+    if (reporter && ((grp == 0 && s != 0) || (grp == p.num_groups - 1 && e != p.batch)))
+        record_error(p.err, PA_ERR_BAD_BLOCK_ID);  // the groups do not cover the batch
+}
+
+// The verdict, once every member's length has been checked against the
+// prefix (`bad` set by any member shorter than it): the reporter CTA flags a
+// bad description and writes each member's prefix length to seq_prefix.
+// Called by all threads, after a barrier that follows the checks.
+__device__ __forceinline__ PrefixGroup prefix_group_verdict(const DecodeParams& p, bool reporter, int start, int n,
+                                                            int prefix, int bad) {
+    const PrefixGroup g{start, n, bad ? 0 : prefix};
+    if (reporter) {
+        if (threadIdx.x == 0 && bad) record_error(p.err, PA_ERR_BAD_BLOCK_ID);
+        for (int m = threadIdx.x; m < g.n; m += blockDim.x) p.seq_prefix[g.start + m] = g.prefix;
+    }
+    return g;
+}
+
 // Check group grp's description; every CTA of the group reaches the same
-// verdict.  The reporter CTA (one per group) flags a bad description and
-// writes each member's prefix length to seq_prefix.  Called by all threads.
+// verdict.  Called by all threads.
 __device__ PrefixGroup prefix_group_setup(const DecodeParams& p, int grp, bool reporter) {
     __shared__ int s_start, s_n, s_prefix, s_bad;
-    if (threadIdx.x == 0) {
-        const int s = p.group_starts[grp], e = p.group_starts[grp + 1], P = p.group_prefix[grp];
-        // a well-formed span gets its members' prefix lengths written in any
-        // case (0 when the group cannot share); a malformed one names no
-        // members, and the sequences it should have covered stay unspecified
-        const bool span_ok = s >= 0 && e >= s && e <= p.batch;
-        const bool ok = span_ok && e - s <= p.max_group && P >= 0 && P <= p.max_prefix && P % p.block_size == 0;
-        s_start = span_ok ? s : 0;
-        s_n = span_ok ? e - s : 0;
-        s_prefix = ok ? P : 0;
-        s_bad = !ok;
-        if (reporter && ((grp == 0 && s != 0) || (grp == p.num_groups - 1 && e != p.batch)))
-            record_error(p.err, PA_ERR_BAD_BLOCK_ID);  // the groups do not cover the batch
-    }
+    if (threadIdx.x == 0) prefix_group_describe(p, grp, reporter, s_start, s_n, s_prefix, s_bad);
     __syncthreads();
     for (int m = threadIdx.x; m < s_n; m += blockDim.x)
         if (clamp_len(p, s_start + m, false) < s_prefix) s_bad = 1;  // a member shorter than the prefix
     __syncthreads();
-    const PrefixGroup g{s_start, s_n, s_bad ? 0 : s_prefix};
-    if (reporter) {
-        if (threadIdx.x == 0 && s_bad) record_error(p.err, PA_ERR_BAD_BLOCK_ID);
-        for (int m = threadIdx.x; m < g.n; m += blockDim.x) p.seq_prefix[g.start + m] = g.prefix;
+    return prefix_group_verdict(p, reporter, s_start, s_n, s_prefix, s_bad);
+}
+
+// Prefix-last order: the groups' descriptions, checked once per call before
+// pass 1 (one CTA).  Every sequence's prefix length in seq_prefix starts at 0;
+// then each member of a well-formed group gets the group's prefix length.  A
+// description that breaks the preconditions is flagged, and its sequences
+// keep prefix 0 (attended without sharing).  The rules are those of
+// prefix_group_describe and prefix_group_setup, so the prefix pass reaches
+// the same verdict on its own.  Also clears the prefix pass's exit counter.
+__global__ void __launch_bounds__(1024) decode_prefix_setup_kernel(const DecodeParams p) {
+    griddep_wait();  // lengths and descriptions may come from the kernel before
+    griddep_launch_dependents();
+    for (int b = threadIdx.x; b < p.batch; b += blockDim.x) p.seq_prefix[b] = 0;
+    if (threadIdx.x == 0) *p.done_count = 0;
+    __syncthreads();
+    for (int g = threadIdx.x; g < p.num_groups; g += blockDim.x) {
+        int start, n, P, bad;
+        prefix_group_describe(p, g, true, start, n, P, bad);
+        for (int m0 = start; !bad && m0 < start + n; m0 += 8) {
+            // a member shorter than the prefix (eight lengths in flight)
+            int Lm[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) Lm[u] = m0 + u < start + n ? clamp_len(p, m0 + u, false) : P;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) bad |= Lm[u] < P;
+        }
+        if (bad) {
+            record_error(p.err, PA_ERR_BAD_BLOCK_ID);
+            continue;
+        }
+        for (int m = start; m < start + n; ++m) p.seq_prefix[m] = P;
     }
-    return g;
 }
 
 template <int D, int MT, int PAR>
@@ -1534,6 +1585,16 @@ __global__ void __launch_bounds__(32 * (1 + MT * PAR), 3)
 //    normalised partial (as float4 rows) and (m, l), as the mma.sync pass
 //    does.
 // ---------------------------------------------------------------------------
+// Prefix-last order: the prefix pass's grid must not complete before pass 1
+// (kernels after the call wait for the prefix pass only).  CTAs with work wait
+// for pass 1 before their epilogue; to cover a grid in which none has work,
+// the last CTA to finish waits too.  One thread per CTA, at its exit.
+__device__ __forceinline__ void prefix_last_exit(const DecodeParams& p) {
+    if (!p.prefix_last) return;
+    const unsigned total = gridDim.x * gridDim.y * gridDim.z;
+    if (atomicAdd(reinterpret_cast<unsigned*>(p.done_count), 1u) == total - 1) griddep_wait();
+}
+
 constexpr int kTcTokens = 128;         // shared tokens per tile (M of S^T)
 constexpr int kTcRows = 32;            // query rows per CTA (N of both MMAs)
 constexpr int kTcThreads = 64 + 128;   // producer, MMA issuer, softmax warpgroup
@@ -1601,13 +1662,20 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     __shared__ uint64_t k_full, k_empty, v_full, v_empty, s_full[2], p_full, pv_done;
     __shared__ uint32_t tmem_base;
     __shared__ int64_t row_off[N];  // epilogue: element offset of row r's partial, or -1
-    __shared__ float row_inv[N];    //           1 / row sum
+    __shared__ float row_inv[N];    //           factor of the row's own O (1 / row sum)
+    __shared__ float row_c1[N];     //           prefix-last order: factor of pass 1's partial
+    __shared__ int64_t row_own[N];  //           prefix-last order: element offset of pass 1's partial
 
     if (threadIdx.x == 0) {
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
     }
-    griddep_wait();  // q, lengths, tables and the pool may come from the kernel before
+    // q, lengths, tables and the pool may come from the kernel before.  In the
+    // prefix-last order that kernel is pass 1, which waited for the set-up
+    // kernel (which waited for the kernels before the call) before this grid
+    // could start: the inputs are final, and only pass 1's partial results,
+    // read in the epilogue, need the wait, taken there.
+    if (!p.prefix_last) griddep_wait();
     griddep_launch_dependents();
     const int split = blockIdx.x;
     const int kvh = blockIdx.y % p.num_kv_heads;
@@ -1615,11 +1683,78 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int G = p.num_q_heads / p.num_kv_heads;
-    const PrefixGroup grp = prefix_group_setup(p, blockIdx.z, split == 0 && blockIdx.y == 0);
+    // the set-up kernel reports (and writes seq_prefix) in the prefix-last order
+    const bool reporter = !p.prefix_last && split == 0 && blockIdx.y == 0;
+    // Tensor memory first: the SM schedules a second CTA of this kernel only
+    // once the first has given up its allocation permit.
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&tmem_base)),
+                     "r"(kTcTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    __shared__ int d_start, d_n, d_prefix, d_bad;
+    if (threadIdx.x == 0) prefix_group_describe(p, blockIdx.z, reporter, d_start, d_n, d_prefix, d_bad);
+    __syncthreads();
     const int tok_begin = split * p.prefix_partition;
-    const int rows_total = grp.n * G;
     const int row0 = chunk * N;
-    if (tok_begin >= grp.prefix || row0 >= rows_total) return;  // uniform over the CTA, before any barrier
+    {
+        // One round trip for the rest of the prologue: the members' lengths
+        // (the check of the prefix against them), and, for the group as
+        // described, the split's slice of the shared blocks (from the first
+        // member's table) and the chunk's query rows, staged K-major with the
+        // 128-byte swizzle (16-byte chunk c of row r of a slab at c ^ (r & 7),
+        // zero past the group).  All loads are issued before any is used.
+        const int rows_d = d_n * G;
+        const bool work = row0 < rows_d && tok_begin < d_prefix;
+        const int nblk_d = work ? (min(d_prefix, tok_begin + p.prefix_partition) - tok_begin + p.block_size - 1) /
+                                      p.block_size
+                                : 0;
+        const int32_t* row = p.block_tables + (int64_t)d_start * p.max_blocks_per_seq + tok_begin / p.block_size;
+        const uint16_t* qv = static_cast<const uint16_t*>(p.q);
+        constexpr int QV = (N * (D / 8) + kTcThreads - 1) / kTcThreads;  // 16-byte query chunks per thread
+        uint4 qr[QV];
+#pragma unroll
+        for (int u = 0; u < QV; ++u) {
+            const int i = threadIdx.x + u * kTcThreads;
+            const int r = i / (D / 8);
+            const int c = i % (D / 8);
+            const int gr = row0 + r;
+            qr[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (work && i < N * (D / 8) && gr < rows_d)
+                qr[u] = *reinterpret_cast<const uint4*>(
+                    qv + ((int64_t)(d_start + gr / G) * p.num_q_heads + (int64_t)kvh * G + gr % G) * D + c * 8);
+        }
+        int tv[2];
+        for (int i0 = threadIdx.x; i0 < nblk_d; i0 += 2 * kTcThreads) {
+#pragma unroll
+            for (int u = 0; u < 2; ++u) tv[u] = i0 + u * kTcThreads < nblk_d ? row[i0 + u * kTcThreads] : 0;
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+                if (i0 + u * kTcThreads < nblk_d) tbl[i0 + u * kTcThreads] = tv[u];
+        }
+        for (int m = threadIdx.x; m < d_n; m += kTcThreads)
+            if (clamp_len(p, d_start + m, false) < d_prefix) d_bad = 1;  // a member shorter than the prefix
+#pragma unroll
+        for (int u = 0; u < QV; ++u) {
+            const int i = threadIdx.x + u * kTcThreads;
+            const int r = i / (D / 8);
+            const int c = i % (D / 8);
+            if (i < N * (D / 8))
+                *reinterpret_cast<uint4*>(sQ + (c >> 3) * kTcQSlab + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = qr[u];
+        }
+        fence_proxy_async_smem();  // the tensor core reads Q through the async proxy
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base;
+    const PrefixGroup grp = prefix_group_verdict(p, reporter, d_start, d_n, d_prefix, d_bad);
+    const int rows_total = grp.n * G;
+    if (tok_begin >= grp.prefix || row0 >= rows_total) {  // uniform over the CTA
+        if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcTmemCols));
+        if (threadIdx.x == 0) prefix_last_exit(p);
+        return;
+    }
     const int ntok = min(grp.prefix, tok_begin + p.prefix_partition) - tok_begin;
     const int nt = (ntok + kTcTokens - 1) / kTcTokens;
 
@@ -1634,36 +1769,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         mbar_init(&pv_done, 1);
         fence_barrier_init();
     }
-    {
-        // the shared blocks, from the first member's table
-        const int first_blk = tok_begin / p.block_size;
-        const int nblk = (ntok + p.block_size - 1) / p.block_size;
-        const int32_t* row = p.block_tables + (int64_t)grp.start * p.max_blocks_per_seq + first_blk;
-        for (int i = threadIdx.x; i < nblk; i += blockDim.x) tbl[i] = row[i];
-        // the chunk's query rows (zero past the group), K-major with the
-        // 128-byte swizzle: 16-byte chunk c of row r of a slab at c ^ (r & 7)
-        const uint16_t* qv = static_cast<const uint16_t*>(p.q);
-        for (int i = threadIdx.x; i < N * (D / 8); i += blockDim.x) {
-            const int r = i / (D / 8);
-            const int c = i % (D / 8);
-            const int gr = row0 + r;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (gr < rows_total)
-                v = *reinterpret_cast<const uint4*>(
-                    qv + ((int64_t)(grp.start + gr / G) * p.num_q_heads + (int64_t)kvh * G + gr % G) * D + c * 8);
-            *reinterpret_cast<uint4*>(sQ + (c >> 3) * kTcQSlab + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
-        }
-        fence_proxy_async_smem();  // the tensor core reads Q through the async proxy
-    }
-    if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&tmem_base)),
-                     "r"(kTcTmemCols));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-    }
-    tc_fence_before();
     __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = tmem_base;
 
     if (warp == 0) {
         // ---------------- producer ----------------
@@ -1890,23 +1996,47 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 #pragma unroll
             for (int r = 0; r < N; ++r) so[r * D + tok] = ov[r];
             consumer_barrier(1, 128);
+            // prefix-last order: pass 1's partial results are needed now
+            if (p.prefix_last) griddep_wait();
             if (q4 == 0) {
-                // row `lane`: its slot, 1 / l, and (m, l)
+                // row `lane`: where it goes and its factors
                 const float lt = (red[lane] + red[N + lane]) + (red[2 * N + lane] + red[3 * N + lane]);
                 float mr = m[0];
 #pragma unroll
                 for (int r = 1; r < N; ++r) mr = lane == r ? m[r] : mr;
                 const int gr = row0 + lane;
-                int64_t off = -1;
+                int64_t off = -1, own = -1;
+                float c0 = 0.f, c1 = 0.f;
                 if (gr < rows_total) {
                     const int64_t qrow = (int64_t)(grp.start + gr / G) * p.num_q_heads + (int64_t)kvh * G + gr % G;
-                    const int64_t slotrow = qrow * p.max_splits + split;
-                    off = slotrow * D;
-                    p.part_ml[2 * slotrow] = mr;
-                    p.part_ml[2 * slotrow + 1] = lt;
+                    if (p.prefix_last) {
+                        // the final row: this split's state folded with pass
+                        // 1's partial of the own tokens (slot 1) by the
+                        // log-sum-exp rescale
+                        const int64_t r1 = qrow * p.max_splits + 1;
+                        const float m1 = __ldcg(p.part_ml + 2 * r1), l1 = __ldcg(p.part_ml + 2 * r1 + 1);
+                        const float Mt = fmaxf(mr, m1);
+                        const float a0 = mr == -INFINITY ? 0.f : exp2f(mr - Mt);
+                        const float w1 = m1 == -INFINITY ? 0.f : l1 * exp2f(m1 - Mt);
+                        const float W = lt * a0 + w1;
+                        const float inv = W > 0.f ? 1.f / W : 0.f;
+                        c0 = a0 * inv;
+                        c1 = w1 * inv;
+                        off = qrow * D;
+                        own = r1 * D;
+                    } else {
+                        // the normalised partial and (m, l) in the split's slot
+                        const int64_t slotrow = qrow * p.max_splits + split;
+                        off = slotrow * D;
+                        p.part_ml[2 * slotrow] = mr;
+                        p.part_ml[2 * slotrow + 1] = lt;
+                        c0 = lt > 0.f ? 1.f / lt : 0.f;
+                    }
                 }
                 row_off[lane] = off;
-                row_inv[lane] = lt > 0.f ? 1.f / lt : 0.f;
+                row_inv[lane] = c0;
+                row_c1[lane] = c1;
+                row_own[lane] = own;
             }
             consumer_barrier(1, 128);
             // each row's 128 elements as 32 float4, one row per warp step
@@ -1915,13 +2045,28 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                 const int r = i / (D / 4);
                 const int64_t off = row_off[r];
                 if (off >= 0) {
+                    const int c = (i % (D / 4)) * 4;
                     float4 o = so4[i];
-                    const float inv = row_inv[r];
-                    o.x *= inv;
-                    o.y *= inv;
-                    o.z *= inv;
-                    o.w *= inv;
-                    *reinterpret_cast<float4*>(p.part_o + off + (i % (D / 4)) * 4) = o;
+                    const float c0 = row_inv[r];
+                    o.x *= c0;
+                    o.y *= c0;
+                    o.z *= c0;
+                    o.w *= c0;
+                    if (p.prefix_last) {
+                        const float c1 = row_c1[r];
+                        const float4 o1 = __ldcg(reinterpret_cast<const float4*>(p.part_o + row_own[r] + c));
+                        o.x = fmaf(c1, o1.x, o.x);
+                        o.y = fmaf(c1, o1.y, o.y);
+                        o.z = fmaf(c1, o1.z, o.z);
+                        o.w = fmaf(c1, o1.w, o.w);
+                        if (p.out_bf16)
+                            *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + off + c) =
+                                make_uint2(pack_bf16x2(o.x, o.y), pack_bf16x2(o.z, o.w));
+                        else
+                            *reinterpret_cast<float4*>(static_cast<float*>(p.out) + off + c) = o;
+                    } else {
+                        *reinterpret_cast<float4*>(p.part_o + off + c) = o;
+                    }
                 }
             }
         }
@@ -1932,6 +2077,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcTmemCols));
     }
+    if (threadIdx.x == 0) prefix_last_exit(p);
 }
 
 // Second pass: out = sum_s w_s o_s / sum_s w_s with w_s = l_s * 2^(m_s - max m),
@@ -2052,6 +2198,7 @@ struct Plan {
     size_t part_o_bytes;
     size_t part_ml_bytes;
     size_t seq_prefix_bytes;
+    size_t done_bytes;
     size_t workspace;
     // shared-prefix calls only
     int prefix_partition;
@@ -2059,6 +2206,9 @@ struct Plan {
     int tc;      // head_dim 128: the tensor-core (tcgen05) prefix pass, 32 query rows per CTA
     int mt;      // otherwise: 16-row query tiles per prefix CTA (consumer warps)
     int chunks;  // prefix CTAs per (group, kv head) along the query rows
+    // one prefix split and one own split on the tensor-core path: set-up
+    // kernel, pass 1, then the prefix pass, which finishes the rows
+    int prefix_last;
 };
 
 constexpr int kPrefixRingBytes = 64 * 1024;
@@ -2118,13 +2268,15 @@ int make_plan(int batch, int num_q_heads, int num_kv_heads, int head_dim, int ma
         plan->prefix_splits = max_prefix > 0 ? (max_prefix + plan->prefix_partition - 1) / plan->prefix_partition : 0;
         plan->max_splits = plan->prefix_splits + splits;
         plan->seq_prefix_bytes = align256((size_t)batch * sizeof(int32_t));
+        plan->prefix_last = plan->tc && plan->prefix_splits == 1 && plan->suffix_splits == 1;
+        plan->done_bytes = plan->prefix_last ? 256 : 0;
     }
     if (plan->max_splits > 1) {
         const size_t rows = (size_t)batch * num_q_heads * plan->max_splits;
         plan->part_o_bytes = align256(rows * head_dim * sizeof(float));
         plan->part_ml_bytes = align256(rows * 2 * sizeof(float));
     }
-    plan->workspace = plan->part_o_bytes + plan->part_ml_bytes + plan->seq_prefix_bytes;
+    plan->workspace = plan->part_o_bytes + plan->part_ml_bytes + plan->seq_prefix_bytes + plan->done_bytes;
     return PA_OK;
 }
 
@@ -2258,6 +2410,9 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
         p.seq_prefix = plan.seq_prefix_bytes
                            ? reinterpret_cast<int32_t*>(ws + plan.part_o_bytes + plan.part_ml_bytes)
                            : nullptr;
+        p.done_count = plan.done_bytes ? reinterpret_cast<int*>(ws + plan.part_o_bytes + plan.part_ml_bytes +
+                                                                plan.seq_prefix_bytes)
+                                       : nullptr;
     } else {
         p.part_o = nullptr;
         p.part_ml = nullptr;
@@ -2286,8 +2441,7 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
     const int table_bytes = p.contiguous ? 0 : (plan.partition / p.block_size) * 4;
     p.ring_offset = (int)((16 * stages + table_bytes + 127) & ~127);
     const size_t ring_bytes = (size_t)stages * stage_bytes;
-    const size_t merge_bytes = ((size_t)kConsumerWarps * G * (head_dim + 2) + (size_t)G * (kMaxFoldSplits + 1)) *
-                               sizeof(float);
+    const size_t merge_bytes = ((size_t)kConsumerWarps * G * (head_dim + 2) + (size_t)G * kCoefStride) * sizeof(float);
     if (merge_bytes > ring_bytes) return PA_ERR_UNSUPPORTED;
     const size_t smem = p.ring_offset + ring_bytes;
     if (smem > (size_t)kMaxDynamicSmem) return PA_ERR_UNSUPPORTED;
@@ -2301,16 +2455,23 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
         CUtensorMap tmk, tmv;
         if ((rc = encode_kv_map(&tmk, p.k, rows, head_dim, p.block_size))) return rc;
         if ((rc = encode_kv_map(&tmv, p.v, rows, head_dim, p.block_size))) return rc;
-        if (p.num_groups > 0 && plan.tc) {
-            // the prefix pass on the tensor cores: 128-token tiles, its own
-            // buffers and tensor memory
+        // the prefix pass on the tensor cores: 128-token tiles, its own
+        // buffers and tensor memory
+        p.prefix_last = p.num_groups > 0 && plan.prefix_last;
+        const auto prefix_tc = [&]() -> int {
             const size_t psmem = prefix_tc_smem_bytes(plan.prefix_partition / p.block_size);
             if (psmem > (size_t)kMaxDynamicSmem) return PA_ERR_UNSUPPORTED;
             const int64_t gy = (int64_t)p.num_kv_heads * plan.chunks;
             if (gy > 65535) return PA_ERR_UNSUPPORTED;
             const dim3 pg((unsigned)(plan.prefix_splits > 0 ? plan.prefix_splits : 1), (unsigned)gy,
                           (unsigned)p.num_groups);
-            if ((rc = launch_prefix_tc(p, tmk, tmv, pg, psmem, st))) return rc;
+            return launch_prefix_tc(p, tmk, tmv, pg, psmem, st);
+        };
+        if (p.prefix_last) {
+            // set-up kernel, pass 1, then the prefix pass (below)
+            if ((rc = launch_pdl(decode_prefix_setup_kernel, dim3(1), dim3(1024), 0, st, p))) return rc;
+        } else if (p.num_groups > 0 && plan.tc) {
+            if ((rc = prefix_tc())) return rc;
         } else if (p.num_groups > 0) {
             // the prefix pass: a deeper ring (few, long-lived CTAs), every
             // consumer warp reads every stage
@@ -2332,7 +2493,11 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
             if (rc) return rc;
         }
         p.ring_offset = (int)((16 * stages + table_bytes + 1023) & ~1023);
-        const size_t smem_mma = p.ring_offset + ring_bytes + 1024;
+        // shared-prefix calls with the prefix pass first: room for the
+        // prefix partial a row folds in
+        p.fold_prefetch = p.num_groups > 0 && !p.prefix_last;
+        const size_t pf_bytes = p.fold_prefetch ? ((size_t)G * (head_dim + 2) * sizeof(float) + 15) & ~(size_t)15 : 0;
+        const size_t smem_mma = p.ring_offset + ring_bytes + pf_bytes + 1024;
         if (smem_mma > (size_t)kMaxDynamicSmem) return PA_ERR_UNSUPPORTED;
         if (head_dim == 128)
             rc = G <= 8 ? launch_pass1_mma<128, 1>(p, tmk, tmv, grid, smem_mma, st)
@@ -2340,14 +2505,17 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
         else
             rc = G <= 8 ? launch_pass1_mma<64, 1>(p, tmk, tmv, grid, smem_mma, st)
                         : launch_pass1_mma<64, 2>(p, tmk, tmv, grid, smem_mma, st);
+        if (!rc && p.prefix_last) rc = prefix_tc();
     } else {
         rc = head_dim == 128 ? dispatch_group<float, 128>(G, p, grid, smem, st)
                              : dispatch_group<float, 64>(G, p, grid, smem, st);
     }
     if (rc) return rc;
     // with shared prefixes, rows whose suffix is one split are finished by
-    // pass 1; the merge pass is needed only when a suffix can be split
-    if (p.num_groups > 0 ? (plan.suffix_splits > 1 || plan.prefix_splits > kMaxFoldSplits) : plan.max_splits > 1) {
+    // pass 1 (or, in the prefix-last order, by the prefix pass); the merge
+    // pass is needed only when a suffix can be split
+    if (p.num_groups > 0 ? !plan.prefix_last && (plan.suffix_splits > 1 || plan.prefix_splits > kMaxFoldSplits)
+                         : plan.max_splits > 1) {
         const int64_t rows = (int64_t)batch * p.num_q_heads;
         // four warps per row, or all eight of a CTA when rows carry many splits
         // and there are too few rows to fill the GPU with four-warp groups

@@ -181,10 +181,15 @@ def test_shared_prefix_workspace_size(lib):
     # no prefix, one suffix split: only the per-sequence prefix lengths
     assert f(4, 8, 2, 128, 100, 16, 2, 2, 0, 128, ctypes.byref(sz)) == OK
     assert sz.value == 256
-    # a prefix: prefix splits + suffix splits per row, then the lengths
+    # a prefix: prefix splits + suffix splits per row, then the lengths and
+    # (head_dim 128, one prefix split and one own split: the prefix pass runs
+    # last) its exit counter
     assert f(4, 8, 2, 128, 100, 16, 2, 2, 64, 128, ctypes.byref(sz)) == OK
     rows = 4 * 8 * 2
-    assert sz.value == -(-rows * 128 * 4 // 256) * 256 + -(-rows * 2 * 4 // 256) * 256 + 256
+    assert sz.value == -(-rows * 128 * 4 // 256) * 256 + -(-rows * 2 * 4 // 256) * 256 + 256 + 256
+    # head_dim 64 keeps the prefix pass first: no counter
+    assert f(4, 8, 2, 64, 100, 16, 2, 2, 64, 128, ctypes.byref(sz)) == OK
+    assert sz.value == -(-rows * 64 * 4 // 256) * 256 + -(-rows * 2 * 4 // 256) * 256 + 256
     assert f(4, 8, 2, 128, 100, 16, 0, 2, 64, 128, ctypes.byref(sz)) == INVALID
     assert f(4, 8, 2, 128, 100, 16, 2, 2, 101, 128, ctypes.byref(sz)) == INVALID
 
