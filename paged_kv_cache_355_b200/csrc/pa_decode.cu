@@ -44,7 +44,13 @@
 //    never multiplied (stale shared memory may hold anything, NaN included).
 //  * Pass 1 and the merge are launched with programmatic stream
 //    serialisation and wait (griddepcontrol.wait) before touching global
-//    memory, so they can be scheduled while the previous kernel drains.
+//    memory, so they can be scheduled while the previous kernel drains.  In
+//    the shared-prefix call's prefix-last order a chain of such waits lets
+//    two kernels read the call's inputs earlier: a grid starts only after
+//    every CTA of the kernel before it has signalled, and each signals after
+//    its own wait, so pass 1 (after the set-up kernel) and the prefix pass
+//    (after pass 1) find the inputs final; each waits only for its
+//    predecessor's results (the prefix lengths; pass 1's partial rows).
 //
 // The contiguous-cache variant is the same kernel: only the producer's source
 // address differs (one bulk copy per 32-token stage instead of one per block).
@@ -116,6 +122,12 @@ struct DecodeParams {
     // shared-prefix calls: pass 1 has room after its ring for the one prefix
     // partial it folds into a row (G rows of D floats, then their (m, l))
     int fold_prefetch;
+    // bf16 paged pass 1: block-table entries of the window that CTA (split,
+    // kvh, b) loads at its start, before it knows the sequence's length and
+    // prefix length: entries split * partition / block_size onwards, enough
+    // for any prefix up to max_prefix plus one partition (0: load the slice
+    // once the length is known)
+    int table_window;
     // shared-prefix calls with one prefix split and one own split, head_dim
     // 128: a set-up kernel checks the groups and writes seq_prefix, pass 1
     // runs next and stores each own part's partial in slot 1, and the
@@ -220,6 +232,23 @@ __device__ __forceinline__ void store_out(const DecodeParams& p, int64_t idx, fl
         static_cast<float*>(p.out)[idx] = v;
 }
 
+// Output elements idx .. idx + 3 (idx a multiple of 4): one vector store when
+// the output buffer is aligned for it (the caller's buffer need not be).
+__device__ __forceinline__ void store_out4(const DecodeParams& p, int64_t idx, float4 v) {
+    const uintptr_t base = reinterpret_cast<uintptr_t>(p.out);
+    if (p.out_bf16 && (base & 7u) == 0)
+        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + idx) =
+            make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+    else if (!p.out_bf16 && (base & 15u) == 0)
+        *reinterpret_cast<float4*>(static_cast<float*>(p.out) + idx) = v;
+    else {
+        store_out(p, idx, v.x);
+        store_out(p, idx + 1, v.y);
+        store_out(p, idx + 2, v.z);
+        store_out(p, idx + 3, v.w);
+    }
+}
+
 // Prefix splits that pass 1 folds into a row itself (more are left to the
 // merge pass).
 constexpr int kMaxFoldSplits = 16;
@@ -289,30 +318,47 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeParams& p, con
         }
     }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+    // four consecutive elements of a row per thread step (D is a multiple of
+    // 4, rows start 16-byte aligned in every array)
+    for (int idx = 4 * threadIdx.x; idx < G * D; idx += 4 * blockDim.x) {
         const int h = idx / D;
         const int d = idx - h * D;
         const int64_t qrow = (int64_t)b * p.num_q_heads + (int64_t)kvh * G + h;
         const float* c = coef + h * kCoefStride;
-        float acc = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) acc = fmaf(sm_o[(w * G + h) * D + d], c[w], acc);
+        for (int w = 0; w < kConsumerWarps; ++w) {
+            const float4 o = *reinterpret_cast<const float4*>(sm_o + (w * G + h) * D + d);
+            const float cw = c[w];
+            acc.x = fmaf(o.x, cw, acc.x);
+            acc.y = fmaf(o.y, cw, acc.y);
+            acc.z = fmaf(o.z, cw, acc.z);
+            acc.w = fmaf(o.w, cw, acc.w);
+        }
         if (sp > 0) {
             const float* po = pf ? pf + h * D + d : p.part_o + qrow * p.max_splits * D + d;
             // four splits' loads in flight at a time
             for (int s0 = 0; s0 < sp; s0 += 4) {
-                float v[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) v[u] = s0 + u < sp ? po[(int64_t)(s0 + u) * D] : 0.f;
+                float4 v[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
-                    if (s0 + u < sp) acc = fmaf(c[kConsumerWarps + s0 + u], v[u], acc);
+                    v[u] = s0 + u < sp ? *reinterpret_cast<const float4*>(po + (int64_t)(s0 + u) * D)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (s0 + u < sp) {
+                        const float cs = c[kConsumerWarps + s0 + u];
+                        acc.x = fmaf(cs, v[u].x, acc.x);
+                        acc.y = fmaf(cs, v[u].y, acc.y);
+                        acc.z = fmaf(cs, v[u].z, acc.z);
+                        acc.w = fmaf(cs, v[u].w, acc.w);
+                    }
             }
         }
         if (final_row)
-            store_out(p, qrow * D + d, acc);
+            store_out4(p, qrow * D + d, acc);
         else
-            p.part_o[(qrow * p.max_splits + split) * D + d] = acc;
+            *reinterpret_cast<float4*>(p.part_o + (qrow * p.max_splits + split) * D + d) = acc;
     }
 }
 
@@ -681,7 +727,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + p.stages;
-    int32_t* tbl = reinterpret_cast<int32_t*>(empty + p.stages);
+    int32_t* const tbl_base = reinterpret_cast<int32_t*>(empty + p.stages);
     // the 128-byte swizzle pattern assumes 1024-byte aligned slabs: align the
     // ring at run time (the launch reserves 1 KB of slack for this)
     uint8_t* ring = smem + p.ring_offset + ((1024u - (smem_addr(smem) & 1023u)) & 1023u);
@@ -691,8 +737,15 @@ __global__ void __launch_bounds__(kDecodeThreads)
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
     }
-    griddep_wait();  // q, lengths, tables and the pool may come from the kernel before
-    griddep_launch_dependents();
+    // q, lengths, tables and the pool may come from the kernel before.  In the
+    // prefix-last order that kernel is the set-up kernel, which waited for the
+    // kernels before the call before this grid could start: only its own
+    // result (the prefix length) needs the wait, taken below, after the
+    // prologue's other loads are in flight.
+    if (!p.prefix_last) {
+        griddep_wait();
+        griddep_launch_dependents();
+    }
     const int split = blockIdx.x;
     const int kvh = blockIdx.y;
     const int b = schedule_sequence(p, ring);
@@ -700,8 +753,22 @@ __global__ void __launch_bounds__(kDecodeThreads)
     const int lane = threadIdx.x & 31;
     const int G = p.num_q_heads / p.num_kv_heads;
 
-    // the length and the prefix length, loaded together
+    // the length, the prefix length and the block-table window, loaded together
     const int len_raw = p.context_lens[b];
+    constexpr int TW = 4;  // window entries per thread in flight
+    const int win0 = (int)(((int64_t)split * p.partition) / p.block_size);
+    const int nwin = (p.contiguous || !p.table_window) ? 0 : max(0, min(p.table_window, p.max_blocks_per_seq - win0));
+    const int32_t* wrow = p.block_tables + (int64_t)b * p.max_blocks_per_seq + win0;
+    int32_t tw[TW];
+#pragma unroll
+    for (int u = 0; u < TW; ++u) {
+        const int i = threadIdx.x + u * kDecodeThreads;
+        tw[u] = i < nwin ? wrow[i] : 0;
+    }
+    if (p.prefix_last) {
+        griddep_wait();
+        griddep_launch_dependents();  // after the wait: the prefix pass relies on the set-up kernel's counter
+    }
     const int pre_raw = p.seq_prefix ? p.seq_prefix[b] : 0;
     const int L = clamp_len_value(p, len_raw, threadIdx.x == 0 && split == 0 && kvh == 0);
     // A length beyond max_context_len is clamped for the attention (and
@@ -733,7 +800,18 @@ __global__ void __launch_bounds__(kDecodeThreads)
         }
         fence_barrier_init();
     }
-    if (!p.contiguous) {
+    // the block ids of the split's tokens: from the window loaded above (the
+    // slice starts pre / block_size entries into it), or loaded now
+    int32_t* tbl = tbl_base;
+    if (nwin) {
+#pragma unroll
+        for (int u = 0; u < TW; ++u) {
+            const int i = threadIdx.x + u * kDecodeThreads;
+            if (i < nwin) tbl_base[i] = tw[u];
+        }
+        for (int i = threadIdx.x + TW * kDecodeThreads; i < nwin; i += kDecodeThreads) tbl_base[i] = wrow[i];
+        tbl = tbl_base + (tok_begin / p.block_size - win0);
+    } else if (!p.contiguous) {
         const int first_blk = tok_begin / p.block_size;
         const int nblk = (ntok + p.block_size - 1) / p.block_size;
         const int32_t* row = p.block_tables + (int64_t)b * p.max_blocks_per_seq + first_blk;
@@ -2059,11 +2137,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                         o.y = fmaf(c1, o1.y, o.y);
                         o.z = fmaf(c1, o1.z, o.z);
                         o.w = fmaf(c1, o1.w, o.w);
-                        if (p.out_bf16)
-                            *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + off + c) =
-                                make_uint2(pack_bf16x2(o.x, o.y), pack_bf16x2(o.z, o.w));
-                        else
-                            *reinterpret_cast<float4*>(static_cast<float*>(p.out) + off + c) = o;
+                        store_out4(p, off + c, o);
                     } else {
                         *reinterpret_cast<float4*>(p.part_o + off + c) = o;
                     }
@@ -2438,7 +2512,14 @@ int run_decode(DecodeParams p, int head_dim, int kv_dtype, int batch, void* work
     int stages = (kRingTargetBytes / stage_bytes) / kConsumerWarps * kConsumerWarps;
     stages = stages < kConsumerWarps ? kConsumerWarps : (stages > 4 * kConsumerWarps ? 4 * kConsumerWarps : stages);
     p.stages = stages;
-    const int table_bytes = p.contiguous ? 0 : (plan.partition / p.block_size) * 4;
+    // bf16 pass 1 loads its block-table window speculatively (one round trip
+    // fewer) while the window stays within twice a partition's blocks
+    const int part_blocks = plan.partition / p.block_size;
+    p.table_window = 0;
+    if (!p.contiguous && kv_dtype == PA_BF16 && (p.num_groups == 0 || p.max_prefix <= plan.partition))
+        p.table_window = min((p.num_groups > 0 ? p.max_prefix : 0) / p.block_size + part_blocks,
+                             max(p.max_blocks_per_seq, 1));
+    const int table_bytes = p.contiguous ? 0 : max(part_blocks, p.table_window) * 4;
     p.ring_offset = (int)((16 * stages + table_bytes + 127) & ~127);
     const size_t ring_bytes = (size_t)stages * stage_bytes;
     const size_t merge_bytes = ((size_t)kConsumerWarps * G * (head_dim + 2) + (size_t)G * kCoefStride) * sizeof(float);

@@ -25,14 +25,17 @@ def pa():
     return pa
 
 
-def run_gpu(pa, case, partition=0, out_dtype=torch.float32, k_pool=None, v_pool=None, block_tables=None):
-    """Paged decode of a case's current pools (no append)."""
+def run_gpu(pa, case, partition=0, out_dtype=torch.float32, k_pool=None, v_pool=None, block_tables=None,
+            out_offset=0):
+    """Paged decode of a case's current pools (no append); out_offset > 0
+    puts the output that many elements into its buffer (misaligned rows)."""
     q = case.q.cuda()
     kp = (case.k_pool if k_pool is None else k_pool).cuda()
     vp = (case.v_pool if v_pool is None else v_pool).cuda()
     bt = (case.block_tables if block_tables is None else block_tables).cuda()
     lens = case.lengths.cuda()
-    out = torch.full(tuple(q.shape), float("nan"), dtype=out_dtype, device="cuda")
+    buf = torch.full((q.numel() + out_offset,), float("nan"), dtype=out_dtype, device="cuda")
+    out = buf[out_offset:].view(tuple(q.shape))
     pa.pa_paged_attention_decode(q, kp, vp, bt, lens, case.max_len, case.scale, out, partition_size=partition)
     torch.cuda.synchronize()
     return out
@@ -364,6 +367,19 @@ def test_bad_block_id_is_flagged_not_dereferenced(pa):
     run_gpu(pa, case, block_tables=bt)
     assert pa.pa_read_error_flag() == 5
     run_gpu(pa, case)
+    assert pa.pa_read_error_flag() == 0
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("partition", [0, 32])
+def test_misaligned_output_is_bit_identical(pa, out_dtype, partition):
+    """An output buffer that starts one element past an alignment boundary
+    (rows no longer 16-byte aligned) gets the same values, element by
+    element, as an aligned one."""
+    case = custom_case([1, 17, 300, 64, 129], 8, 2, 128, 16, torch.bfloat16, seed=77)
+    a = run_gpu(pa, case, partition=partition, out_dtype=out_dtype)
+    b = run_gpu(pa, case, partition=partition, out_dtype=out_dtype, out_offset=1)
+    assert torch.equal(a, b)
     assert pa.pa_read_error_flag() == 0
 
 

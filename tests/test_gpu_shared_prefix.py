@@ -36,9 +36,10 @@ def _groups(bs):
 
 
 def run_shared(pa, case, starts, plens, partition=0, max_prefix=None, max_group=None, bt=None, kp=None, vp=None,
-               out_dtype=torch.float32):
+               out_dtype=torch.float32, out_offset=0):
     B, Hq, D = case.q.shape
-    out = torch.full((B, Hq, D), float("nan"), dtype=out_dtype, device="cuda")
+    buf = torch.full((B * Hq * D + out_offset,), float("nan"), dtype=out_dtype, device="cuda")
+    out = buf[out_offset:].view(B, Hq, D)
     gs = torch.tensor(starts, dtype=torch.int32, device="cuda")
     gl = torch.tensor(plens, dtype=torch.int32, device="cuda")
     mp = max(plens) if max_prefix is None else max_prefix
@@ -200,8 +201,13 @@ def test_block_manager_groups_drive_the_shared_prefix_call(pa):
 # ---- many groups (the GPU-filling case), head_dim 128 ---------------------
 # 16 copies of the five groups above with 2 kv heads: 80 groups x 2 kv heads x
 # the row chunks >= 160 prefix CTAs, so every group's prefix is one split (the
-# tensor-core pass's widest tiling) and pass 1 folds it into each row.
+# tensor-core pass's widest tiling).  With the automatic partition (512
+# tokens here) the own tokens take up to 3 splits: the prefix pass runs first,
+# pass 1 folds the prefix into one-split rows and the merge pass finishes the
+# others.  With a 4096-token partition the own tokens are one split: a set-up
+# kernel, pass 1, then the prefix pass, which finishes every shared row.
 MANY_COPIES = 16
+ORDERS = pytest.mark.parametrize("partition", [0, 4096], ids=["prefix_first", "prefix_last"])
 
 
 def _many_case(bs, G, seed, extra=(), extra_blocks=4):
@@ -209,22 +215,24 @@ def _many_case(bs, G, seed, extra=(), extra_blocks=4):
     return shared_prefix_case(groups, 2 * G, 2, 128, bs, torch.bfloat16, seed=seed, extra_blocks=extra_blocks)
 
 
+@ORDERS
 @pytest.mark.parametrize("bs", [8, 16, 32])
 @pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
-def test_many_groups_sweep(pa, bs, G):
+def test_many_groups_sweep(pa, bs, G, partition):
     """Own parts of 0..517 tokens, members whose context is the prefix, a
     group without a prefix; several row chunks per group for G >= 4."""
     case, starts, plens = _many_case(bs, G, seed=100 + bs + G)
-    out = run_shared(pa, case, starts, plens)
-    assert_matches_oracle(out, run_oracle(case), True, f"many groups bs{bs} G{G}")
+    out = run_shared(pa, case, starts, plens, partition=partition)
+    assert_matches_oracle(out, run_oracle(case), True, f"many groups bs{bs} G{G} partition {partition}")
     assert pa.pa_read_error_flag() == 0
 
 
-def test_many_groups_bf16_output_and_empty_sequences(pa):
+@ORDERS
+def test_many_groups_bf16_output_and_empty_sequences(pa, partition):
     """bf16 rows; groups without a prefix whose members are empty (rows of
     zeros) or mixed with a non-empty one."""
     case, starts, plens = _many_case(16, 4, seed=131, extra=[(0, [0, 0]), (0, [0, 9])])
-    out = run_shared(pa, case, starts, plens, out_dtype=torch.bfloat16)
+    out = run_shared(pa, case, starts, plens, partition=partition, out_dtype=torch.bfloat16)
     ref = run_oracle(case)
     assert_matches_oracle(out, ref, True, "many groups, bf16 out")
     empty = [b for b, L in enumerate(case.lengths.tolist()) if L == 0]
@@ -232,24 +240,38 @@ def test_many_groups_bf16_output_and_empty_sequences(pa):
     assert pa.pa_read_error_flag() == 0
 
 
-def test_many_groups_are_deterministic_and_placement_free(pa):
+@ORDERS
+def test_many_groups_are_deterministic_and_placement_free(pa, partition):
     case, starts, plens = _many_case(16, 4, seed=137, extra_blocks=40)
-    a = run_shared(pa, case, starts, plens)
-    assert torch.equal(a, run_shared(pa, case, starts, plens))
+    a = run_shared(pa, case, starts, plens, partition=partition)
+    assert torch.equal(a, run_shared(pa, case, starts, plens, partition=partition))
     perm = torch.randperm(case.num_blocks, generator=torch.Generator().manual_seed(138))
     kp, vp = torch.empty_like(case.k_pool), torch.empty_like(case.v_pool)
     kp[perm] = case.k_pool
     vp[perm] = case.v_pool
     bt = torch.where(case.block_tables >= 0, perm[case.block_tables.clamp(min=0).long()].to(torch.int32),
                      case.block_tables)
-    assert torch.equal(a, run_shared(pa, case, starts, plens, bt=bt, kp=kp, vp=vp))
+    assert torch.equal(a, run_shared(pa, case, starts, plens, partition=partition, bt=bt, kp=kp, vp=vp))
 
 
-def test_many_groups_never_read_outside_the_sequences(pa):
+@ORDERS
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_many_groups_misaligned_output_is_bit_identical(pa, partition, out_dtype):
+    """An output buffer one element past an alignment boundary gets the same
+    values as an aligned one."""
+    case, starts, plens = _many_case(16, 4, seed=141)
+    a = run_shared(pa, case, starts, plens, partition=partition, out_dtype=out_dtype)
+    b = run_shared(pa, case, starts, plens, partition=partition, out_dtype=out_dtype, out_offset=1)
+    assert torch.equal(a, b)
+    assert pa.pa_read_error_flag() == 0
+
+
+@ORDERS
+def test_many_groups_never_read_outside_the_sequences(pa, partition):
     """NaN in every pool slot no sequence uses (the rest of each partly used
     block included) and junk block ids past each table's used entries."""
     case, starts, plens = _many_case(16, 2, seed=139, extra_blocks=24)
-    clean = run_shared(pa, case, starts, plens)
+    clean = run_shared(pa, case, starts, plens, partition=partition)
     kp, vp = case.k_pool.clone(), case.v_pool.clone()
     used = torch.zeros(case.num_blocks, 16, dtype=torch.bool)
     for b, L in enumerate(case.lengths.tolist()):
@@ -259,12 +281,13 @@ def test_many_groups_never_read_outside_the_sequences(pa):
     vp.permute(0, 2, 1, 3)[~used] = float("nan")
     bt = case.block_tables.clone()
     bt[bt < 0] = case.num_blocks + 1000
-    assert torch.equal(clean, run_shared(pa, case, starts, plens, bt=bt, kp=kp, vp=vp))
+    assert torch.equal(clean, run_shared(pa, case, starts, plens, partition=partition, bt=bt, kp=kp, vp=vp))
     assert pa.pa_read_error_flag() == 0
 
 
+@ORDERS
 @pytest.mark.parametrize("fault", ["longer_than_a_member", "above_max_prefix", "not_whole_blocks"])
-def test_many_groups_broken_group_is_flagged_and_attended_without_sharing(pa, fault):
+def test_many_groups_broken_group_is_flagged_and_attended_without_sharing(pa, fault, partition):
     case, starts, plens = _many_case(16, 4, seed=149)
     starts, plens = list(starts), list(plens)
     kw = {}
@@ -275,12 +298,13 @@ def test_many_groups_broken_group_is_flagged_and_attended_without_sharing(pa, fa
     else:
         plens[5] = 56                     # not a multiple of 16
     pa.pa_read_error_flag()
-    out = run_shared(pa, case, starts, plens, **kw)
+    out = run_shared(pa, case, starts, plens, partition=partition, **kw)
     assert pa.pa_read_error_flag() == 5
-    assert_matches_oracle(out, run_oracle(case), True, f"many groups, {fault}")
+    assert_matches_oracle(out, run_oracle(case), True, f"many groups, {fault}, partition {partition}")
 
 
-def test_many_groups_flag_lengths_above_max_context(pa):
+@ORDERS
+def test_many_groups_flag_lengths_above_max_context(pa, partition):
     """A length above max_context_len is clamped to it and flagged, as the
     plain decode does."""
     case, starts, plens = _many_case(16, 4, seed=151)
@@ -295,7 +319,7 @@ def test_many_groups_flag_lengths_above_max_context(pa):
     mg = max(e - s for s, e in zip(starts[:-1], starts[1:]))
     pa.pa_paged_attention_decode_shared_prefix(case.q.cuda(), case.k_pool.cuda(), case.v_pool.cuda(),
                                                case.block_tables.cuda(), lens.cuda(), L, case.scale, out, gs, gl,
-                                               max(plens), mg)
+                                               max(plens), mg, partition_size=partition)
     torch.cuda.synchronize()
     assert pa.pa_read_error_flag() == 5
     assert_matches_oracle(out, run_oracle(case), True, "many groups, clamped length")
