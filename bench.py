@@ -33,7 +33,10 @@ e2e    = the same metric through the public API with the step's inputs in
 roofline = the decode call alone (pass 1 + merge; at least 100 timed replays,
          mean, median, p10 and p90 reported) against the measured HBM copy
          bandwidth, and against the read ceiling that pa_hbm_read_probe (a
-         plain bulk read stream of 2 GiB) reaches in the same run.
+         plain bulk read stream of 2 GiB) reaches in the same run.  Its
+         algorithmic bytes are the distinct K/V bytes the call must read:
+         every sequence's K/V, except that on the shared-prefix workload a
+         prompt block shared by a group counts once.
 other_workloads = (default run only) the decode calls of the GQA,
          long-context and shared-prefix workloads, timed the same way, with
          their paging overheads; the shared-prefix workload also by the
@@ -752,7 +755,8 @@ def run_ours(args):
 
     if rank != 0:
         return
-    achieved = kv_bytes / (ms_dec * 1e-3) / 1e9
+    # the decode call's algorithmic bytes: the distinct K/V slots it reads
+    achieved = unique_bytes / (ms_dec * 1e-3) / 1e9
     value = world * kv_bytes / (ms_step * 1e-3) / 1e9
     # the committed ncu record covers the workloads at their own batch only
     traffic = dram_traffic(args.workload) if args.batch in (None, WORKLOADS[args.workload].batch) else None
@@ -779,8 +783,9 @@ def run_ours(args):
                        "note": "distinct pool slots read; shared prompt blocks counted once"}
                       if unique_bytes != kv_bytes else None),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": traffic,
-                     "kernel": ("pa_paged_attention_decode_shared_prefix (prefix pass + suffix pass + merge)"
+                     "traffic": traffic, "algorithmic_bytes": unique_bytes,
+                     "kernel": ("pa_paged_attention_decode_shared_prefix (set-up kernel, pass 1 over each sample's "
+                                "own tokens, then the tensor-core prefix pass over each group's shared blocks)"
                                 if groups is not None else "pa_paged_attention_decode (pass 1 + split merge)"),
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)",
                      "read_ceiling_gbs": read_ceiling, "frac_of_read_ceiling": achieved / read_ceiling,
