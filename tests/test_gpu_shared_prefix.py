@@ -92,6 +92,23 @@ def test_no_prefix_is_bit_identical_to_plain_decode(pa):
         assert torch.equal(out, ref)
 
 
+def test_prefix_last_with_no_shared_tokens_is_bit_identical_to_plain_decode(pa):
+    """A prefix bound above 0 but every group's prefix 0, own tokens in one
+    split (4096-token partition), head_dim 128: the prefix pass is launched
+    after pass 1 and none of its CTAs has work (its last CTA still waits for
+    pass 1 before the grid ends).  Pass 1 alone writes every row: the plain
+    decode's bits, and the next call sees a finished result."""
+    groups = [(0, [70, 5]), (0, [300]), (0, [1, 2, 1000])]
+    case, starts, plens = shared_prefix_case(groups, 16, 4, 128, 16, torch.bfloat16, seed=19)
+    ref = torch.full((case.q.shape[0], 16, 128), float("nan"), device="cuda")
+    pa.pa_paged_attention_decode(case.q.cuda(), case.k_pool.cuda(), case.v_pool.cuda(), case.block_tables.cuda(),
+                                 case.lengths.cuda(), case.max_len, case.scale, ref, partition_size=4096)
+    for _ in range(3):
+        out = run_shared(pa, case, starts, plens, partition=4096, max_prefix=64)
+        assert torch.equal(out, ref)
+    assert pa.pa_read_error_flag() == 0
+
+
 def test_repeat_runs_and_physical_permutation_are_bit_identical(pa):
     case, starts, plens = shared_prefix_case(_groups(16), 32, 8, 128, 16, torch.bfloat16, seed=13, extra_blocks=30)
     a = run_shared(pa, case, starts, plens)
