@@ -321,6 +321,27 @@ def test_many_groups_broken_group_is_flagged_and_attended_without_sharing(pa, fa
 
 
 @ORDERS
+@pytest.mark.parametrize("bad", [-3, 1 << 20])
+def test_many_groups_bad_shared_block_id_is_flagged_not_dereferenced(pa, partition, bad):
+    """A shared prompt block id out of range (in every member's table, as
+    the sharing requires) is flagged and never loaded; the other groups'
+    rows are unaffected, and the next call with a clean table is clean."""
+    case, starts, plens = _many_case(16, 4, seed=171)
+    s, e = starts[3], starts[4]  # the first copy of the 640-token prefix group
+    bt = case.block_tables.clone()
+    bt[s:e, 5] = bad
+    pa.pa_read_error_flag()
+    out = run_shared(pa, case, starts, plens, partition=partition, bt=bt)
+    assert pa.pa_read_error_flag() == 5
+    ref = run_oracle(case)
+    others = [b for b in range(case.q.shape[0]) if not s <= b < e]
+    assert_matches_oracle(out[others], ref[others], True, f"bad shared block {bad}, partition {partition}")
+    clean = run_shared(pa, case, starts, plens, partition=partition)
+    assert pa.pa_read_error_flag() == 0
+    assert_matches_oracle(clean, ref, True, f"clean after a bad shared block, partition {partition}")
+
+
+@ORDERS
 def test_many_groups_flag_lengths_above_max_context(pa, partition):
     """A length above max_context_len is clamped to it and flagged, as the
     plain decode does."""
