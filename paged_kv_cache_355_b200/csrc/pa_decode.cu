@@ -1648,8 +1648,10 @@ __global__ void __launch_bounds__(32 * (1 + MT * PAR), 3)
 //    soon as its P.V is.  With one buffer each a CTA takes ~90 KB of shared
 //    memory, so two run on an SM: one's start-up and epilogue overlap the
 //    other's stream, and the GPU holds the whole grid of a typical call;
-//  * warp 1 owns the tensor memory and issues the MMAs from one thread:
-//    P_{j-1}.V_{j-1} once the softmax has written P_{j-1}, then S_j;
+//  * warp 1 owns the tensor memory (allocated first thing: the SM starts a
+//    second CTA of this kernel only once the first has given up its
+//    allocation permit) and issues the MMAs from one thread: P_{j-1}.V_{j-1}
+//    once the softmax has written P_{j-1}, then S_j;
 //  * warps 2..5 (one per TMEM lane quarter) run the softmax: thread t holds
 //    token t's scores for all 32 rows.  Every thread keeps the rows' running
 //    maxima; they move only when a score exceeds them by more than 2^8
@@ -1661,7 +1663,11 @@ __global__ void __launch_bounds__(32 * (1 + MT * PAR), 3)
 //    high and residual parts (M/N-major, 64-byte swizzle), for the next P.V;
 //  * at the end they stage O^T through shared memory and write each row's
 //    normalised partial (as float4 rows) and (m, l), as the mma.sync pass
-//    does.
+//    does; in the prefix-last order (the pass launched after pass 1) they
+//    instead wait for pass 1, fold its partial of each row's own tokens in
+//    by the log-sum-exp rescale, and write the final rows.
+// The group's check, the table slice and the query rows are fetched in one
+// round trip before any of them is used.
 // ---------------------------------------------------------------------------
 // Prefix-last order: the prefix pass's grid must not complete before pass 1
 // (kernels after the call wait for the prefix pass only).  CTAs with work wait
