@@ -6,7 +6,10 @@ Each csrc/*.cu (and host-only csrc/*.cpp) is compiled separately (in parallel) w
 ``-gencode arch=compute_100a,code=sm_100a -O3 -lineinfo`` into _build/, then
 linked into paged_kv_cache_355_b200/libpa.so with the CUDA runtime linked
 statically, so the library does not depend on which libcudart the host
-process has loaded.
+process has loaded.  The same objects, with pa_decode.cu compiled once more
+with -DPA_TIMELINE, make libpa_timeline.so (per-CTA timelines of the decode
+kernels, include/pa_timeline.h; read by ``python -m
+paged_kv_cache_355_b200.timeline``).
 """
 from __future__ import annotations
 
@@ -23,6 +26,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpa.so")
+TIMELINE_LIB = os.path.join(PKG, "libpa_timeline.so")
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",
@@ -55,11 +59,14 @@ def build(force: bool = False, verbose: bool = False) -> str:
     os.makedirs(BUILD_DIR, exist_ok=True)
     newest_header = max((_mtime(h) for h in _headers()), default=0.0)
     jobs, objs = [], []
-    for src in _sources():
-        obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
-        objs.append(obj)
+    timeline_obj = os.path.join(BUILD_DIR, "pa_decode_timeline.cu.o")
+    units = [(src, os.path.join(BUILD_DIR, os.path.basename(src) + ".o"), []) for src in _sources()]
+    units.append((os.path.join(CSRC, "pa_decode.cu"), timeline_obj, ["-DPA_TIMELINE"]))
+    for src, obj, extra in units:
+        if obj != timeline_obj:
+            objs.append(obj)
         if force or _mtime(obj) < max(_mtime(src), newest_header):
-            cmd = [nvcc, *ARCH_FLAGS, *CFLAGS, "-c", src, "-o", obj]
+            cmd = [nvcc, *ARCH_FLAGS, *CFLAGS, *extra, "-c", src, "-o", obj]
             if verbose:
                 cmd.insert(1, "-Xptxas=-v")
             jobs.append((src, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)))
@@ -72,10 +79,12 @@ def build(force: bool = False, verbose: bool = False) -> str:
             failed.append(os.path.basename(src))
     if failed:
         raise RuntimeError(f"nvcc failed for {', '.join(failed)}")
-    if force or jobs or _mtime(LIB) < max(_mtime(o) for o in objs):
-        tmp = LIB + f".tmp{os.getpid()}"
-        subprocess.run([nvcc, *ARCH_FLAGS, "-shared", "-cudart", "static", "-o", tmp, *objs], check=True)
-        os.replace(tmp, LIB)
+    timeline_objs = [timeline_obj if os.path.basename(o) == "pa_decode.cu.o" else o for o in objs]
+    for lib, lib_objs in ((LIB, objs), (TIMELINE_LIB, timeline_objs)):
+        if force or jobs or _mtime(lib) < max(_mtime(o) for o in lib_objs):
+            tmp = lib + f".tmp{os.getpid()}"
+            subprocess.run([nvcc, *ARCH_FLAGS, "-shared", "-cudart", "static", "-o", tmp, *lib_objs], check=True)
+            os.replace(tmp, lib)
     return LIB
 
 

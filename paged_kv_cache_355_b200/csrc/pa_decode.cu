@@ -68,6 +68,7 @@
 #include "pa_device.cuh"
 #include "pa_internal.h"
 #include "pa_tc.cuh"
+#include "pa_timeline.cuh"
 
 namespace pa {
 namespace {
@@ -734,6 +735,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
     __shared__ int s_abort;
 
     if (threadIdx.x == 0) {
+        PA_TL(2, 0);
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
     }
@@ -818,6 +820,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
         for (int i = threadIdx.x; i < nblk; i += blockDim.x) tbl[i] = row[i];
     }
     __syncthreads();
+    if (threadIdx.x == 0) PA_TL(2, 1);
 
     if (overflow && split == 0 && warp == 1) {
         const int pos = p.context_lens[b] - 1;
@@ -963,6 +966,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
                 s_abort = 1;
                 break;
             }
+            if (threadIdx.x == 32 && j == 0) PA_TL(2, 3);
             uint8_t* kstage = ring + (size_t)slot * 2 * STAGE_BYTES;
             uint8_t* vstage = kstage + STAGE_BYTES;
             const uint32_t kst = smem_addr(kstage);
@@ -1131,6 +1135,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
             }
     }
     __syncthreads();  // pipeline drained: the ring is free for the merge scratch
+    if (threadIdx.x == 0) PA_TL(2, 4);
     if (s_abort) return;
 
     float* sm_o = reinterpret_cast<float*>(ring);  // [warps][G][D]
@@ -1164,6 +1169,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
     __syncthreads();
     merge_warps_and_store(p, sm_o, sm_m, sm_l, sm_l + kConsumerWarps * G, G, D, b, kvh, prefix_splits + split,
                           num_splits_b, prefix_splits, !p.prefix_last, pf);
+    if (threadIdx.x == 0) PA_TL(2, 2);
 }
 
 // ---------------------------------------------------------------------------
@@ -1262,8 +1268,10 @@ __device__ PrefixGroup prefix_group_setup(const DecodeParams& p, int grp, bool r
 // prefix_group_describe and prefix_group_setup, so the prefix pass reaches
 // the same verdict on its own.  Also clears the prefix pass's exit counter.
 __global__ void __launch_bounds__(1024) decode_prefix_setup_kernel(const DecodeParams p) {
+    if (threadIdx.x == 0) PA_TL(0, 0);
     griddep_wait();  // lengths and descriptions may come from the kernel before
     griddep_launch_dependents();
+    if (threadIdx.x == 0) PA_TL(0, 1);
     for (int b = threadIdx.x; b < p.batch; b += blockDim.x) p.seq_prefix[b] = 0;
     if (threadIdx.x == 0) *p.done_count = 0;
     __syncthreads();
@@ -1284,6 +1292,7 @@ __global__ void __launch_bounds__(1024) decode_prefix_setup_kernel(const DecodeP
         }
         for (int m = start; m < start + n; ++m) p.seq_prefix[m] = P;
     }
+    if (threadIdx.x == 0) PA_TL(0, 2);
 }
 
 template <int D, int MT, int PAR>
@@ -1751,6 +1760,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     __shared__ int64_t row_own[N];  //           prefix-last order: element offset of pass 1's partial
 
     if (threadIdx.x == 0) {
+        PA_TL(1, 0);
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
     }
@@ -1828,6 +1838,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         }
         fence_proxy_async_smem();  // the tensor core reads Q through the async proxy
     }
+    if (threadIdx.x == 0) PA_TL(1, 1);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1854,6 +1865,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         fence_barrier_init();
     }
     __syncthreads();
+    if (threadIdx.x == 0) PA_TL(1, 3);
 
     if (warp == 0) {
         // ---------------- producer ----------------
@@ -1883,7 +1895,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                 if (lane == 0) ok = mbar_wait(&k_empty, (j - 1) & 1, p.err);
                 if (!(streamed = __shfl_sync(0xffffffffu, ok, 0))) break;
             }
-            if (lane == 0) mbar_arrive_expect_tx(&k_full, total);
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&k_full, total);
+                PA_TT(j, 5);
+            }
             __syncwarp();
             if (nbytes) {
                 tma_load_2d(sK + r * 128, &tmk, 0, y, &k_full, policy);
@@ -1908,7 +1923,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                 fence_proxy_async_smem();
                 __syncwarp();
             }
-            if (lane == 0) mbar_arrive_expect_tx(&v_full, total);
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&v_full, total);
+                PA_TT(j, 6);
+            }
             __syncwarp();
             if (nbytes) {
                 tma_load_2d(sV + r * 128, &tmv, 0, y, &v_full, policy);
@@ -1936,6 +1954,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                     if (!mbar_wait(&p_full, jp & 1, p.err)) break;
                     if (!mbar_wait(&v_full, jp & 1, p.err)) break;
                     tc_fence_after();
+                    PA_TT(jp, 3);
 #pragma unroll
                     for (int kk = 0; kk < kTcTokens / 16; ++kk) {
                         const uint64_t da = umma_desc(v_base + kk * 16 * 128, kTcSlab, 1024);
@@ -1953,6 +1972,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                     // loaded S_{j-2} before it signalled P_{j-2})
                     if (!mbar_wait(&k_full, j & 1, p.err)) break;
                     tc_fence_after();
+                    PA_TT(j, 4);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t off = (kk >> 2) * kTcSlab + (kk & 3) * 32;
@@ -1988,6 +2008,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                 break;
             }
             tc_fence_after();
+            if (threadIdx.x == 64) {
+                PA_TT(j, 0);
+                if (j == 0) PA_TL(1, 4);
+            }
             const uint32_t s_col = lane_base + N + (j & 1) * N;
             const bool tvalid = j * kTcTokens + tok < ntok;
             float x[N];
@@ -2056,6 +2080,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full);
+            if (threadIdx.x == 64) PA_TT(j, 1);
         }
         // the last P.V done: O^T is complete (and every MMA has read its
         // operands, so the K buffer is free for the epilogue)
@@ -2157,7 +2182,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcTmemCols));
     }
-    if (threadIdx.x == 0) prefix_last_exit(p);
+    if (threadIdx.x == 0) {
+        prefix_last_exit(p);
+        PA_TL(1, 2);
+    }
 }
 
 // Second pass: out = sum_s w_s o_s / sum_s w_s with w_s = l_s * 2^(m_s - max m),
@@ -2847,3 +2875,25 @@ extern "C" int pa_paged_attention_decode_contiguous(const void* q, const void* k
     return run_decode(p, head_dim, kv_dtype, batch, workspace, workspace_bytes, max_context_len, partition_size,
                       static_cast<cudaStream_t>(stream));
 }
+
+#ifdef PA_TIMELINE
+// The timeline build's readers (include/pa_timeline.h).
+extern "C" int pa_timeline_clear(void) {
+    void* a = nullptr;
+    void* t = nullptr;
+    if (cudaGetSymbolAddress(&a, pa::g_pa_tl) != cudaSuccess || cudaGetSymbolAddress(&t, pa::g_pa_tt) != cudaSuccess)
+        return PA_ERR_CUDA;
+    if (cudaMemset(a, 0, sizeof(pa::g_pa_tl)) != cudaSuccess || cudaMemset(t, 0, sizeof(pa::g_pa_tt)) != cudaSuccess)
+        return PA_ERR_CUDA;
+    return cudaDeviceSynchronize() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+extern "C" int pa_timeline_read(int which, void* dst, size_t bytes) {
+    if (!dst || (which != 0 && which != 1)) return PA_ERR_INVALID_ARG;
+    const size_t size = which == 0 ? sizeof(pa::g_pa_tl) : sizeof(pa::g_pa_tt);
+    if (bytes > size) return PA_ERR_INVALID_ARG;
+    const cudaError_t e = which == 0 ? cudaMemcpyFromSymbol(dst, pa::g_pa_tl, bytes)
+                                     : cudaMemcpyFromSymbol(dst, pa::g_pa_tt, bytes);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+#endif

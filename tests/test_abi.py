@@ -15,8 +15,8 @@ HEADER = os.path.join(ROOT, "include", "pa.h")
 OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
 
 
-def declared_entry_points():
-    text = open(HEADER).read()
+def declared_entry_points(header=HEADER):
+    text = open(header).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)))
 
@@ -34,6 +34,20 @@ def test_every_declared_symbol_is_exported(lib):
     assert len(names) >= 10
     missing = [n for n in names if not hasattr(lib, n)]
     assert not missing, missing
+
+
+def test_timeline_build_exports_the_same_abi_and_its_readers(lib):
+    """libpa_timeline.so (the decode kernels with per-CTA stamps) exports
+    everything include/pa.h declares plus include/pa_timeline.h's readers;
+    libpa.so has none of the readers."""
+    from paged_kv_cache_355_b200 import build
+
+    tl = ctypes.CDLL(build.TIMELINE_LIB)
+    readers = declared_entry_points(os.path.join(ROOT, "include", "pa_timeline.h"))
+    assert readers == ["pa_timeline_clear", "pa_timeline_read"]
+    missing = [n for n in declared_entry_points() + readers if not hasattr(tl, n)]
+    assert not missing, missing
+    assert not any(hasattr(lib, n) for n in readers)
 
 
 def test_binding_wraps_every_declared_symbol(lib):
