@@ -12,9 +12,12 @@ entry:
   * each kernel's CTA entries and exits (percentiles) and the end of the call;
   * resident CTAs of each kernel every 5 us;
   * pass 1's phases per CTA (prologue: entry to the block-table slice staged;
-    first stage: to the first K/V stage landed; stream; epilogue) and, on the
-    shared-prefix workload (sequences in index order), a least-squares fit of
-    a CTA's life against its own tokens;
+    first stage: to the first K/V stage landed; stream; epilogue), a
+    least-squares fit of a CTA's life against the tokens it reads (its
+    sequence found through the launch order: longest first, as the kernel
+    ranks it, for the plain call on batches up to 2048, index order
+    otherwise), and the CTAs' summed lives divided by the most that were
+    resident at once;
   * the prefix pass's per-tile chain: medians over CTAs of the time from a
     tile's scores to its P, from P to its P.V issue, from the V request to the
     P.V issue, from the K request to the S issue, and the tile period.
@@ -78,6 +81,9 @@ def _summary(ev: np.ndarray, tt: np.ndarray, own_tokens) -> dict:
         phases = {"prologue": p1[:, 1] - p1[:, 0], "first stage": p1[:, 3] - p1[:, 1], "stream": p1[:, 4] - p1[:, 3],
                   "epilogue": p1[:, 2] - p1[:, 4], "life": p1[:, 2] - p1[:, 0]}
         out["pass1_phases_us"] = {n: _pct(v) for n, v in phases.items()}
+        peak = max(out["resident"]["pass 1"]) if "pass 1" in out["resident"] else 0
+        if peak:
+            out["pass1_summed_life_per_slot_us"] = round(float(np.nansum(phases["life"])) / peak, 2)
         if own_tokens is not None:
             ids = np.nonzero(ev[2][:, 0] > 0)[0]
             tok = np.asarray(own_tokens(ids), float)
@@ -99,6 +105,18 @@ def _summary(ev: np.ndarray, tt: np.ndarray, own_tokens) -> dict:
                           "Kreq_to_S": med(a[:, 4] - a[:, 5]), "S_to_scores": med(a[:, 0] - a[:, 4])})
         out["prefix_tiles_us"] = chain
     return out
+
+
+def launch_order(lengths: np.ndarray, max_len: int, max_batch: int = 2048) -> np.ndarray:
+    """The sequence at each rank of plain decode's longest-first launch
+    order: 64 length buckets (longest first), ties by index; index order for
+    batches above max_batch, where the kernel does not rank."""
+    n = len(lengths)
+    if n > max_batch:
+        return np.arange(n)
+    L = np.clip(lengths.astype(np.int64), 0, max_len)
+    key = 63 - np.minimum(63, (L * 64) // (max_len + 1))
+    return np.array(sorted(range(n), key=lambda b: (key[b], b)))
 
 
 def run(workload: str = "cow", repeats: int = 3) -> list:
@@ -134,13 +152,21 @@ def run(workload: str = "cow", repeats: int = 3) -> list:
             prefix = np.zeros(w.batch, np.int64)
             for g, P in enumerate(groups[1]):
                 prefix[groups[0][g]:groups[0][g + 1]] = P
-            own = case.lengths.numpy() - prefix
-            # pass 1's grid is (splits, kv heads, batch) in index order here
-            own_tokens = lambda ids: own[ids // w.num_kv_heads]
+            order = np.arange(w.batch)  # the shared-prefix call keeps index order
         else:
             fn = lambda: b.pa_paged_attention_decode(case.q, case.k_pool, case.v_pool, bt, lens, case.max_len,
                                                      case.scale, out, partition_size=part)
-            own_tokens = None  # plain decode ranks its sequences: CTA ids are not sequence ids
+            prefix = np.zeros(w.batch, np.int64)
+            order = launch_order(case.lengths.numpy(), case.max_len)
+        # pass 1's grid is (splits, kv heads, rank): a CTA reads the tokens of
+        # its split of the sequence at its rank, after the sequence's prefix
+        L = np.clip(case.lengths.numpy().astype(np.int64), 0, case.max_len)
+        splits = -(-case.max_len // part)
+
+        def own_tokens(ids):
+            x, z = ids % splits, ids // (splits * w.num_kv_heads)
+            seq = order[z]
+            return np.clip(L[seq] - prefix[seq] - x * part, 0, part)
         fn()
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
@@ -187,8 +213,10 @@ def main() -> None:
             print(f"  pass 1 {name:12s} {v}")
         if "pass1_life_fit" in r:
             f = r["pass1_life_fit"]
-            print(f"  pass 1 life = {f['fixed_us']} us + {f['ns_per_token']} ns per own token "
+            print(f"  pass 1 life = {f['fixed_us']} us + {f['ns_per_token']} ns per token read "
                   f"(mean {f['mean_tokens']} tokens)")
+        if "pass1_summed_life_per_slot_us" in r:
+            print(f"  pass 1 summed CTA lives / peak resident CTAs: {r['pass1_summed_life_per_slot_us']} us")
         for c in r.get("prefix_tiles_us", []):
             print(f"  prefix tile {c['tile']}: period {c['period']}, scores->P {c['scores_to_P']}, "
                   f"P->P.V {c['P_to_PV']}, V req->P.V {c['Vreq_to_PV']}, K req->S {c['Kreq_to_S']}, "
