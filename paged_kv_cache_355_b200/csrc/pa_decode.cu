@@ -1234,11 +1234,11 @@ __device__ __forceinline__ void prefix_group_describe(const DecodeParams& p, int
         record_error(p.err, PA_ERR_BAD_BLOCK_ID);  // the groups do not cover the batch
 }
 
-// The verdict, once every member's length has been checked against the
+// The outcome, once every member's length has been checked against the
 // prefix (`bad` set by any member shorter than it): the reporter CTA flags a
 // bad description and writes each member's prefix length to seq_prefix.
 // Called by all threads, after a barrier that follows the checks.
-__device__ __forceinline__ PrefixGroup prefix_group_verdict(const DecodeParams& p, bool reporter, int start, int n,
+__device__ __forceinline__ PrefixGroup prefix_group_outcome(const DecodeParams& p, bool reporter, int start, int n,
                                                             int prefix, int bad) {
     const PrefixGroup g{start, n, bad ? 0 : prefix};
     if (reporter) {
@@ -1249,7 +1249,7 @@ __device__ __forceinline__ PrefixGroup prefix_group_verdict(const DecodeParams& 
 }
 
 // Check group grp's description; every CTA of the group reaches the same
-// verdict.  Called by all threads.
+// outcome.  Called by all threads.
 __device__ PrefixGroup prefix_group_setup(const DecodeParams& p, int grp, bool reporter) {
     __shared__ int s_start, s_n, s_prefix, s_bad;
     if (threadIdx.x == 0) prefix_group_describe(p, grp, reporter, s_start, s_n, s_prefix, s_bad);
@@ -1257,7 +1257,7 @@ __device__ PrefixGroup prefix_group_setup(const DecodeParams& p, int grp, bool r
     for (int m = threadIdx.x; m < s_n; m += blockDim.x)
         if (clamp_len(p, s_start + m, false) < s_prefix) s_bad = 1;  // a member shorter than the prefix
     __syncthreads();
-    return prefix_group_verdict(p, reporter, s_start, s_n, s_prefix, s_bad);
+    return prefix_group_outcome(p, reporter, s_start, s_n, s_prefix, s_bad);
 }
 
 // Prefix-last order: the groups' descriptions, checked once per call before
@@ -1266,7 +1266,7 @@ __device__ PrefixGroup prefix_group_setup(const DecodeParams& p, int grp, bool r
 // description that breaks the preconditions is flagged, and its sequences
 // keep prefix 0 (attended without sharing).  The rules are those of
 // prefix_group_describe and prefix_group_setup, so the prefix pass reaches
-// the same verdict on its own.  Also clears the prefix pass's exit counter.
+// the same outcome on its own.  Also clears the prefix pass's exit counter.
 __global__ void __launch_bounds__(1024) decode_prefix_setup_kernel(const DecodeParams p) {
     if (threadIdx.x == 0) PA_TL(0, 0);
     griddep_wait();  // lengths and descriptions may come from the kernel before
@@ -1843,7 +1843,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base;
-    const PrefixGroup grp = prefix_group_verdict(p, reporter, d_start, d_n, d_prefix, d_bad);
+    const PrefixGroup grp = prefix_group_outcome(p, reporter, d_start, d_n, d_prefix, d_bad);
     const int rows_total = grp.n * G;
     if (tok_begin >= grp.prefix || row0 >= rows_total) {  // uniform over the CTA
         if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcTmemCols));
