@@ -150,3 +150,44 @@ def test_prefill_rejects_fp32(pa):
         pa.pa_paged_attention_prefill(q, case.k_pool.cuda(), case.v_pool.cuda(), case.block_tables.cuda(),
                                       case.lengths.cuda(), torch.tensor([0, 8], dtype=torch.int32, device="cuda"), 8,
                                       case.scale, torch.empty(8, 4, 64, device="cuda"))
+
+
+# The chunked-prefill workload the benchmark times: batch 8, 32 q / 8 kv heads,
+# head_dim 128, bs 16, context 4096 of which the last 2048 tokens are new.
+FULL = (8, 32, 8, 128, 16, 4096, 2048)
+SAMPLED_TOKENS = [0, 1, 31, 32, 63, 64, 127, 128, 1023, 1024, 2015, 2046, 2047]
+
+
+@pytest.mark.parametrize("q_scale", [1.0, 4.0], ids=["as_benchmarked", "peaked"])
+def test_prefill_full_size_sampled_rows(pa, q_scale):
+    """The full chunked-prefill workload, built and launched as the benchmark
+    does (same seeds, bf16 output, the whole grid), with sampled query tokens
+    of every sequence (all 32 heads: tile edges, both ends of the chunk, plus
+    seeded random ones) against the oracle.  A query at position p attends
+    keys 0..p, so its row is decode attention over a sequence of length p + 1
+    with the same block table.  q scaled by 4 makes the softmax peaked, the
+    case where a bf16 P without its residual part leaves the bar."""
+    B, Hq, Hkv, D, bs, L, n = FULL
+    dev = torch.device("cuda", 0)
+    case = custom_case([L] * B, Hq, Hkv, D, bs, torch.bfloat16, seed=2001, device=dev)
+    qs = torch.arange(0, (B + 1) * n, n, dtype=torch.int32, device=dev)
+    g = torch.Generator(device=dev).manual_seed(2002)
+    q = (torch.randn(B * n, Hq, D, generator=g, device=dev) * q_scale).to(torch.bfloat16)
+    out = torch.full((B * n, Hq, D), float("nan"), dtype=torch.bfloat16, device=dev)
+    bt, lens = case.block_tables.to(dev), case.lengths.to(dev)
+    pa.pa_paged_attention_prefill(q, case.k_pool, case.v_pool, bt, lens, qs, n, case.scale, out)
+    torch.cuda.synchronize()
+    assert pa.pa_read_error_flag() == 0
+    rng = np.random.default_rng(2003)
+    rows = []  # (sequence, query token)
+    for b in range(B):
+        toks = sorted(set(SAMPLED_TOKENS) | set(int(x) for x in rng.integers(0, n, 3)))
+        rows += [(b, i) for i in toks]
+    sel = torch.tensor([b * n + i for b, i in rows], dtype=torch.long)
+    q_rows = q.cpu()[sel]
+    bt_rows = np_of(case.block_tables)[[b for b, _ in rows]]
+    len_rows = np.array([L - n + i + 1 for _, i in rows], np.int32)
+    ref = oracle.paged_decode(np_of(q_rows), np_of(case.k_pool), np_of(case.v_pool), bt_rows, len_rows,
+                              case.scale, bs)
+    got = out.cpu()[sel]
+    assert_matches_oracle(got, ref, True, f"full-size prefill, q x {q_scale}")
