@@ -31,7 +31,8 @@
 //    bits).  With two warpgroups per CTA one tile's softmax overlaps the
 //    other tile's MMAs.  At the end they read O, divide by the row sum and
 //    store the row.
-// The heaviest pairs of tiles (latest query tokens, most keys) start first.
+// The heaviest pairs of tiles (latest query tokens, most keys) start first,
+// across windows of four (sequence, kv head) groups.
 // Every wait is a bounded mbarrier wait; on expiry the CTA records
 // PA_ERR_TIMEOUT and winds down (tensor memory is always released).
 #include <cuda.h>
@@ -58,6 +59,11 @@ constexpr int kKeys = 64;     // keys per tile
 constexpr int kThreads = 96 + kTiles * 128;  // producer, two MMA issuers, one softmax warpgroup per query tile
 static_assert(kTiles == 2, "the softmax warpgroups select their tile's values between two");
 constexpr int kStages = 4;     // K/V ring depth
+// (sequence, kv head) groups per launch-order window: wide enough that the
+// grid's tail holds light pairs, narrow enough that the window's K/V stays
+// in L2 (chunked-prefill workload: 1 group 766-770, 4 groups 773-779, 8
+// groups 772, 64 groups 746 TFLOP/s)
+constexpr int kWindow = 4;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.f;  // lazy-rescale threshold of the running max (log2 units)
 // P.V with P as a bf16 high part plus a bf16 residual (two MMAs per key
@@ -85,6 +91,8 @@ struct PrefillParams {
     int block_size;
     int out_bf16;
     float scale_log2;
+    int pairs;   // pairs of query tiles per (sequence, kv head)
+    int groups;  // batch x kv heads
 };
 
 // ---- the kernel ------------------------------------------------------------
@@ -116,10 +124,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ uint32_t tmem_base;
     __shared__ int s_abort;
 
-    // heaviest pairs (latest query tokens, most keys) first
-    const int pair = gridDim.x - 1 - blockIdx.x;
-    const int kvh = blockIdx.y;
-    const int b = blockIdx.z;
+    // Launch order (the hardware dispatches CTAs by index): the (sequence,
+    // kv head) groups are taken kWindow at a time, and inside a window the
+    // pairs go heaviest first (latest query tokens, most keys) across its
+    // groups.  The grid's tail then holds light pairs, while the K/V that a
+    // window's pairs share stays within L2.
+    const int P = p.pairs;
+    const int wi = (int)(blockIdx.x / (unsigned)(kWindow * P));
+    const int r = (int)blockIdx.x - wi * kWindow * P;
+    const int g0 = wi * kWindow;
+    const int wn = min(kWindow, p.groups - g0);
+    const int pr = r / wn;
+    const int grp = g0 + (r - pr * wn);
+    const int pair = P - 1 - pr;
+    const int b = grp / p.num_kv_heads;
+    const int kvh = grp - b * p.num_kv_heads;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int G = p.num_q_heads / p.num_kv_heads;
@@ -520,7 +539,6 @@ extern "C" int pa_paged_attention_prefill(const void* q, const void* k_pool, con
         (G != 1 && G != 2 && G != 4 && G != 8 && G != 16))
         return PA_ERR_UNSUPPORTED;
     if (batch == 0 || num_tokens == 0 || max_query_len == 0) return PA_OK;
-    if (batch > 65535 || num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
     if (!q || !k_pool || !v_pool || !block_tables || !context_lens || !query_start || !out) return PA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out)) return PA_ERR_INVALID_ARG;
     const uint64_t pool_rows = (uint64_t)num_blocks * num_kv_heads * (uint64_t)block_size;
@@ -560,7 +578,11 @@ extern "C" int pa_paged_attention_prefill(const void* q, const void* k_pool, con
     p.out_bf16 = out_dtype == PA_BF16;
     p.scale_log2 = scale * kLog2e;
     const int q_tiles = (max_query_len + TQ - 1) / TQ;
-    dim3 grid((unsigned)((q_tiles + kTiles - 1) / kTiles), (unsigned)num_kv_heads, (unsigned)batch);
+    p.pairs = (q_tiles + kTiles - 1) / kTiles;
+    p.groups = batch * num_kv_heads;
+    const int64_t ctas = (int64_t)p.pairs * p.groups;
+    if (ctas > INT32_MAX) return PA_ERR_UNSUPPORTED;
+    dim3 grid((unsigned)ctas);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return head_dim == 128 ? launch_prefill<128>(p, tq, tk, tv, grid, st) : launch_prefill<64>(p, tq, tk, tv, grid, st);
 }
