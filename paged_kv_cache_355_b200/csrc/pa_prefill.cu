@@ -28,7 +28,8 @@
 //    rescales O in tensor memory only when the max has grown by more than
 //    2^8 (lazy rescale), and stores P as a bf16 high part plus a bf16
 //    residual (both multiplied by V, so the weights keep ~16 significant
-//    bits).  With two warpgroups per CTA one tile's softmax overlaps the
+//    bits), in two halves of 32 keys, each handed to the MMA thread as soon
+//    as it is written.  With two warpgroups per CTA one tile's softmax overlaps the
 //    other tile's MMAs.  At the end they read O, divide by the row sum and
 //    store the row.
 // The heaviest pairs of tiles (latest query tokens, most keys) start first,
@@ -59,6 +60,12 @@ constexpr int kKeys = 64;     // keys per tile
 constexpr int kThreads = 96 + kTiles * 128;  // producer, two MMA issuers, one softmax warpgroup per query tile
 static_assert(kTiles == 2, "the softmax warpgroups select their tile's values between two");
 constexpr int kStages = 4;     // K/V ring depth
+// Parts of a P tile handed to the MMA thread one by one (chunked-prefill
+// workload, results bit-identical: 1 part 781, 2 parts 790, 4 parts 771
+// TFLOP/s; with four the extra hand-offs cost more than the overlap gives).
+constexpr int kHandoffs = 2;
+constexpr int kPartKeys = kKeys / kHandoffs;    // keys per part (a multiple of the MMA's 16)
+static_assert(kHandoffs == 2 || kHandoffs == 4, "P hand-off parts of 32 or 16 keys");
 // (sequence, kv head) groups per launch-order window: wide enough that the
 // grid's tail holds light pairs, narrow enough that the window's K/V stays
 // in L2 (chunked-prefill workload: 1 group 766-770, 4 groups 773-779, 8
@@ -120,7 +127,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* sV = sK + kStages * KV_BYTES;       // [kStages][KV_BYTES]
 
     __shared__ uint64_t q_full, kv_full[kStages], kv_empty[kStages];
-    __shared__ uint64_t s_full[kTiles][2], p_full[kTiles][2], pv_done[kTiles][2];
+    // p_full[t][s][h]: part h (keys kPartKeys * h ..) of P in S buffer s of tile t
+    __shared__ uint64_t s_full[kTiles][2], p_full[kTiles][2][kHandoffs], pv_done[kTiles][2];
     __shared__ uint32_t tmem_base;
     __shared__ int s_abort;
 
@@ -178,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < kTiles; ++t)
             for (int s = 0; s < 2; ++s) {
                 mbar_init(&s_full[t][s], 1);
-                mbar_init(&p_full[t][s], 4);
+                for (int h = 0; h < kHandoffs; ++h) mbar_init(&p_full[t][s][h], 4);
                 mbar_init(&pv_done[t][s], 1);
             }
         fence_barrier_init();
@@ -281,18 +289,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (j >= 1) {
                     const int jp = j - 1;
-                    if (!(ok = mbar_wait(&p_full[t][jp & 1], (jp >> 1) & 1, p.err))) break;
-                    tc_fence_after();
                     const uint32_t v_base = smem_addr(sV + (jp % kStages) * KV_BYTES);
                     const uint32_t p_col = tmem + t * TILE_COLS + (jp & 1) * S_COLS;
+                    // each part of P's keys as soon as the softmax has written it
 #pragma unroll
-                    for (int kk = 0; kk < kKeys / 16; ++kk) {
-                        const uint64_t db = umma_desc(v_base + kk * 2048, KV_SLAB, 1024);
-                        umma_tmem_a(tmem + t * TILE_COLS + O_COL, p_col + kk * 8, db, IDESC_O,
-                                    (jp > 0 || kk > 0) ? 1u : 0u);
-                        if (kSplitP)
-                            umma_tmem_a(tmem + t * TILE_COLS + O_COL, p_col + S_COLS / 2 + kk * 8, db, IDESC_O, 1u);
+                    for (int h = 0; h < kHandoffs; ++h) {
+                        if (!(ok = mbar_wait(&p_full[t][jp & 1][h], (jp >> 1) & 1, p.err))) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = h * (kPartKeys / 16); kk < (h + 1) * (kPartKeys / 16); ++kk) {
+                            const uint64_t db = umma_desc(v_base + kk * 2048, KV_SLAB, 1024);
+                            umma_tmem_a(tmem + t * TILE_COLS + O_COL, p_col + kk * 8, db, IDESC_O,
+                                        (jp > 0 || kk > 0) ? 1u : 0u);
+                            if (kSplitP)
+                                umma_tmem_a(tmem + t * TILE_COLS + O_COL, p_col + S_COLS / 2 + kk * 8, db, IDESC_O,
+                                            1u);
+                        }
                     }
+                    if (!ok) break;
                     umma_commit(&pv_done[t][jp & 1]);
                     umma_commit(&kv_empty[jp % kStages]);
                 }
@@ -360,69 +374,79 @@ __global__ void __launch_bounds__(kThreads, 1)
                 alpha = m == -INFINITY ? 0.f : exp2f(m - mx);
                 m = mx;
             }
+            // P_j over S_j's columns: bf16 high parts of the 64 weights in the
+            // first 32 columns (two per column, lower key in the low half),
+            // bf16 residuals in the last 32.  It goes to the MMA thread in
+            // kHandoffs parts of kPartKeys keys (kPartKeys / 2 columns of each
+            // of the two): a part's P.V runs while the next part's
+            // exponentials are computed.
             float sum8[8];
 #pragma unroll
             for (int c = 0; c < 8; ++c) sum8[c] = 0.f;
-            if (m != -INFINITY) {
-                const float neg_m = -m;
-                const float mul = fold ? p.scale_log2 : 1.f;
+            const float neg_m = -m;
+            const float mul = fold ? p.scale_log2 : 1.f;
 #pragma unroll
-                for (int c = 0; c < kKeys; ++c) {
-                    sv[c] = ex2_approx(fmaf(sv[c], mul, neg_m));
+            for (int h = 0; h < kHandoffs; ++h) {
+#pragma unroll
+                for (int c = kPartKeys * h; c < kPartKeys * (h + 1); ++c) {
+                    sv[c] = m != -INFINITY ? ex2_approx(fmaf(sv[c], mul, neg_m)) : 0.f;
                     sum8[c & 7] += sv[c];
                 }
-            } else {
+                if (h == 0 && j > 0 && __any_sync(0xffffffffu, grow)) {
+                    // O holds P.V of tiles < j: wait for the last of them, then
+                    // rescale (before any of P_j is handed over)
+                    if (!(ok = mbar_wait(&pv_done[t][(j - 1) & 1], ((j - 1) >> 1) & 1, p.err))) break;
+                    tc_fence_after();
 #pragma unroll
-                for (int c = 0; c < kKeys; ++c) sv[c] = 0.f;
+                    for (int c0 = 0; c0 < D; c0 += 32) {
+                        float ov[32];
+                        tmem_ld32(lane_base + O_COL + c0, ov);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+                        tmem_st32(lane_base + O_COL + c0, ov);
+                    }
+                }
+                constexpr int PC = kPartKeys / 2;  // columns of one part
+                uint32_t hi[PC], lo[PC];
+#pragma unroll
+                for (int c = 0; c < PC; ++c) {
+                    const float a = sv[kPartKeys * h + 2 * c], bb = sv[kPartKeys * h + 2 * c + 1];
+                    hi[c] = pack_bf16x2(a, bb);
+                    if (kSplitP) lo[c] = pack_bf16x2(a - bf16_lo_to_f32(hi[c]), bb - bf16_hi_to_f32(hi[c]));
+                }
+                if constexpr (PC == 16) {
+                    tmem_st16u(lane_base + s * S_COLS + PC * h, hi);
+                    if (kSplitP) tmem_st16u(lane_base + s * S_COLS + S_COLS / 2 + PC * h, lo);
+                } else {
+                    tmem_st8u(lane_base + s * S_COLS + PC * h, hi);
+                    if (kSplitP) tmem_st8u(lane_base + s * S_COLS + S_COLS / 2 + PC * h, lo);
+                }
+                // keys past the sequence end carry weight 0, but 0 * NaN is NaN
+                // in the MMA: zero those V rows of the CTA's last tile (both
+                // warpgroups that use it do, each before it signals its first
+                // part of P)
+                if (h == 0 && j == nt_cta - 1 && n_kv < nt_cta * kKeys) {
+                    uint8_t* vs = sV + (j % kStages) * KV_BYTES;
+                    const int first = n_kv - j * kKeys;
+                    const int nch = (kKeys - first) * SLABS * 8;
+                    for (int c = row; c < nch; c += 128) {
+                        const int r = first + c / (SLABS * 8);
+                        const int rem = c % (SLABS * 8);
+                        *reinterpret_cast<uint4*>(vs + (rem >> 3) * KV_SLAB + r * 128 + (rem & 7) * 16) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                }
+                tmem_wait_st();
+                // each warp signals its 32 rows' part of P (and its share of
+                // the V zeroing) to the MMA thread once all its lanes are done
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[t][s][h]);
             }
+            if (!ok) break;
             l = l * alpha + (((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7])));
-            if (j > 0 && __any_sync(0xffffffffu, grow)) {
-                // O holds P.V of tiles < j: wait for the last of them, then rescale
-                if (!(ok = mbar_wait(&pv_done[t][(j - 1) & 1], ((j - 1) >> 1) & 1, p.err))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    float ov[32];
-                    tmem_ld32(lane_base + O_COL + c0, ov);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-                    tmem_st32(lane_base + O_COL + c0, ov);
-                }
-            }
-            // P_j over S_j's columns: bf16 high parts of the 64 weights in the
-            // first 32 columns (two per column, lower key in the low half),
-            // bf16 residuals in the last 32
-            uint32_t hi[kKeys / 2], lo[kKeys / 2];
-#pragma unroll
-            for (int c = 0; c < kKeys / 2; ++c) {
-                const float a = sv[2 * c], bb = sv[2 * c + 1];
-                hi[c] = pack_bf16x2(a, bb);
-                if (kSplitP) lo[c] = pack_bf16x2(a - bf16_lo_to_f32(hi[c]), bb - bf16_hi_to_f32(hi[c]));
-            }
-            tmem_st32u(lane_base + s * S_COLS, hi);
-            if (kSplitP) tmem_st32u(lane_base + s * S_COLS + S_COLS / 2, lo);
-            // keys past the sequence end carry weight 0, but 0 * NaN is NaN in
-            // the MMA: zero those V rows of the CTA's last tile (both
-            // warpgroups that use it do, each before it signals its P)
-            if (j == nt_cta - 1 && n_kv < nt_cta * kKeys) {
-                uint8_t* vs = sV + (j % kStages) * KV_BYTES;
-                const int first = n_kv - j * kKeys;
-                const int nch = (kKeys - first) * SLABS * 8;
-                for (int c = row; c < nch; c += 128) {
-                    const int r = first + c / (SLABS * 8);
-                    const int rem = c % (SLABS * 8);
-                    *reinterpret_cast<uint4*>(vs + (rem >> 3) * KV_SLAB + r * 128 + (rem & 7) * 16) =
-                        make_uint4(0u, 0u, 0u, 0u);
-                }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            }
-            tmem_wait_st();
-            // each warp signals its 32 P rows (and its share of the V zeroing)
-            // to the MMA thread once all its lanes are done
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[t][s]);
         }
         // epilogue: O / l for this row
         if (ok && ntt > 0 && (ok = mbar_wait(&pv_done[t][(ntt - 1) & 1], ((ntt - 1) >> 1) & 1, p.err))) {
