@@ -131,11 +131,12 @@ def code_sha256(path: str) -> str:
     return hashlib.sha256("\n".join(lines).encode()).hexdigest()
 
 
-def dram_traffic(workload: str):
-    """Per-launch DRAM bytes of the decode kernel from the committed ncu
-    summary, if it was taken on the current kernel code; else None."""
-    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
-    src = os.path.join(ROOT, "paged_kv_cache_355_b200", "csrc", "pa_decode.cu")
+def dram_traffic(workload: str, record: str = "decode_traffic.json", source: str = "pa_decode.cu"):
+    """Per-launch DRAM bytes of a kernel from a committed ncu summary
+    (profiles/<record>), if it was taken on the current code of its source
+    file (csrc/<source>); else None."""
+    path = os.path.join(ROOT, "profiles", record)
+    src = os.path.join(ROOT, "paged_kv_cache_355_b200", "csrc", source)
     try:
         rec = json.load(open(path))
         sha = code_sha256(src)
@@ -876,7 +877,8 @@ def run_prefill(args):
         "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "dtype": "bf16", "data": "synthetic", "config": {"workload": PREFILL_WORKLOAD},
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
-                     "traffic": None, "kernel": "prefill_tc_kernel (tcgen05)",
+                     "traffic": dram_traffic("prefill", "prefill_traffic.json", "pa_prefill.cu"),
+                     "kernel": "prefill_tc_kernel (tcgen05)",
                      "peak_source": "measured (MEASURED_PEAKS.json bf16_tflops, cuBLAS burst)" if peaks
                      else "fallback"},
         "note": "useful FLOPs only; the kernel multiplies P by V twice (bf16 high part and residual), "

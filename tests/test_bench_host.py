@@ -42,6 +42,14 @@ def test_traffic_record_matches_the_current_decode_code(bench):
     assert bench.dram_traffic("tiny") is None
 
 
+def test_traffic_record_matches_the_current_prefill_code(bench):
+    """The same for the prefill kernel's record."""
+    rec = json.load(open(os.path.join(ROOT, "profiles", "prefill_traffic.json")))
+    entry = rec["prefill"]
+    assert bench.dram_traffic("prefill", "prefill_traffic.json", "pa_prefill.cu") == entry["dram_bytes_per_launch"]
+    assert entry["dram_bytes_per_launch"] == entry["read_bytes"] + entry["write_bytes"]
+
+
 class _W:
     def __init__(self, bs, hkv, d):
         self.block_size, self.num_kv_heads, self.head_dim = bs, hkv, d
