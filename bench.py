@@ -831,6 +831,15 @@ PREFILL_WORKLOAD = ("chunked prefill: batch 8, 32 q / 8 kv heads, head_dim 128, 
                     "context 4096 of which the last 2048 tokens are the new chunk, blocks scattered")
 
 
+def prefill_useful_flops(lengths, news, num_q_heads: int, head_dim: int) -> float:
+    """Useful FLOPs of causal multi-query attention: the last n of a
+    sequence's L tokens are queries, query i (position L - n + i) sees
+    L - n + i + 1 keys, and each visible (query, key) pair costs 2 * D for
+    q.k and 2 * D for p.v in every query head."""
+    pairs = sum(n * (L - n) + n * (n + 1) // 2 for L, n in zip(lengths, news))
+    return 4.0 * head_dim * num_q_heads * pairs
+
+
 def run_prefill(args):
     """Causal multi-query paged attention on one GPU: useful FLOPs (4 * D per
     (query, visible key, query head)) / CUDA-event time."""
@@ -846,8 +855,7 @@ def run_prefill(args):
     q = torch.randn(B * n, Hq, D, generator=g, device=dev).to(torch.bfloat16)
     out = torch.empty(B * n, Hq, D, dtype=torch.bfloat16, device=dev)
     bt, lens = case.block_tables.to(dev), case.lengths.to(dev)
-    pairs = sum(n * (L - n) + n * (n + 1) // 2 for _ in range(B))  # visible (query, key) pairs per head
-    flops = 4.0 * D * Hq * pairs
+    flops = prefill_useful_flops([L] * B, [n] * B, Hq, D)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     clean = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     run = lambda: pa.pa_paged_attention_prefill(q, case.k_pool, case.v_pool, bt, lens, qs, n, case.scale, out)

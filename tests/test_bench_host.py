@@ -74,3 +74,18 @@ def test_unique_bytes_count_shared_slots_once(bench):
     # a partial block shared by both: only its filled slots count, once
     case = _Case([5, 9], [[2, -1], [2, -1]], bs=16)
     assert bench.unique_kv_bytes(case) == 9 * per_token
+
+
+def test_prefill_useful_flops_counts_the_visible_pairs(bench):
+    """The prefill metric's FLOP count against a brute-force count of the
+    (query, key) pairs the causal mask leaves visible."""
+    lengths, news = [1, 7, 64, 65, 300, 0], [1, 3, 64, 1, 130, 0]
+    pairs = 0
+    for L, n in zip(lengths, news):
+        for i in range(n):
+            pos = L - n + i
+            pairs += sum(1 for t in range(L) if t <= pos)
+    assert bench.prefill_useful_flops(lengths, news, 32, 128) == 4.0 * 128 * 32 * pairs
+    # the benchmark's workload: batch 8, context 4096, the last 2048 tokens new
+    assert bench.prefill_useful_flops([4096] * 8, [2048] * 8, 32, 128) == 4.0 * 128 * 32 * 8 * (
+        2048 * 2048 + 2048 * 2049 // 2)
