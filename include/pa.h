@@ -101,7 +101,7 @@ int pa_selftest_wait_timeout(uint32_t limit_us, void* stream);
 /*
  * pa_hbm_read_probe -- read `bytes` of device memory at `buffer` as one
  * stream and discard them: the HBM read ceiling against which paged decode
- * attention, itself a read stream of K/V bytes, is judged.  No counterpart in
+ * attention, itself a read stream of K/V bytes, is measured.  No counterpart in
  * the pages: a measurement aid.  Each CTA (2 per SM) moves a grid-strided
  * series of 8 KB chunks of the buffer into a 6-stage shared-memory ring with
  * bulk TMA copies and never looks at them; nothing is written to global

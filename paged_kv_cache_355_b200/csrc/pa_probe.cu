@@ -1,6 +1,6 @@
 // pa_probe.cu -- HBM streaming-read probe: the read bandwidth a plain bulk
 // read stream reaches on this device, the ceiling against which the decode
-// kernel's K/V read rate is judged.
+// kernel's K/V read rate is measured.
 //
 // The decode pass reads every K/V byte once and writes almost nothing, so its
 // natural roofline is a read-only stream, which runs faster than the
