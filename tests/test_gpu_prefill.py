@@ -152,6 +152,23 @@ def test_prefill_rejects_fp32(pa):
                                       case.scale, torch.empty(8, 4, 64, device="cuda"))
 
 
+@pytest.mark.parametrize("G", [4, 16])
+def test_prefill_many_items_per_cta(pa, G):
+    """Far more work items (pairs of query tiles per sequence and kv head)
+    than SMs, of mixed shapes: chunks of random length (zero, odd tile counts,
+    whole sequences), so that every CTA of the kernel takes many items,
+    among them empty ones and ones where the second tile has no rows."""
+    rng = np.random.default_rng(41 + G)
+    B, Hkv = 48, 8 if G == 4 else 2
+    lengths = [int(x) for x in rng.integers(1, 400, B)]
+    news = [int(rng.integers(0, L + 1)) if i % 5 else L for i, L in enumerate(lengths)]
+    news[3] = 0
+    case = custom_case(lengths, Hkv * G, Hkv, 128, 16, torch.bfloat16, seed=43 + G)
+    out, ref = _run(pa, case, news)
+    assert_matches_oracle(out, ref, True, f"many items G{G}")
+    assert pa.pa_read_error_flag() == 0
+
+
 # The chunked-prefill workload the benchmark times: batch 8, 32 q / 8 kv heads,
 # head_dim 128, bs 16, context 4096 of which the last 2048 tokens are new.
 FULL = (8, 32, 8, 128, 16, 4096, 2048)
