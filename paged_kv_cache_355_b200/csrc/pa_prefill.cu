@@ -110,7 +110,8 @@ struct PrefillParams {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmq,
-                      const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
+                      const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                      const __grid_constant__ CUtensorMap tmo) {
     constexpr int SLABS = D / 64;
     constexpr int Q_BYTES = SLABS * kRows * 128;  // 128 rows x D
     constexpr int KV_SLAB = kKeys * 128;          // 64 rows x 64 elements
@@ -448,10 +449,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             l = l * alpha + (((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7])));
         }
-        // epilogue: O / l for this row
+        // epilogue: O / l for this row.  A whole tile with bf16 output is
+        // staged in the tile's Q buffer (its S MMAs are done), laid out as a
+        // Q tile is loaded (row r, 16-byte chunk c of a 64-element slab at
+        // chunk c ^ (r & 7)), and written by tiled TMA stores through the
+        // output map; other tiles store their rows directly.
         if (ok && ntt > 0 && (ok = mbar_wait(&pv_done[t][(ntt - 1) & 1], ((ntt - 1) >> 1) & 1, p.err))) {
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
+            if (p.out_bf16 && (t ? nq[1] : nq[0]) == TQ) {
+                uint8_t* so = sQ + t * Q_BYTES;
+#pragma unroll
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    float ov[32];
+                    tmem_ld32(lane_base + O_COL + c0, ov);
+                    tmem_wait_ld();
+                    uint8_t* slab_row = so + (c0 >> 6) * (kRows * 128) + row * 128;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const int c = ((c0 & 63) >> 3) + q4;
+                        const float* v = ov + 8 * q4;
+                        *reinterpret_cast<uint4*>(slab_row + ((c ^ (row & 7)) << 4)) =
+                            make_uint4(pack_bf16x2(v[0] * inv, v[1] * inv), pack_bf16x2(v[2] * inv, v[3] * inv),
+                                       pack_bf16x2(v[4] * inv, v[5] * inv), pack_bf16x2(v[6] * inv, v[7] * inv));
+                    }
+                }
+                fence_proxy_async_smem();  // the TMA store reads the rows through the async proxy
+                asm volatile("bar.sync %0, 128;" ::"r"(1 + t) : "memory");  // the warpgroup's 128 rows
+                if (quarter == 0 && lane == 0) {
+#pragma unroll
+                    for (int sl = 0; sl < SLABS; ++sl)
+                        tma_store_3d(&tmo, sl * 64, kvh * G, q0 + my_t0, so + sl * (kRows * 128));
+                    bulk_commit_group();
+                    bulk_wait_group_read0();
+                }
+            } else {
             const int64_t orow =
                 ((int64_t)(q0 + my_t0 + tq) * p.num_q_heads + (int64_t)kvh * G + (row % G)) * D;
 #pragma unroll
@@ -475,6 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             o[i / 4] = make_float4(ov[i] * inv, ov[i + 1] * inv, ov[i + 2] * inv, ov[i + 3] * inv);
                     }
                 }
+            }
             }
         }
         if (!ok) s_abort = 1;
@@ -525,7 +558,7 @@ size_t prefill_smem_bytes() {
 
 template <int D>
 int launch_prefill(const PrefillParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                   dim3 grid, cudaStream_t st) {
+                   const CUtensorMap& to, dim3 grid, cudaStream_t st) {
     static std::atomic<unsigned long long> configured{0};
     const size_t smem = prefill_smem_bytes<D>();
     int dev = 0;
@@ -537,7 +570,7 @@ int launch_prefill(const PrefillParams& p, const CUtensorMap& tq, const CUtensor
             return PA_ERR_CUDA;
         configured.fetch_or(bit);
     }
-    prefill_tc_kernel<D><<<grid, kThreads, smem, st>>>(p, tq, tk, tv);
+    prefill_tc_kernel<D><<<grid, kThreads, smem, st>>>(p, tq, tk, tv, to);
     return launch_status();
 }
 
@@ -570,13 +603,16 @@ extern "C" int pa_paged_attention_prefill(const void* q, const void* k_pool, con
     int* err = error_word_ptr();
     if (!err) return PA_ERR_CUDA;
 
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     const int TQ = kRows / G;
     {
+        // q, and bf16 out (the same [num_tokens][Hq][D] geometry) for the
+        // epilogue's stores of whole tiles
         cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_q_heads, (cuuint64_t)num_tokens};
         cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2, (cuuint64_t)num_q_heads * head_dim * 2};
         cuuint32_t box[3] = {64u, (cuuint32_t)G, (cuuint32_t)TQ};
         int rc = encode(&tq, q, 3, dims, strides, box);
+        if (!rc) rc = out_dtype == PA_BF16 ? encode(&to, out, 3, dims, strides, box) : (to = tq, PA_OK);
         if (rc) return rc;
     }
     {
@@ -608,5 +644,6 @@ extern "C" int pa_paged_attention_prefill(const void* q, const void* k_pool, con
     if (ctas > INT32_MAX) return PA_ERR_UNSUPPORTED;
     dim3 grid((unsigned)ctas);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return head_dim == 128 ? launch_prefill<128>(p, tq, tk, tv, grid, st) : launch_prefill<64>(p, tq, tk, tv, grid, st);
+    return head_dim == 128 ? launch_prefill<128>(p, tq, tk, tv, to, grid, st)
+                           : launch_prefill<64>(p, tq, tk, tv, to, grid, st);
 }
