@@ -29,9 +29,10 @@
 //    2^8 (lazy rescale), and stores P as a bf16 high part plus a bf16
 //    residual (both multiplied by V, so the weights keep ~16 significant
 //    bits), in two halves of 32 keys, each handed to the MMA thread as soon
-//    as it is written.  With two warpgroups per CTA one tile's softmax overlaps the
-//    other tile's MMAs.  At the end they read O, divide by the row sum and
-//    store the row.
+//    as it is written.  With two warpgroups per CTA one tile's softmax
+//    overlaps the other tile's MMAs.  At the end they read O and divide by
+//    the row sum; a whole tile with bf16 output goes out through its Q
+//    buffer by tiled TMA stores, other rows are stored directly.
 // The heaviest pairs of tiles (latest query tokens, most keys) start first,
 // across windows of four (sequence, kv head) groups.
 // Every wait is a bounded mbarrier wait; on expiry the CTA records
