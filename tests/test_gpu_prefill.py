@@ -61,6 +61,23 @@ def test_prefill_long_chunk_and_bf16_out(pa):
     assert_matches_oracle(out, ref, True, "prefill long")
 
 
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
+def test_prefill_bf16_out_every_shape(pa, D, G):
+    """bf16 output, whose whole query tiles leave through shared memory by
+    tiled TMA stores (box: 64 dims x G heads x 128 / G tokens) while partial
+    tiles store rows directly: chunks of whole tiles, whole tiles plus a
+    ragged tail, and a sequence's first tokens, for every head_dim and group
+    size."""
+    TQ = 128 // G
+    lengths = [4 * TQ + 37, 6 * TQ, 2 * TQ + 1, 300]
+    news = [4 * TQ, 6 * TQ, 2 * TQ + 1, 5]
+    case = custom_case(lengths, 2 * G, 2, D, 16, torch.bfloat16, seed=70 + D + G)
+    out, ref = _run(pa, case, news, out_dtype=torch.bfloat16)
+    assert_matches_oracle(out, ref, True, f"prefill bf16 out D{D} G{G}")
+    assert pa.pa_read_error_flag() == 0
+
+
 def test_prefill_single_token_equals_decode(pa):
     case = custom_case([5, 77, 300, 1], 16, 4, 128, 16, torch.bfloat16, seed=6)
     out, ref = _run(pa, case, [1, 1, 1, 1])
