@@ -6,10 +6,10 @@ Each csrc/*.cu (and host-only csrc/*.cpp) is compiled separately (in parallel) w
 ``-gencode arch=compute_100a,code=sm_100a -O3 -lineinfo`` into _build/, then
 linked into paged_kv_cache_355_b200/libpa.so with the CUDA runtime linked
 statically, so the library does not depend on which libcudart the host
-process has loaded.  The same objects, with pa_decode.cu compiled once more
-with -DPA_TIMELINE, make libpa_timeline.so (per-CTA timelines of the decode
-kernels, include/pa_timeline.h; read by ``python -m
-paged_kv_cache_355_b200.timeline``).
+process has loaded.  The same objects, with pa_decode.cu and pa_prefill.cu
+compiled once more with -DPA_TIMELINE, make libpa_timeline.so (per-CTA
+timelines of the decode and prefill kernels, include/pa_timeline.h; read by
+``python -m paged_kv_cache_355_b200.timeline``).
 """
 from __future__ import annotations
 
@@ -59,11 +59,13 @@ def build(force: bool = False, verbose: bool = False) -> str:
     os.makedirs(BUILD_DIR, exist_ok=True)
     newest_header = max((_mtime(h) for h in _headers()), default=0.0)
     jobs, objs = [], []
-    timeline_obj = os.path.join(BUILD_DIR, "pa_decode_timeline.cu.o")
+    # the timeline build's objects, replacing these of libpa.so
+    timeline_objs_of = {name: os.path.join(BUILD_DIR, name.replace(".cu", "_timeline.cu") + ".o")
+                        for name in ("pa_decode.cu", "pa_prefill.cu")}
     units = [(src, os.path.join(BUILD_DIR, os.path.basename(src) + ".o"), []) for src in _sources()]
-    units.append((os.path.join(CSRC, "pa_decode.cu"), timeline_obj, ["-DPA_TIMELINE"]))
+    units += [(os.path.join(CSRC, name), obj, ["-DPA_TIMELINE"]) for name, obj in timeline_objs_of.items()]
     for src, obj, extra in units:
-        if obj != timeline_obj:
+        if not extra:
             objs.append(obj)
         if force or _mtime(obj) < max(_mtime(src), newest_header):
             cmd = [nvcc, *ARCH_FLAGS, *CFLAGS, *extra, "-c", src, "-o", obj]
@@ -79,7 +81,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
             failed.append(os.path.basename(src))
     if failed:
         raise RuntimeError(f"nvcc failed for {', '.join(failed)}")
-    timeline_objs = [timeline_obj if os.path.basename(o) == "pa_decode.cu.o" else o for o in objs]
+    timeline_objs = [timeline_objs_of.get(os.path.basename(o)[:-2], o) for o in objs]
     for lib, lib_objs in ((LIB, objs), (TIMELINE_LIB, timeline_objs)):
         if force or jobs or _mtime(lib) < max(_mtime(o) for o in lib_objs):
             tmp = lib + f".tmp{os.getpid()}"

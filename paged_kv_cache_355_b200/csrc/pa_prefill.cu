@@ -52,6 +52,27 @@
 #include "pa_internal.h"
 #include "pa_tc.cuh"
 
+// Per-CTA timeline stamps, compiled in only for libpa_timeline.so (the
+// switch PA_TIMELINE; events listed in include/pa_timeline.h).
+#ifdef PA_TIMELINE
+namespace pa {
+constexpr int kPfTlCtas = 65536;
+constexpr int kPfTlSlots = 8;
+__device__ unsigned long long g_pa_prefill_tl[(size_t)kPfTlCtas * kPfTlSlots];
+__device__ __forceinline__ void prefill_stamp(int slot) {
+    if (blockIdx.x >= (unsigned)kPfTlCtas) return;
+    unsigned smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    unsigned long long* row = g_pa_prefill_tl + (size_t)blockIdx.x * kPfTlSlots;
+    row[slot] = global_timer_ns();
+    row[kPfTlSlots - 1] = smid;
+}
+}  // namespace pa
+#define PF_TL(slot) ::pa::prefill_stamp(slot)
+#else
+#define PF_TL(slot) ((void)0)
+#endif
+
 namespace pa {
 namespace {
 
@@ -162,6 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (threadIdx.x == 0 && pair == 0 && kvh == 0) record_error(p.err, PA_ERR_BAD_BLOCK_ID);
         return;
     }
+    if (threadIdx.x == 0) PF_TL(0);
     // per tile: first query token, tokens, position of the first one, key tiles
     int t0[kTiles], nq[kTiles], pos_first[kTiles], nt[kTiles];
     int n_kv = 0, nt_cta = 0;
@@ -202,6 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base;
+    if (threadIdx.x == 0) PF_TL(1);
 
     if (warp == 0) {
         // ---------------- producer ----------------
@@ -288,6 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         umma(d_s, da, db, IDESC_S, kk > 0 ? 1u : 0u);
                     }
                     umma_commit(&s_full[t][j & 1]);
+                    if (t == 0 && j == 0) PF_TL(2);
                 }
                 if (j >= 1) {
                     const int jp = j - 1;
@@ -310,6 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (!ok) break;
                     umma_commit(&pv_done[t][jp & 1]);
+                    if (jp == ntt - 1) PF_TL(3 + t);
                     umma_commit(&kv_empty[jp % kStages]);
                 }
             }
@@ -515,6 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc_fence_before();
     __syncthreads();
+    if (threadIdx.x == 0) PF_TL(5);
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTiles * TILE_COLS));
@@ -648,3 +674,18 @@ extern "C" int pa_paged_attention_prefill(const void* q, const void* k_pool, con
     return head_dim == 128 ? launch_prefill<128>(p, tq, tk, tv, to, grid, st)
                            : launch_prefill<64>(p, tq, tk, tv, to, grid, st);
 }
+
+#ifdef PA_TIMELINE
+extern "C" int pa_timeline_clear_prefill(void) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, pa::g_pa_prefill_tl) != cudaSuccess ||
+        cudaMemset(a, 0, sizeof(pa::g_pa_prefill_tl)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
+        return PA_ERR_CUDA;
+    return PA_OK;
+}
+
+extern "C" int pa_timeline_read_prefill(void* dst, size_t bytes) {
+    if (!dst || bytes > sizeof(pa::g_pa_prefill_tl)) return PA_ERR_INVALID_ARG;
+    return cudaMemcpyFromSymbol(dst, pa::g_pa_prefill_tl, bytes) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+#endif

@@ -1,8 +1,16 @@
-"""Per-CTA timelines of one decode-attention call, from libpa_timeline.so
-(libpa with globaltimer stamps compiled into the decode kernels; the events
-are listed in include/pa_timeline.h).
+"""Per-CTA timelines of one decode-attention or prefill call, from
+libpa_timeline.so (libpa with globaltimer stamps compiled into the decode and
+prefill kernels; the events are listed in include/pa_timeline.h).
 
     python -m paged_kv_cache_355_b200.timeline [--workload cow] [--repeats 3] [--json out.json]
+
+With --workload prefill the call is pa_paged_attention_prefill on the
+chunked-prefill workload (batch 8, 32 q / 8 kv heads, head_dim 128, bs 16,
+context 4096 of which the last 2048 tokens are new), launched directly after
+an L2 flush; printed per repeat: the CTAs' lives, entry to the first S MMA,
+last P.V to exit, exit to the next CTA's entry on the same SM, the CTAs per
+SM, the share of SM time between each CTA's first S and last P.V, and when
+each SM finished.
 
 The workload's decode call (the shared-prefix call for the shared-prefix
 workload, the plain call otherwise) is captured as a CUDA graph and replayed
@@ -35,6 +43,10 @@ import numpy as np
 KERNELS = ("set-up kernel", "prefix pass", "pass 1")
 TL_CTAS, TL_SLOTS = 65536, 16
 TT_CTAS, TT_TILES, TT_EVENTS = 512, 16, 8
+PF_CTAS, PF_SLOTS = 65536, 8
+# the chunked-prefill workload: batch, q heads, kv heads, head_dim, block
+# size, context, new tokens (seeds 2001 for the cache, 2002 for q)
+PREFILL_SHAPE = (8, 32, 8, 128, 16, 4096, 2048)
 
 
 def _load(path: str):
@@ -47,6 +59,9 @@ def _load(path: str):
     lib.pa_timeline_clear.argtypes, lib.pa_timeline_clear.restype = [], ctypes.c_int
     lib.pa_timeline_read.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t]
     lib.pa_timeline_read.restype = ctypes.c_int
+    lib.pa_timeline_clear_prefill.argtypes, lib.pa_timeline_clear_prefill.restype = [], ctypes.c_int
+    lib.pa_timeline_read_prefill.argtypes = [ctypes.c_void_p, ctypes.c_size_t]
+    lib.pa_timeline_read_prefill.restype = ctypes.c_int
     return lib
 
 
@@ -105,6 +120,81 @@ def _summary(ev: np.ndarray, tt: np.ndarray, own_tokens) -> dict:
                           "Kreq_to_S": med(a[:, 4] - a[:, 5]), "S_to_scores": med(a[:, 0] - a[:, 4])})
         out["prefix_tiles_us"] = chain
     return out
+
+
+def _prefill_summary(ev: np.ndarray) -> dict:
+    """ev: [PF_CTAS, PF_SLOTS] u64 of one prefill launch (slots: 0 entry, 1
+    ready, 2 first S, 3 and 4 the tiles' last P.V, 5 exit, 7 SM id)."""
+    ev = ev.astype(np.int64)
+    ran = ev[:, 0] > 0
+    e = ev[ran]
+    t0 = e[:, 0].min()
+    us = lambda c: (e[:, c] - t0) / 1000.0
+    entry, ready, first_s, exit_ = us(0), us(1), us(2), us(5)
+    last_pv = np.maximum(us(3), np.where(e[:, 4] > 0, us(4), 0.0))
+    sm = e[:, PF_SLOTS - 1]
+    span = float(exit_.max())
+    gaps, windows, per_sm, last_exit = [], 0.0, [], []
+    for s in np.unique(sm):
+        idx = np.where(sm == s)[0]
+        o = idx[np.argsort(entry[idx])]
+        gaps += list(entry[o[1:]] - exit_[o[:-1]])
+        windows += float(np.sum(last_pv[o] - first_s[o]))
+        per_sm.append(len(o))
+        last_exit.append(float(exit_[o].max()))
+    sms = len(per_sm)
+    return {"ctas": int(ran.sum()), "sms": sms, "span_us": round(span, 2), "life_us": _pct(exit_ - entry),
+            "entry_to_ready_us": _pct(ready - entry), "entry_to_first_S_us": _pct(first_s - entry),
+            "last_PV_to_exit_us": _pct(exit_ - last_pv), "exit_to_next_entry_us": _pct(gaps),
+            "ctas_per_sm": _pct(per_sm), "first_S_to_last_PV_share": round(windows / (sms * span), 4) if sms else 0.0,
+            "sm_last_exit_us": _pct(last_exit)}
+
+
+def run_prefill(repeats: int = 3) -> list:
+    import torch
+
+    from . import _binding as b
+    from .build import TIMELINE_LIB
+    from .workloads import custom_case
+
+    if not os.path.exists(TIMELINE_LIB):
+        raise RuntimeError("libpa_timeline.so is not built (python -m paged_kv_cache_355_b200.build)")
+    lib = _load(TIMELINE_LIB)
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    B, Hq, Hkv, D, bs, L, n = PREFILL_SHAPE
+    case = custom_case([L] * B, Hq, Hkv, D, bs, torch.bfloat16, seed=2001, device=dev)
+    qs = torch.arange(0, (B + 1) * n, n, dtype=torch.int32, device=dev)
+    g = torch.Generator(device=dev).manual_seed(2002)
+    q = torch.randn(B * n, Hq, D, generator=g, device=dev).to(torch.bfloat16)
+    out = torch.empty(B * n, Hq, D, dtype=torch.bfloat16, device=dev)
+    bt, lens = case.block_tables.to(dev), case.lengths.to(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    saved = b._lib
+    b._lib = lib
+    try:
+        fn = lambda: b.pa_paged_attention_prefill(q, case.k_pool, case.v_pool, bt, lens, qs, n, case.scale, out)
+        results = []
+        for _ in range(repeats):
+            for _ in range(3):
+                flush.zero_()
+                fn()
+            torch.cuda.synchronize()
+            if lib.pa_timeline_clear_prefill() != 0:
+                raise RuntimeError("pa_timeline_clear_prefill failed")
+            flush.zero_()
+            torch.cuda.synchronize()
+            fn()
+            torch.cuda.synchronize()
+            if b.pa_read_error_flag() != 0:
+                raise RuntimeError("the prefill call flagged an error")
+            ev = np.zeros(PF_CTAS * PF_SLOTS, np.uint64)
+            if lib.pa_timeline_read_prefill(ev.ctypes.data, ev.nbytes):
+                raise RuntimeError("pa_timeline_read_prefill failed")
+            results.append(_prefill_summary(ev.reshape(PF_CTAS, PF_SLOTS)))
+    finally:
+        b._lib = saved
+    return results
 
 
 def launch_order(lengths: np.ndarray, max_len: int, max_batch: int = 2048) -> np.ndarray:
@@ -204,6 +294,19 @@ def main() -> None:
     ap.add_argument("--repeats", type=int, default=3)
     ap.add_argument("--json", default=None, help="also write the summaries here")
     a = ap.parse_args()
+    if a.workload == "prefill":
+        res = run_prefill(a.repeats)
+        for i, r in enumerate(res):
+            print(f"== prefill, launch {i}: span {r['span_us']} us, {r['ctas']} CTAs on {r['sms']} SMs "
+                  f"(p0 p10 p50 p90 p100, us)")
+            for k in ("life_us", "entry_to_ready_us", "entry_to_first_S_us", "last_PV_to_exit_us",
+                      "exit_to_next_entry_us", "ctas_per_sm", "sm_last_exit_us"):
+                print(f"  {k:24s} {r[k]}")
+            print(f"  first S to last P.V, share of SM time: {r['first_S_to_last_PV_share']}")
+        if a.json:
+            with open(a.json, "w") as f:
+                json.dump(res, f, indent=1)
+        return
     res = run(a.workload, a.repeats)
     for i, r in enumerate(res):
         print(f"== {a.workload}, replay {i}: call end {r['call_end_us']} us, CTAs {r['ctas']}")

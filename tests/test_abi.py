@@ -37,14 +37,15 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_timeline_build_exports_the_same_abi_and_its_readers(lib):
-    """libpa_timeline.so (the decode kernels with per-CTA stamps) exports
-    everything include/pa.h declares plus include/pa_timeline.h's readers;
-    libpa.so has none of the readers."""
+    """libpa_timeline.so (the decode and prefill kernels with per-CTA stamps)
+    exports everything include/pa.h declares plus include/pa_timeline.h's
+    readers; libpa.so has none of the readers."""
     from paged_kv_cache_355_b200 import build
 
     tl = ctypes.CDLL(build.TIMELINE_LIB)
     readers = declared_entry_points(os.path.join(ROOT, "include", "pa_timeline.h"))
-    assert readers == ["pa_timeline_clear", "pa_timeline_read"]
+    assert sorted(readers) == ["pa_timeline_clear", "pa_timeline_clear_prefill", "pa_timeline_read",
+                               "pa_timeline_read_prefill"]
     missing = [n for n in declared_entry_points() + readers if not hasattr(tl, n)]
     assert not missing, missing
     assert not any(hasattr(lib, n) for n in readers)

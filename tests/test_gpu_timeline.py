@@ -86,3 +86,48 @@ def test_timeline_build_gives_the_same_bits_and_ordered_stamps():
     assert len(t) == 3 * Hkv
     assert (t[:, 5] <= t[:, 4]).all() and (t[:, 4] <= t[:, 0]).all() and (t[:, 0] <= t[:, 1]).all()
     assert (t[:, 1] <= t[:, 3]).all()
+
+
+def test_prefill_timeline_gives_the_same_bits_and_ordered_stamps():
+    """The prefill kernel of the timeline build: bit-identical output, and
+    for every CTA with query rows entry <= ready <= first S <= tile 0's last
+    P.V <= exit (tile 1's last P.V before the exit when it has rows)."""
+    import paged_kv_cache_355_b200._binding as b
+    from paged_kv_cache_355_b200.build import TIMELINE_LIB
+    from paged_kv_cache_355_b200.timeline import PF_CTAS, PF_SLOTS, _load
+    from paged_kv_cache_355_b200.workloads import custom_case
+
+    lengths, news = [700, 300, 129, 64], [700, 170, 1, 64]
+    case = custom_case(lengths, 32, 8, 128, 16, torch.bfloat16, seed=191)
+    qs = torch.tensor(np.concatenate([[0], np.cumsum(news)]), dtype=torch.int32, device="cuda")
+    g = torch.Generator().manual_seed(192)
+    q = torch.randn(int(sum(news)), 32, 128, generator=g).to(torch.bfloat16).cuda()
+    args = (q, case.k_pool.cuda(), case.v_pool.cuda(), case.block_tables.cuda(), case.lengths.cuda(), qs, max(news),
+            case.scale)
+    ref = torch.full((q.shape[0], 32, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    b.pa_paged_attention_prefill(*args, ref)
+    torch.cuda.synchronize()
+    tl = _load(TIMELINE_LIB)
+    saved = b._lib
+    b._lib = tl
+    try:
+        assert tl.pa_timeline_clear_prefill() == 0
+        out = torch.full_like(ref, float("nan"))
+        b.pa_paged_attention_prefill(*args, out)
+        torch.cuda.synchronize()
+        assert b.pa_read_error_flag() == 0
+        ev = np.zeros(PF_CTAS * PF_SLOTS, np.uint64)
+        assert tl.pa_timeline_read_prefill(ev.ctypes.data, ev.nbytes) == 0
+        assert tl.pa_timeline_read_prefill(ev.ctypes.data, ev.nbytes + 8) != 0
+    finally:
+        b._lib = saved
+    assert torch.equal(out, ref)
+    e = ev.reshape(PF_CTAS, PF_SLOTS).astype(np.int64)
+    e = e[e[:, 0] > 0]
+    # CTAs with rows: pairs of 32-token tiles (G = 4) per (sequence, kv head)
+    assert len(e) == 8 * sum(-(-n // 64) for n in news)
+    assert (e[:, 0] <= e[:, 1]).all() and (e[:, 1] <= e[:, 2]).all() and (e[:, 2] <= e[:, 3]).all()
+    assert (e[:, 3] <= e[:, 5]).all()
+    two = e[:, 4] > 0
+    assert (e[two, 4] <= e[two, 5]).all() and two.any() and (~two).any()
+    assert (e[:, PF_SLOTS - 1] < torch.cuda.get_device_properties(0).multi_processor_count).all()

@@ -81,3 +81,37 @@ def test_summary_tile_chain_medians():
     c = chain[0]
     assert c["period"] == 3.0 and c["scores_to_P"] == 0.8 and c["P_to_PV"] == 0.2
     assert c["Vreq_to_PV"] == 2.0 and c["Kreq_to_S"] == 1.0 and c["S_to_scores"] == 0.5
+
+
+def test_prefill_summary_on_synthetic_stamps():
+    from paged_kv_cache_355_b200.timeline import PF_CTAS, PF_SLOTS, _prefill_summary
+
+    ev = np.zeros((PF_CTAS, PF_SLOTS), np.uint64)
+    base = 5_000_000
+    # two SMs, two CTAs each: entry, ready +0.5, first S +2, last P.V (tile 0,
+    # tile 1) at +20/+21, exit +23; the second CTA on an SM enters 1.5 us
+    # after the first exits
+    for i, (sm, start) in enumerate([(0, 0.0), (1, 0.0), (0, 24.5), (1, 24.5)]):
+        t = base + int(start * 1000)
+        ev[i, 0], ev[i, 1], ev[i, 2] = t, t + 500, t + 2000
+        ev[i, 3], ev[i, 4], ev[i, 5] = t + 20000, t + 21000, t + 23000
+        ev[i, PF_SLOTS - 1] = sm
+    r = _prefill_summary(ev)
+    assert r["ctas"] == 4 and r["sms"] == 2 and r["span_us"] == 47.5
+    assert r["life_us"] == [23.0] * 5 and r["entry_to_first_S_us"] == [2.0] * 5
+    assert r["last_PV_to_exit_us"] == [2.0] * 5 and r["exit_to_next_entry_us"] == [1.5] * 5
+    assert r["ctas_per_sm"] == [2.0] * 5 and r["sm_last_exit_us"] == [47.5] * 5
+    assert abs(r["first_S_to_last_PV_share"] - (4 * 19.0) / (2 * 47.5)) < 1e-4
+
+
+def test_prefill_timeline_runs_the_benchmarked_workload():
+    import importlib.util
+    import os
+
+    from paged_kv_cache_355_b200.timeline import PREFILL_SHAPE
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    spec = importlib.util.spec_from_file_location("bench_for_timeline", os.path.join(root, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    assert PREFILL_SHAPE == bench.PREFILL_SHAPE
